@@ -1,0 +1,11 @@
+"""Float64 CPU oracle (test infrastructure only; see ``la2_oracle``)."""
+
+from .la2_oracle import (  # noqa: F401
+    backward,
+    backward_rows,
+    blocked_forward,
+    forward,
+    forward_rows,
+    recurrent_forward,
+    relative_frobenius,
+)

@@ -1,0 +1,243 @@
+"""CPU float64 oracle for Lightning Attention-2 causal linear attention.
+
+TEST INFRASTRUCTURE ONLY. Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import or run
+this module. The CUDA library never calls it, and it shares no code, table or
+helper with the CUDA path.
+
+Source of every formula: the news article "Lightning Attention-2 新一代注意力机制"
+(youleyou.com), section "Lightning Attention-2简介":
+
+* point 1 (with Fig. 2): with softmax removed, the output is the *left product*
+  ``O = ((Q K^T) ⊙ M) V``; ``M`` is the lower-triangular all-ones mask in the
+  unidirectional (GPT) case and is dropped in the bidirectional case, where
+  associativity gives the *right product* ``O = Q (K^T V)``;
+* point 2 (with Fig. 3): Q, K, V are cut into the same number of blocks; inside a
+  block the masked left product is kept, across blocks the right product is used
+  with a KV state that is accumulated for the next block, and the two partial
+  outputs are added to give ``O_i``;
+* section "Lightning Attention-2速度对比": linear attention converts losslessly
+  to an RNN at inference (one token at a time with a constant-size state).
+
+Readings where the article is silent (each is listed in the design notes):
+
+* ``M`` includes the diagonal (token t attends to itself);
+* no normalisation, no ``1/sqrt(d)`` inside the op, no feature map, no decay;
+* tensors are ``[B, H, N, d]`` (``dv`` for V and O), each (b, h) independent;
+* gradients are those of ``L = <dO, O>`` for the closed form above.
+
+All arithmetic is float64 on the exact (already rounded) input values.
+``forward`` / ``backward`` / ``*_rows`` are the plain definition. ``recurrent_*``
+is the RNN form and ``blocked_forward`` the block algorithm of point 2; those two
+exist to pin the definition (and to check very long sequences where the O(N^2)
+definition is too slow on a CPU), never the other way round.
+
+Parity status: every function here is pinned by ``tests/test_oracle.py``
+(brute force on tiny integer inputs, closed forms, RNN-form equality, block-size
+invariance, associativity, exact directional derivatives, autograd).
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+# Rows of scores held at once by the row-group loops below. It only bounds
+# memory (ROW_GROUP x N float64); every output row is still its own sum.
+ROW_GROUP = 512
+
+
+def _f64(x) -> np.ndarray:
+    """Upcast a torch tensor or array to a float64 numpy array."""
+    try:
+        import torch
+
+        if isinstance(x, torch.Tensor):
+            return x.detach().to("cpu", torch.float64).numpy()
+    except ImportError:  # pragma: no cover - torch is always present here
+        pass
+    return np.asarray(x, dtype=np.float64)
+
+
+def _check(q, k, v):
+    if q.ndim != 4 or k.shape != q.shape or v.shape[:3] != q.shape[:3]:
+        raise ValueError("expected q,k [B,H,N,d] and v [B,H,N,dv]")
+
+
+def forward(q, k, v, causal: bool = True) -> np.ndarray:
+    """Left product ``O = ((Q K^T) ⊙ M) V`` for every (b, h).
+
+    Row t of O is ``sum_{s in mask(t)} (q_t . k_s) v_s`` with ``mask(t) = {0..t}``
+    when ``causal`` and ``{0..N-1}`` otherwise (article, point 1).
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    _check(q, k, v)
+    B, H, N, _ = q.shape
+    out = np.empty(q.shape[:3] + (v.shape[3],), dtype=np.float64)
+    for b in range(B):
+        for h in range(H):
+            K, V = k[b, h], v[b, h]
+            for r0 in range(0, N, ROW_GROUP):
+                r1 = min(N, r0 + ROW_GROUP)
+                S = q[b, h, r0:r1] @ K.T  # scores q_t . k_s, shape [rows, N]
+                if causal:
+                    t = np.arange(r0, r1)[:, None]
+                    s = np.arange(N)[None, :]
+                    S = np.where(s <= t, S, 0.0)  # M: lower-triangular ones, diagonal kept
+                out[b, h, r0:r1] = S @ V
+    return out
+
+
+def forward_rows(q, k, v, rows, causal: bool = True) -> np.ndarray:
+    """The same definition evaluated only at the given output rows.
+
+    Returns ``[B, H, len(rows), dv]``. Used at sizes where the full O(N^2)
+    product is too slow on a CPU.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    _check(q, k, v)
+    rows = np.asarray(rows, dtype=np.int64)
+    B, H, N, _ = q.shape
+    out = np.empty((B, H, len(rows), v.shape[3]), dtype=np.float64)
+    group = max(1, min(64, (1 << 27) // max(1, N * 8)))
+    for b in range(B):
+        for h in range(H):
+            K, V = k[b, h], v[b, h]
+            for g0 in range(0, len(rows), group):
+                rr = rows[g0:g0 + group]
+                S = q[b, h, rr] @ K.T
+                if causal:
+                    S = np.where(np.arange(N)[None, :] <= rr[:, None], S, 0.0)
+                out[b, h, g0:g0 + len(rr)] = S @ V
+    return out
+
+
+def backward(q, k, v, do, causal: bool = True):
+    """Closed-form gradients of ``L = <dO, O>`` with ``O = ((Q K^T) ⊙ M) V``.
+
+    With ``P = (Q K^T) ⊙ M`` and ``dP = (dO V^T) ⊙ M``:
+    ``dQ = dP K``, ``dK = dP^T Q``, ``dV = P^T dO``.
+    Returns ``(dq, dk, dv)`` as float64 arrays.
+    """
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    _check(q, k, v)
+    B, H, N, _ = q.shape
+    dq = np.empty_like(q)
+    dk = np.empty_like(k)
+    dvv = np.empty_like(v)
+    for b in range(B):
+        for h in range(H):
+            Q, K, V, dO = q[b, h], k[b, h], v[b, h], do[b, h]
+            dk_acc = np.zeros_like(K)
+            dv_acc = np.zeros_like(V)
+            for r0 in range(0, N, ROW_GROUP):
+                r1 = min(N, r0 + ROW_GROUP)
+                P = Q[r0:r1] @ K.T
+                dP = dO[r0:r1] @ V.T
+                if causal:
+                    keep = np.arange(N)[None, :] <= np.arange(r0, r1)[:, None]
+                    P = np.where(keep, P, 0.0)
+                    dP = np.where(keep, dP, 0.0)
+                dq[b, h, r0:r1] = dP @ K
+                dk_acc += dP.T @ Q[r0:r1]
+                dv_acc += P.T @ dO[r0:r1]
+            dk[b, h] = dk_acc
+            dvv[b, h] = dv_acc
+    return dq, dk, dvv
+
+
+def backward_rows(q, k, v, do, rows, causal: bool = True):
+    """Rows of the closed-form gradients, one output row at a time.
+
+    ``dq_t = sum_{s<=t} (do_t . v_s) k_s``;
+    ``dk_s = sum_{t>=s} (do_t . v_s) q_t``;
+    ``dv_s = sum_{t>=s} (q_t . k_s) do_t`` (all s, t for the non-causal case).
+    Returns three ``[B, H, len(rows), .]`` arrays.
+    """
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    rows = np.asarray(rows, dtype=np.int64)
+    B, H, N, d = q.shape
+    dvd = v.shape[3]
+    dq = np.empty((B, H, len(rows), d))
+    dk = np.empty((B, H, len(rows), d))
+    dvv = np.empty((B, H, len(rows), dvd))
+    group = max(1, min(64, (1 << 27) // max(1, N * 8)))
+    cols = np.arange(N)[None, :]
+    for b in range(B):
+        for h in range(H):
+            Q, K, V, dO = q[b, h], k[b, h], v[b, h], do[b, h]
+            for g0 in range(0, len(rows), group):
+                rr = rows[g0:g0 + group]
+                sl = slice(g0, g0 + len(rr))
+                a = dO[rr] @ V.T  # (do_t . v_s) for t in rr
+                if causal:
+                    a = np.where(cols <= rr[:, None], a, 0.0)
+                dq[b, h, sl] = a @ K
+                c = V[rr] @ dO.T  # (do_t . v_s) for s in rr, all t
+                e = K[rr] @ Q.T   # (q_t . k_s) for s in rr, all t
+                if causal:
+                    later = cols >= rr[:, None]
+                    c = np.where(later, c, 0.0)
+                    e = np.where(later, e, 0.0)
+                dk[b, h, sl] = c @ Q
+                dvv[b, h, sl] = e @ dO
+    return dq, dk, dvv
+
+
+def recurrent_forward(q, k, v) -> np.ndarray:
+    """RNN form of the causal op: ``KV_t = KV_{t-1} + k_t^T v_t``, ``o_t = q_t KV_t``.
+
+    The state is d x dv and starts at zero (article, speed section: lossless
+    conversion to an RNN). One token at a time; a pin for ``forward`` only.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    _check(q, k, v)
+    B, H, N, d = q.shape
+    out = np.empty(q.shape[:3] + (v.shape[3],))
+    for b in range(B):
+        for h in range(H):
+            kv = np.zeros((d, v.shape[3]))
+            for t in range(N):
+                kv += np.outer(k[b, h, t], v[b, h, t])
+                out[b, h, t] = q[b, h, t] @ kv
+    return out
+
+
+def blocked_forward(q, k, v, block: int, causal: bool = True) -> np.ndarray:
+    """The block algorithm of the article's point 2, in float64.
+
+    Blocks of ``block`` rows. For block i: intra part ``((Q_i K_i^T) ⊙ M_B) V_i``
+    (left product), inter part ``Q_i KV`` with ``KV = sum_{j<i} K_j^T V_j`` (right
+    product); the two are added to give ``O_i``, then ``KV += K_i^T V_i``.
+    Without the mask it is ``Q (K^T V)``. A cross-check of ``forward`` (block-size
+    invariance) and the full-tensor reference for very long sequences.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    _check(q, k, v)
+    B, H, N, d = q.shape
+    dvd = v.shape[3]
+    out = np.empty(q.shape[:3] + (dvd,))
+    for b in range(B):
+        for h in range(H):
+            Q, K, V = q[b, h], k[b, h], v[b, h]
+            if not causal:
+                out[b, h] = Q @ (K.T @ V)
+                continue
+            kv = np.zeros((d, dvd))
+            for i0 in range(0, N, block):
+                i1 = min(N, i0 + block)
+                S = Q[i0:i1] @ K[i0:i1].T
+                S = np.tril(S)  # M_B, diagonal kept
+                out[b, h, i0:i1] = S @ V[i0:i1] + Q[i0:i1] @ kv
+                kv += K[i0:i1].T @ V[i0:i1]
+    return out
+
+
+def relative_frobenius(x, ref) -> float:
+    """``||x - ref||_F / ||ref||_F`` in float64 (0 if both are zero)."""
+    x = _f64(x)
+    ref = _f64(ref)
+    num = float(np.linalg.norm((x - ref).ravel()))
+    den = float(np.linalg.norm(ref.ravel()))
+    if den == 0.0:
+        return 0.0 if num == 0.0 else float("inf")
+    return num / den
