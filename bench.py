@@ -1,0 +1,457 @@
+#!/usr/bin/env python
+"""Causal linear-attention forward throughput on B200 (Lightning Attention-2).
+
+One step = one causal forward pass O = ((Q K^T) ⊙ M) V over one batch of the
+workload (default: B=4, H=16, N=2048, d=dv=128, block 64, bf16 in/out, fp32
+accumulation and state), through libla2's C ABI. Prints one JSON line.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                  [--impl reference] [--sweep]
+
+N > 1 is launched with torch.distributed.run: every rank runs the same
+workload on its own GPU (independent (b, h) sequences, no data-path
+collective; weak scaling) and rank 0 reports the aggregate.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+L2_BYTES = 126 * 1024 * 1024
+METRIC = "causal linear-attn fwd tokens/s (B·H·N/s), TFLOP/s, % of roofline, 1 B200"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="bf16_b4h16_n2k")
+    ap.add_argument("--block", type=int, default=0, help="override the workload's block size")
+    ap.add_argument("--N", type=int, default=0, help="override the sequence length")
+    ap.add_argument("--impl", default="la2", choices=["la2", "reference"])
+    ap.add_argument("--sweep", action="store_true",
+                    help="also print one line per sequence-length sweep point and the 512K case")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ helpers
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p["bf16_tflops_sustained"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+def source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "linear_attention_la2_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel, workload):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    e = rec.get(f"{kernel}/{workload}")
+    if not e or e.get("source_hash") != source_hash():
+        return None
+    return e.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.t:
+            self.t.join(timeout=2)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def workload_from_args(args):
+    from linear_attention_la2_b200 import inputs as I
+
+    if args.workload in I.WORKLOADS:
+        w = I.WORKLOADS[args.workload]
+    elif args.workload.startswith("bf16_sweep_n"):
+        n, b = args.workload[len("bf16_sweep_n"):].split("_b")
+        w = I.sweep_workload(int(n), int(b))
+    else:
+        raise SystemExit(f"unknown workload {args.workload}")
+    if args.block or args.N:
+        from dataclasses import replace
+
+        w = replace(w, block=args.block or w.block, N=args.N or w.N,
+                    name=f"{w.name}_N{args.N or w.N}_b{args.block or w.block}")
+    return w
+
+
+def flops_per_token(w):
+    return 2 * w.block * (w.d + w.dv) + 4 * w.d * w.dv
+
+
+def bytes_per_token(w):
+    es = 2 if w.dtype == "bf16" else 4
+    return (2 * w.d + 2 * w.dv) * es
+
+
+# -------------------------------------------------------------- CPU oracle
+
+
+def cpu_oracle_rate(w, budget_s=10.0, max_heads=None):
+    """Time the float64 oracle (as it stands) on whole (b, h) sequences of the
+    workload until ~budget_s of CPU work; returns (tokens/s, sample text, cores)."""
+    import torch
+
+    import oracle
+    from linear_attention_la2_b200 import inputs as I
+
+    try:
+        from threadpoolctl import threadpool_info
+
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:  # pragma: no cover
+        cores = os.cpu_count() or 1
+    g = torch.Generator().manual_seed(w.seed)
+    scale = 1.0 / math.sqrt(w.d)
+    heads, tokens, elapsed = 0, 0, 0.0
+    limit = max_heads or w.B * w.H
+    while heads == 0 or (elapsed < budget_s and heads < limit):
+        q = (torch.randn((1, 1, w.N, w.d), generator=g) * scale).to(w.torch_dtype)
+        k = (torch.randn((1, 1, w.N, w.d), generator=g) * scale).to(w.torch_dtype)
+        v = (torch.randn((1, 1, w.N, w.dv), generator=g) * scale).to(w.torch_dtype)
+        t0 = time.perf_counter()
+        oracle.forward(q, k, v, True)
+        elapsed += time.perf_counter() - t0
+        heads += 1
+        tokens += w.N
+    sample = (f"{heads} whole (b,h) sequences of N={w.N} (of {w.B * w.H}), float64 left product "
+              f"O=((QK^T)⊙M)V, {elapsed:.1f} s")
+    return tokens / elapsed, sample, cores
+
+
+def run_reference(args):
+    """--impl reference: the oracle on the host cores, same metric and config."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = workload_from_args(args)
+    # one step = one whole (b, h) sequence of the workload
+    rate_steps = []
+    for i in range(args.warmup + args.steps):
+        r, sample, cores = cpu_oracle_rate(w, budget_s=0.0, max_heads=1)
+        if i >= args.warmup:
+            rate_steps.append(w.N / r)
+    total = sum(rate_steps)
+    value = args.steps * w.N / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(w),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"each step: one (b,h) sequence of N={w.N} of the workload, "
+                                   "float64 left product on host cores"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def config_of(w):
+    return {"workload": f"{w.name}: causal forward B={w.B} H={w.H} N={w.N} d={w.d} dv={w.dv} "
+                        f"block={w.block} {w.dtype}", "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+            "dv": w.dv, "block": w.block, "causal": True}
+
+
+# ------------------------------------------------------------------- GPU
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    from linear_attention_la2_b200 import inputs as I
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    from linear_attention_la2_b200 import la2
+
+    w = workload_from_args(args)
+    hbm, tf_burst, tf_sust, peak_kind = peaks()
+
+    line = bench_workload(args, w, dev, la2, world, rank, local, hbm, peak_kind, main=True)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if args.sweep:
+        for N in I.SWEEP_N:
+            for b in I.SWEEP_BLOCKS:
+                sw = I.sweep_workload(N, b)
+                ln = bench_workload(args, sw, dev, la2, world, rank, local, hbm, peak_kind, main=False)
+                if rank == 0:
+                    print(json.dumps(ln), flush=True)
+        lw = I.WORKLOADS["bf16_long_512k"]
+        ln = bench_workload(args, lw, dev, la2, world, rank, local, hbm, peak_kind, main=False)
+        if rank == 0:
+            print(json.dumps(ln), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def _max_over_ranks(x, world, dev):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def bench_workload(args, w, dev, la2, world, rank, local, hbm, peak_kind, main):
+    import torch
+
+    from linear_attention_la2_b200 import inputs as I
+
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    set_bytes = w.tokens * bytes_per_token(w)
+    nsets = max(1, math.ceil(3 * L2_BYTES / set_bytes)) if set_bytes < 3 * L2_BYTES else 1
+    nsets = min(nsets, 8)
+    base = I.make_inputs(w, device="cpu")
+    sets = []
+    for s in range(nsets):
+        q = base["q"].to(dev)
+        k = base["k"].to(dev)
+        v = base["v"].to(dev)
+        if s > 0:  # distinct buffers, same values
+            pass
+        o = torch.empty((w.B, w.H, w.N, w.dv), dtype=w.torch_dtype, device=dev)
+        sets.append((q, k, v, o))
+    dt = la2.LA2_BF16 if w.dtype == "bf16" else la2.LA2_F32
+    ws_bytes = la2.workspace_bytes(w.B, w.H, w.N, w.d, w.dv, True, w.block, dt, False)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+    st = la2._stream_handle(stream)
+
+    def step(i):
+        q, k, v, o = sets[i % nsets]
+        rc = la2.la2_forward(la2._ptr(q), la2._ptr(k), la2._ptr(v), la2._ptr(o), w.B, w.H, w.N, w.d,
+                             w.dv, 1, w.block, dt, la2._ptr(ws), ws_bytes, st)
+        if rc != 0:
+            raise la2.La2Error(rc)
+
+    for i in range(args.warmup):
+        step(i)
+    la2.check(stream)
+
+    sampler = ClockSampler(local) if main else None
+    la2.la2_profile_enable(1)
+    _barrier(world)
+    torch.cuda.synchronize(dev)
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop() if sampler else None
+    _barrier(world)
+    la2.la2_profile_enable(0)
+    la2.check(stream)
+    ms = e0.elapsed_time(e1)
+    ms_max = _max_over_ranks(ms, world, dev)
+
+    per_kernel = {}
+    launches = 0
+    for kid in range(la2.la2_profile_num_kernels()):
+        n, kms = la2.la2_profile_collect(kid)
+        if n:
+            per_kernel[la2.la2_profile_kernel_name(kid)] = {"launches": n, "ms": kms}
+            launches += n
+    dom = max(per_kernel, key=lambda k: per_kernel[k]["ms"]) if per_kernel else None
+
+    tokens = w.tokens * args.steps * world
+    value = tokens / (ms_max / 1e3)
+    tflops = flops_per_token(w) * tokens / (ms_max / 1e3) / 1e12
+    roofline = None
+    if dom:
+        avg_ms = per_kernel[dom]["ms"] / per_kernel[dom]["launches"]
+        alg_bytes = w.tokens * bytes_per_token(w)
+        achieved = alg_bytes / (avg_ms / 1e3) / 1e9
+        roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                    "frac": achieved / hbm, "traffic": recorded_traffic(dom, w.name),
+                    "kernel": dom, "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)"
+                    if peak_kind == "measured" else "fallback 6.65 TB/s"}
+    step_frac = (w.tokens * bytes_per_token(w) * args.steps * world / (ms_max / 1e3) / 1e9) / (hbm * world)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
+        "data": "synthetic", "config": dict(config_of(w), l2=(
+            f"{nsets} rotating input sets of {set_bytes / 1e6:.0f} MB (> L2 126 MB)" if nsets > 1
+            else f"inputs {set_bytes / 1e6:.0f} MB > L2"), parallelism=f"dp{world} (independent "
+            "(b,h) sequences per rank)"),
+        "tflops": tflops, "step_roofline_frac": step_frac, "roofline": roofline,
+        "gpu_launches": launches, "kernels": per_kernel,
+    }
+    if clocks:
+        line["clocks"] = clocks
+    if main and not args.no_e2e:
+        line["e2e"] = e2e_measure(args, w, dev, la2, world, base, ws, ws_bytes, dt)
+    if main and rank == 0 and world == 1 and not args.no_cpu_baseline:
+        r, sample, cores = cpu_oracle_rate(w, budget_s=10.0)
+        line["cpu_baseline"] = {"value": r, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                "sample": sample}
+    return line
+
+
+def e2e_measure(args, w, dev, la2, world, base, ws, ws_bytes, dt):
+    """Same metric through the public binding with host buffers: every step copies
+    Q, K, V from pinned host memory, runs the forward and reads O back."""
+    import torch
+
+    stream = torch.cuda.current_stream(dev)
+    hq, hk, hv = (base[n].pin_memory() for n in "qkv")
+    ho = torch.empty((w.B, w.H, w.N, w.dv), dtype=w.torch_dtype).pin_memory()
+    dq = torch.empty_like(hq, device=dev)
+    dk = torch.empty_like(hk, device=dev)
+    dvv = torch.empty_like(hv, device=dev)
+    do = torch.empty_like(ho, device=dev)
+
+    def step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dvv.copy_(hv, non_blocking=True)
+        la2.forward(dq, dk, dvv, causal=True, block=w.block, out=do, workspace=ws if ws_bytes else None)
+        ho.copy_(do, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        step()
+    _barrier(world)
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = _max_over_ranks(e0.elapsed_time(e1), world, dev)
+    h2d = (hq.numel() + hk.numel() + hv.numel()) * hq.element_size()
+    d2h = ho.numel() * ho.element_size()
+    return {"value": w.tokens * args.steps * world / (ms / 1e3), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,161 @@
+/*
+ * la2.h - C ABI of libla2.so: Lightning Attention-2 causal linear attention
+ * on NVIDIA B200 (sm_100a).
+ *
+ * The operation (article "Lightning Attention-2 新一代注意力机制", section
+ * "Lightning Attention-2简介", point 1 and Fig. 2):
+ *
+ *     O = ((Q K^T) ⊙ M) V
+ *
+ * with no softmax, M the lower-triangular all-ones mask (diagonal included)
+ * when causal = 1, and no mask when causal = 0, in which case the result is
+ * the right product O = Q (K^T V). Point 2 (Fig. 3) gives the computation the
+ * library follows: each sequence is cut into blocks of `block` rows; inside a
+ * block the masked left product is used, across blocks the right product
+ * Q_i * KV with a running fp32 state KV += K_i^T V_i.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Tensors are dense, contiguous, row-major [B, H, N, d] (q, k, dq, dk) and
+ *    [B, H, N, dv] (v, o, dout, dv-gradient). Each (b, h) sequence is
+ *    independent. Element type is given by `dt` for every tensor of a call.
+ *  - All tensor pointers are DEVICE pointers owned by the caller, 16-byte
+ *    aligned. Outputs are overwritten (never accumulated into) and must not
+ *    overlap any input. The library allocates no device memory on the call
+ *    path: scratch is the caller's `workspace` (256-byte aligned).
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream). The return value covers argument validation and
+ *    launch errors only; errors raised later on the device are reported by
+ *    la2_check().
+ *  - B, H or N equal to 0 is an empty problem: LA2_OK, nothing is launched,
+ *    pointers may then be NULL. Negative sizes, d or dv < 1, causal not in
+ *    {0, 1}, an unknown dtype, a NULL or misaligned pointer, or outputs
+ *    overlapping inputs give LA2_ERR_INVALID_ARG.
+ *  - Supported shapes. LA2_BF16: d, dv in {64, 128}, block in {64, 128}
+ *    (tensor-core path, fp32 accumulation and fp32 state). LA2_F32: any
+ *    1 <= d, dv <= 128 and block in {16, 32, 64, 128} whose tiles fit in
+ *    shared memory (fp32 CUDA-core path). Anything else gives
+ *    LA2_ERR_UNSUPPORTED.
+ *  - `block` is the algorithm's block size Bk. N need not be a multiple of
+ *    it: the ragged last block is zero-padded on load and not stored.
+ *  - Gradients are those of L = <dO, O>; backward needs no saved forward
+ *    activations (states are recomputed).
+ */
+#ifndef LA2_H
+#define LA2_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LA2_API __attribute__((visibility("default")))
+#else
+#define LA2_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *la2_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  LA2_OK = 0,
+  LA2_ERR_INVALID_ARG = 1, /* bad pointer, size, flag or alignment            */
+  LA2_ERR_UNSUPPORTED = 2, /* valid but unsupported dtype/d/dv/block combo    */
+  LA2_ERR_WORKSPACE = 3,   /* workspace NULL or smaller than required         */
+  LA2_ERR_CUDA = 4,        /* a CUDA runtime/driver call or launch failed     */
+  LA2_ERR_TIMEOUT = 5      /* a bounded device-side wait gave up (la2_check)  */
+} la2_status;
+
+typedef enum { LA2_F32 = 0, LA2_BF16 = 1 } la2_dtype;
+
+/*
+ * Bytes of workspace a la2_forward (is_backward = 0) or la2_backward
+ * (is_backward = 1) call with these arguments needs on the CURRENT device.
+ * 0 means no workspace is needed. Returns (size_t)-1 for arguments the call
+ * would reject. The size depends on the chunk plan (see la2_set_chunk_len) and
+ * on the device's SM count.
+ */
+LA2_API size_t la2_workspace_size(int64_t B, int64_t H, int64_t N, int64_t d, int64_t dv,
+                          int causal, int block, la2_dtype dt, int is_backward);
+
+/*
+ * Forward: o = ((q k^T) ⊙ M) v (causal = 1) or q (k^T v) (causal = 0).
+ * Article section "Lightning Attention-2简介", points 1-3 (Fig. 2, Fig. 3).
+ * q, k: [B,H,N,d]; v, o: [B,H,N,dv]; all of type dt. fp32 accumulation.
+ */
+LA2_API la2_status la2_forward(const void *q, const void *k, const void *v, void *o,
+                       int64_t B, int64_t H, int64_t N, int64_t d, int64_t dv,
+                       int causal, int block, la2_dtype dt,
+                       void *workspace, size_t workspace_bytes, la2_stream_t stream);
+
+/*
+ * Backward of L = <dout, o> for the same op (the article names its Algorithm 2
+ * but does not print it; the gradients are those of the closed form above):
+ *   dq = ((dout v^T) ⊙ M) k,  dk = ((dout v^T) ⊙ M)^T q,  dvv = ((q k^T) ⊙ M)^T dout.
+ * q, k, dq, dk: [B,H,N,d]; v, dout, dvv: [B,H,N,dv]. `dout` is the upstream
+ * gradient dO; `dvv` receives dV (named so to differ from the size dv).
+ */
+LA2_API la2_status la2_backward(const void *q, const void *k, const void *v, const void *dout,
+                        void *dq, void *dk, void *dvv,
+                        int64_t B, int64_t H, int64_t N, int64_t d, int64_t dv,
+                        int causal, int block, la2_dtype dt,
+                        void *workspace, size_t workspace_bytes, la2_stream_t stream);
+
+/*
+ * Synchronises `stream`, then reports and clears the device-side error word
+ * that kernels set when a bounded wait gives up (LA2_ERR_TIMEOUT), or
+ * LA2_ERR_CUDA if the stream holds a CUDA error. LA2_OK otherwise.
+ */
+LA2_API la2_status la2_check(la2_stream_t stream);
+
+/* Static, human-readable name of a status code. */
+LA2_API const char *la2_status_string(la2_status s);
+
+/*
+ * Chunk plan. Sequences with few (b, h) pairs are split into chunks of
+ * `chunk_len` rows that run in parallel from a prefix of per-chunk KV states
+ * (a sum, so any split gives the same result up to fp32 rounding order).
+ * 0 (the default) lets the library choose from B*H, N and the SM count; a
+ * positive value is rounded up to a multiple of `block`. Process-wide; it
+ * changes la2_workspace_size for later calls. Returns LA2_ERR_INVALID_ARG
+ * for a negative value.
+ */
+LA2_API la2_status la2_set_chunk_len(int64_t chunk_len);
+
+/*
+ * Number of chunks per (b, h) sequence the next call with these arguments
+ * uses (1 = no split). -1 for arguments the call would reject.
+ */
+LA2_API int64_t la2_num_chunks(int64_t B, int64_t H, int64_t N, int block, la2_dtype dt);
+
+/*
+ * Upper bound, in spin iterations, of every device-side wait (mbarrier or
+ * flag). When a wait exceeds it the kernel records LA2_ERR_TIMEOUT in the
+ * device error word, stops its work and returns; la2_check() reports it.
+ * 0 restores the default (large enough to be reached only by a fault).
+ */
+LA2_API la2_status la2_set_spin_limit(int64_t iterations);
+
+/*
+ * Per-kernel launch timing, for benchmarks. While enabled, every kernel the
+ * library launches is bracketed by a pair of CUDA events on its stream.
+ * la2_profile_collect() synchronises those events and returns, for kernel id
+ * `kernel`, the number of launches and their summed device time in ms since
+ * the last la2_profile_enable(1). Ids run from 0 to la2_profile_num_kernels()-1
+ * and la2_profile_kernel_name() names them. Not thread-safe.
+ */
+LA2_API la2_status la2_profile_enable(int on);
+LA2_API int la2_profile_num_kernels(void);
+LA2_API const char *la2_profile_kernel_name(int kernel);
+LA2_API la2_status la2_profile_collect(int kernel, int64_t *launches, double *total_ms);
+
+/* Library version, (major << 16) | minor. */
+LA2_API int la2_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LA2_H */

@@ -1,0 +1,422 @@
+// libla2: host side of the C ABI declared in include/la2.h.
+//
+// Argument validation, the chunk plan, workspace carving, kernel launches and
+// the optional per-kernel event timing. Every kernel of the library is in this
+// translation unit (the .cuh files below), so the device error word is one
+// symbol.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "la2.h"
+#include "la2_common.cuh"
+#include "la2_simt.cuh"
+#include "la2_sm100.cuh"
+
+namespace la2 {
+
+// ------------------------------------------------------------------ profiler
+
+enum KernelId : int {
+  K_CHUNK_STATE = 0,
+  K_CHUNK_SCAN,
+  K_FWD_SIMT,
+  K_BWD_DQ_SIMT,
+  K_BWD_DKDV_SIMT,
+  K_FWD_TC,
+  K_STATE_TC,
+  K_BWD_DQ_TC,
+  K_BWD_DKDV_TC,
+  K_COUNT
+};
+
+static const char* kKernelNames[K_COUNT] = {
+    "la2_chunk_state_simt", "la2_chunk_scan",      "la2_fwd_simt",
+    "la2_bwd_dq_simt",      "la2_bwd_dkdv_simt",   "la2_fwd_sm100",
+    "la2_chunk_state_sm100", "la2_bwd_dq_sm100",   "la2_bwd_dkdv_sm100"};
+
+struct EventRecord {
+  int kernel;
+  cudaEvent_t start, stop;
+};
+
+struct Profiler {
+  bool on = false;
+  std::vector<EventRecord> pool;  // events are reused across enable() calls
+  size_t used = 0;
+};
+static Profiler g_prof;
+
+struct LaunchTimer {
+  EventRecord* rec = nullptr;
+  cudaStream_t stream;
+  LaunchTimer(int kernel, cudaStream_t s) : stream(s) {
+    if (!g_prof.on) return;
+    if (g_prof.used == g_prof.pool.size()) {
+      EventRecord r{};
+      if (cudaEventCreate(&r.start) != cudaSuccess || cudaEventCreate(&r.stop) != cudaSuccess) return;
+      g_prof.pool.push_back(r);
+    }
+    rec = &g_prof.pool[g_prof.used++];
+    rec->kernel = kernel;
+    cudaEventRecord(rec->start, stream);
+  }
+  ~LaunchTimer() {
+    if (rec) cudaEventRecord(rec->stop, stream);
+  }
+};
+
+// ------------------------------------------------------------------ settings
+
+static int64_t g_chunk_len = 0;           // 0: automatic
+static int64_t g_spin_limit = 0;          // 0: default
+constexpr int64_t kDefaultSpinLimit = int64_t(1) << 31;
+
+static int64_t spin_limit() { return g_spin_limit > 0 ? g_spin_limit : kDefaultSpinLimit; }
+
+static int device_sm_count() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+  return sms;
+}
+
+// ------------------------------------------------------------------ planning
+
+struct Plan {
+  int64_t L = 0;        // chunk length (rows), multiple of block
+  int64_t C = 1;        // chunks per (b, h)
+  bool tc = false;      // tensor-core (sm_100a) path
+  bool need_states = false;
+  size_t ws_bytes = 0;
+};
+
+static bool is_aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+static bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+// Shape checks shared by every entry point. Returns LA2_OK or an error.
+static la2_status check_shape(int64_t B, int64_t H, int64_t N, int64_t d, int64_t dv, int causal,
+                              int block, la2_dtype dt, bool is_bwd) {
+  if (B < 0 || H < 0 || N < 0 || d < 1 || dv < 1) return LA2_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return LA2_ERR_INVALID_ARG;
+  if (dt != LA2_F32 && dt != LA2_BF16) return LA2_ERR_INVALID_ARG;
+  if (block < 1) return LA2_ERR_INVALID_ARG;
+  // int64 overflow guard on the largest index the kernels form.
+  const double elems = double(B) * double(H) * double(N) * double(std::max(d, dv));
+  if (elems > 9.0e18) return LA2_ERR_INVALID_ARG;
+  if (dt == LA2_BF16) {
+    if ((d != 64 && d != 128) || (dv != 64 && dv != 128)) return LA2_ERR_UNSUPPORTED;
+    if (block != 64 && block != 128) return LA2_ERR_UNSUPPORTED;
+  } else {
+    if (d > 128 || dv > 128) return LA2_ERR_UNSUPPORTED;
+    if (block != 16 && block != 32 && block != 64 && block != 128) return LA2_ERR_UNSUPPORTED;
+  }
+  const size_t smem = is_bwd ? std::max(bwd_dq_simt_smem((int)d, (int)dv, block),
+                                        bwd_dkdv_simt_smem((int)d, (int)dv, block))
+                             : fwd_simt_smem((int)d, (int)dv, block);
+  const bool tc = (dt == LA2_BF16) && sm100_supports(d, dv, block, is_bwd);
+  if (!tc && smem > 227 * 1024) return LA2_ERR_UNSUPPORTED;
+  return LA2_OK;
+}
+
+static Plan make_plan(int64_t B, int64_t H, int64_t N, int64_t d, int64_t dv, int causal, int block,
+                      la2_dtype dt, bool is_bwd, int sms) {
+  Plan p;
+  const int64_t BH = B * H;
+  const int64_t T = (N + block - 1) / block;
+  p.tc = (dt == LA2_BF16) && sm100_supports(d, dv, block, is_bwd);
+  int64_t L;
+  if (g_chunk_len > 0) {
+    L = ((g_chunk_len + block - 1) / block) * block;
+  } else {
+    // Enough (b, h, chunk) units for about two per SM, chunks no shorter than
+    // four blocks so the chunk-state pass stays a small fraction of the work.
+    const int64_t target = 2 * (int64_t)std::max(sms, 1);
+    int64_t C = std::max<int64_t>(1, (target + BH - 1) / std::max<int64_t>(BH, 1));
+    C = std::min<int64_t>(C, std::max<int64_t>(1, T / 4));
+    L = ((T + C - 1) / C) * block;
+  }
+  L = std::max<int64_t>(L, block);
+  p.L = L;
+  p.C = std::max<int64_t>(1, (N + L - 1) / L);
+  p.need_states = (p.C > 1) || !causal;
+  const size_t one = (size_t)BH * (size_t)p.C * (size_t)d * (size_t)dv * sizeof(float);
+  p.ws_bytes = p.need_states ? one * (is_bwd ? 2 : 1) : 0;
+  return p;
+}
+
+// ------------------------------------------------------------------ launches
+
+static la2_status launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? LA2_OK : LA2_ERR_CUDA;
+}
+
+template <typename T>
+static la2_status run_chunk_states(const void* a, const void* b, float* out, int64_t BH, int64_t N,
+                                   int da, int db, const Plan& p, cudaStream_t st) {
+  const size_t smem = chunk_state_smem(da, db);
+  LaunchTimer t(K_CHUNK_STATE, st);
+  chunk_state_kernel<T><<<(unsigned)(BH * p.C), kSimtThreads, smem, st>>>(
+      static_cast<const T*>(a), static_cast<const T*>(b), out, N, da, db, p.L, p.C);
+  return launch_status();
+}
+
+static la2_status run_scan(float* s, int64_t BH, int nel, const Plan& p, int mode, cudaStream_t st) {
+  dim3 grid((nel + kSimtThreads - 1) / kSimtThreads, (unsigned)BH);
+  LaunchTimer t(K_CHUNK_SCAN, st);
+  chunk_scan_kernel<<<grid, kSimtThreads, 0, st>>>(s, p.C, nel, mode);
+  return launch_status();
+}
+
+template <typename T>
+static la2_status forward_simt(const void* q, const void* k, const void* v, void* o, int64_t BH,
+                               int64_t N, int d, int dv, int causal, int block, float* states,
+                               const Plan& p, cudaStream_t st) {
+  const size_t smem = fwd_simt_smem(d, dv, block);
+  if (cudaFuncSetAttribute(fwd_simt_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return LA2_ERR_CUDA;
+  LaunchTimer t(K_FWD_SIMT, st);
+  fwd_simt_kernel<T><<<(unsigned)(BH * p.C), kSimtThreads, smem, st>>>(
+      static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v),
+      static_cast<T*>(o), states, N, d, dv, block, p.L, p.C, causal);
+  return launch_status();
+}
+
+template <typename T>
+static la2_status backward_simt(const void* q, const void* k, const void* v, const void* dout,
+                                void* dq, void* dk, void* dvv, int64_t BH, int64_t N, int d,
+                                int dv, int causal, int block, float* s_kv, float* s_u,
+                                const Plan& p, cudaStream_t st) {
+  const size_t smem_q = bwd_dq_simt_smem(d, dv, block);
+  const size_t smem_kv = bwd_dkdv_simt_smem(d, dv, block);
+  if (cudaFuncSetAttribute(bwd_dq_simt_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem_q) != cudaSuccess ||
+      cudaFuncSetAttribute(bwd_dkdv_simt_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem_kv) != cudaSuccess)
+    return LA2_ERR_CUDA;
+  {
+    LaunchTimer t(K_BWD_DQ_SIMT, st);
+    bwd_dq_simt_kernel<T><<<(unsigned)(BH * p.C), kSimtThreads, smem_q, st>>>(
+        static_cast<const T*>(k), static_cast<const T*>(v), static_cast<const T*>(dout),
+        static_cast<T*>(dq), s_kv, N, d, dv, block, p.L, p.C, causal);
+  }
+  la2_status s = launch_status();
+  if (s != LA2_OK) return s;
+  {
+    LaunchTimer t(K_BWD_DKDV_SIMT, st);
+    bwd_dkdv_simt_kernel<T><<<(unsigned)(BH * p.C), kSimtThreads, smem_kv, st>>>(
+        static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v),
+        static_cast<const T*>(dout), static_cast<T*>(dk), static_cast<T*>(dvv), s_u, N, d, dv,
+        block, p.L, p.C, causal);
+  }
+  return launch_status();
+}
+
+}  // namespace la2
+
+using namespace la2;
+
+// ====================================================================== C ABI
+
+extern "C" {
+
+size_t la2_workspace_size(int64_t B, int64_t H, int64_t N, int64_t d, int64_t dv, int causal,
+                          int block, la2_dtype dt, int is_backward) {
+  if (check_shape(B, H, N, d, dv, causal, block, dt, is_backward != 0) != LA2_OK) return (size_t)-1;
+  if (B == 0 || H == 0 || N == 0) return 0;
+  const int sms = device_sm_count();
+  if (sms <= 0) return (size_t)-1;
+  return make_plan(B, H, N, d, dv, causal, block, dt, is_backward != 0, sms).ws_bytes;
+}
+
+int64_t la2_num_chunks(int64_t B, int64_t H, int64_t N, int block, la2_dtype dt) {
+  const int64_t d = 128, dv = 128;
+  if (check_shape(B, H, N, d, dv, 1, block, dt, false) != LA2_OK) return -1;
+  if (B == 0 || H == 0 || N == 0) return 0;
+  const int sms = device_sm_count();
+  if (sms <= 0) return -1;
+  return make_plan(B, H, N, d, dv, 1, block, dt, false, sms).C;
+}
+
+la2_status la2_set_chunk_len(int64_t chunk_len) {
+  if (chunk_len < 0) return LA2_ERR_INVALID_ARG;
+  g_chunk_len = chunk_len;
+  return LA2_OK;
+}
+
+la2_status la2_set_spin_limit(int64_t iterations) {
+  if (iterations < 0) return LA2_ERR_INVALID_ARG;
+  g_spin_limit = iterations;
+  return LA2_OK;
+}
+
+la2_status la2_forward(const void* q, const void* k, const void* v, void* o, int64_t B, int64_t H,
+                       int64_t N, int64_t d, int64_t dv, int causal, int block, la2_dtype dt,
+                       void* workspace, size_t workspace_bytes, la2_stream_t stream) {
+  la2_status s = check_shape(B, H, N, d, dv, causal, block, dt, false);
+  if (s != LA2_OK) return s;
+  if (B == 0 || H == 0 || N == 0) return LA2_OK;
+  if (!q || !k || !v || !o) return LA2_ERR_INVALID_ARG;
+  if (!is_aligned(q, 16) || !is_aligned(k, 16) || !is_aligned(v, 16) || !is_aligned(o, 16))
+    return LA2_ERR_INVALID_ARG;
+  const size_t es = dt == LA2_BF16 ? 2 : 4;
+  const size_t nq = (size_t)B * H * N * d * es, nv = (size_t)B * H * N * dv * es;
+  if (overlaps(o, nv, q, nq) || overlaps(o, nv, k, nq) || overlaps(o, nv, v, nv))
+    return LA2_ERR_INVALID_ARG;
+  const int sms = device_sm_count();
+  if (sms <= 0) return LA2_ERR_CUDA;
+  const Plan p = make_plan(B, H, N, d, dv, causal, block, dt, false, sms);
+  if (p.ws_bytes > 0) {
+    if (!workspace || workspace_bytes < p.ws_bytes) return LA2_ERR_WORKSPACE;
+    if (!is_aligned(workspace, 256)) return LA2_ERR_INVALID_ARG;
+    if (overlaps(workspace, p.ws_bytes, o, nv)) return LA2_ERR_INVALID_ARG;
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t BH = B * H;
+  float* states = p.need_states ? static_cast<float*>(workspace) : nullptr;
+  const int nel = (int)(d * dv);
+  if (p.tc) return sm100_forward(q, k, v, o, BH, N, (int)d, (int)dv, causal, block, states, p.L,
+                                 p.C, spin_limit(), st);
+  if (p.need_states) {
+    s = dt == LA2_BF16
+            ? run_chunk_states<__nv_bfloat16>(k, v, states, BH, N, (int)d, (int)dv, p, st)
+            : run_chunk_states<float>(k, v, states, BH, N, (int)d, (int)dv, p, st);
+    if (s != LA2_OK) return s;
+    s = run_scan(states, BH, nel, p, causal ? 0 : 2, st);
+    if (s != LA2_OK) return s;
+  }
+  return dt == LA2_BF16
+             ? forward_simt<__nv_bfloat16>(q, k, v, o, BH, N, (int)d, (int)dv, causal, block,
+                                           states, p, st)
+             : forward_simt<float>(q, k, v, o, BH, N, (int)d, (int)dv, causal, block, states, p,
+                                   st);
+}
+
+la2_status la2_backward(const void* q, const void* k, const void* v, const void* dout, void* dq,
+                        void* dk, void* dvv, int64_t B, int64_t H, int64_t N, int64_t d,
+                        int64_t dv, int causal, int block, la2_dtype dt, void* workspace,
+                        size_t workspace_bytes, la2_stream_t stream) {
+  la2_status s = check_shape(B, H, N, d, dv, causal, block, dt, true);
+  if (s != LA2_OK) return s;
+  if (B == 0 || H == 0 || N == 0) return LA2_OK;
+  const void* ins[4] = {q, k, v, dout};
+  void* outs[3] = {dq, dk, dvv};
+  for (const void* p : ins)
+    if (!p || !is_aligned(p, 16)) return LA2_ERR_INVALID_ARG;
+  for (void* p : outs)
+    if (!p || !is_aligned(p, 16)) return LA2_ERR_INVALID_ARG;
+  const size_t es = dt == LA2_BF16 ? 2 : 4;
+  const size_t nq = (size_t)B * H * N * d * es, nv = (size_t)B * H * N * dv * es;
+  const size_t in_sz[4] = {nq, nq, nv, nv};
+  const size_t out_sz[3] = {nq, nq, nv};
+  for (int i = 0; i < 3; ++i) {
+    for (int j = 0; j < 4; ++j)
+      if (overlaps(outs[i], out_sz[i], ins[j], in_sz[j])) return LA2_ERR_INVALID_ARG;
+    for (int j = i + 1; j < 3; ++j)
+      if (overlaps(outs[i], out_sz[i], outs[j], out_sz[j])) return LA2_ERR_INVALID_ARG;
+  }
+  const int sms = device_sm_count();
+  if (sms <= 0) return LA2_ERR_CUDA;
+  const Plan p = make_plan(B, H, N, d, dv, causal, block, dt, true, sms);
+  if (p.ws_bytes > 0) {
+    if (!workspace || workspace_bytes < p.ws_bytes) return LA2_ERR_WORKSPACE;
+    if (!is_aligned(workspace, 256)) return LA2_ERR_INVALID_ARG;
+    for (int i = 0; i < 3; ++i)
+      if (overlaps(workspace, p.ws_bytes, outs[i], out_sz[i])) return LA2_ERR_INVALID_ARG;
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t BH = B * H;
+  const int nel = (int)(d * dv);
+  float* s_kv = p.need_states ? static_cast<float*>(workspace) : nullptr;
+  float* s_u = p.need_states ? s_kv + (size_t)BH * p.C * nel : nullptr;
+  if (p.need_states) {
+    const bool bf = dt == LA2_BF16;
+    s = bf ? run_chunk_states<__nv_bfloat16>(k, v, s_kv, BH, N, (int)d, (int)dv, p, st)
+           : run_chunk_states<float>(k, v, s_kv, BH, N, (int)d, (int)dv, p, st);
+    if (s != LA2_OK) return s;
+    s = bf ? run_chunk_states<__nv_bfloat16>(q, dout, s_u, BH, N, (int)d, (int)dv, p, st)
+           : run_chunk_states<float>(q, dout, s_u, BH, N, (int)d, (int)dv, p, st);
+    if (s != LA2_OK) return s;
+    s = run_scan(s_kv, BH, nel, p, causal ? 0 : 2, st);
+    if (s != LA2_OK) return s;
+    s = run_scan(s_u, BH, nel, p, causal ? 1 : 2, st);
+    if (s != LA2_OK) return s;
+  }
+  if (p.tc)
+    return sm100_backward(q, k, v, dout, dq, dk, dvv, BH, N, (int)d, (int)dv, causal, block, s_kv,
+                          s_u, p.L, p.C, spin_limit(), st);
+  return dt == LA2_BF16
+             ? backward_simt<__nv_bfloat16>(q, k, v, dout, dq, dk, dvv, BH, N, (int)d, (int)dv,
+                                            causal, block, s_kv, s_u, p, st)
+             : backward_simt<float>(q, k, v, dout, dq, dk, dvv, BH, N, (int)d, (int)dv, causal,
+                                    block, s_kv, s_u, p, st);
+}
+
+la2_status la2_check(la2_stream_t stream) {
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return LA2_ERR_CUDA;
+  int code = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&code, g_error_code, sizeof(int)) != cudaSuccess) return LA2_ERR_CUDA;
+  if (code != 0) {
+    if (cudaMemcpyToSymbol(g_error_code, &zero, sizeof(int)) != cudaSuccess) return LA2_ERR_CUDA;
+    return code == DEV_ERR_TIMEOUT ? LA2_ERR_TIMEOUT : LA2_ERR_CUDA;
+  }
+  return LA2_OK;
+}
+
+const char* la2_status_string(la2_status s) {
+  switch (s) {
+    case LA2_OK: return "LA2_OK";
+    case LA2_ERR_INVALID_ARG: return "LA2_ERR_INVALID_ARG: invalid argument";
+    case LA2_ERR_UNSUPPORTED: return "LA2_ERR_UNSUPPORTED: unsupported dtype/shape/block";
+    case LA2_ERR_WORKSPACE: return "LA2_ERR_WORKSPACE: workspace missing or too small";
+    case LA2_ERR_CUDA: return "LA2_ERR_CUDA: CUDA call or launch failed";
+    case LA2_ERR_TIMEOUT: return "LA2_ERR_TIMEOUT: a device-side wait gave up";
+  }
+  return "LA2: unknown status";
+}
+
+la2_status la2_profile_enable(int on) {
+  g_prof.on = on != 0;
+  if (g_prof.on) g_prof.used = 0;
+  return LA2_OK;
+}
+
+int la2_profile_num_kernels(void) { return K_COUNT; }
+
+const char* la2_profile_kernel_name(int kernel) {
+  return (kernel >= 0 && kernel < K_COUNT) ? kKernelNames[kernel] : nullptr;
+}
+
+la2_status la2_profile_collect(int kernel, int64_t* launches, double* total_ms) {
+  if (kernel < 0 || kernel >= K_COUNT || !launches || !total_ms) return LA2_ERR_INVALID_ARG;
+  int64_t n = 0;
+  double ms = 0.0;
+  for (size_t i = 0; i < g_prof.used; ++i) {
+    EventRecord& r = g_prof.pool[i];
+    if (r.kernel != kernel) continue;
+    if (cudaEventSynchronize(r.stop) != cudaSuccess) return LA2_ERR_CUDA;
+    float t = 0.f;
+    if (cudaEventElapsedTime(&t, r.start, r.stop) != cudaSuccess) return LA2_ERR_CUDA;
+    ms += t;
+    ++n;
+  }
+  *launches = n;
+  *total_ms = ms;
+  return LA2_OK;
+}
+
+int la2_version(void) { return (0 << 16) | 1; }
+
+}  // extern "C"

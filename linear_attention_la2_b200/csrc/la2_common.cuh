@@ -1,0 +1,35 @@
+// Shared device-side definitions for the libla2 kernels (one translation unit).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace la2 {
+
+// Device error word. The first bounded wait that gives up stores its code
+// here; la2_check() reads and clears it. Value 0 means no error.
+__device__ int g_error_code = 0;
+__device__ int g_error_where = 0;
+
+enum DeviceError : int {
+  DEV_ERR_NONE = 0,
+  DEV_ERR_TIMEOUT = 5,
+};
+
+__device__ __forceinline__ void record_error(int code, int where) {
+  if (atomicCAS(&g_error_code, 0, code) == 0) g_error_where = where;
+}
+
+__device__ __forceinline__ int64_t imin64(int64_t a, int64_t b) { return a < b ? a : b; }
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+}  // namespace la2

@@ -1,0 +1,362 @@
+// CUDA-core kernels of libla2: chunk states, the state scan, and the fp32
+// forward / backward block loops.
+//
+// Article "Lightning Attention-2 新一代注意力机制", section
+// "Lightning Attention-2简介", point 2 (Fig. 3): every (b, h) sequence is cut
+// into blocks of Bk rows; a block's output is the masked left product of the
+// block plus the right product of its queries with the KV state accumulated
+// over earlier blocks, and the state then absorbs the block's K^T V.
+//
+// Work unit = one chunk of one (b, h) sequence: rows [c*L, min(N, (c+1)*L)),
+// L a multiple of Bk. A chunk starts from the exclusive prefix of the chunk
+// states of its sequence (la2_chunk_state + la2_chunk_scan), so chunks of one
+// sequence run in parallel. Everything accumulates in fp32; inputs of type T
+// (float or bf16) are widened on load and outputs rounded to T on store.
+#pragma once
+
+#include "la2_common.cuh"
+
+namespace la2 {
+
+constexpr int kSimtThreads = 256;
+
+// ----------------------------------------------------------------------------
+// Chunk states: S[bh][c] = sum over rows t of chunk c of a_t^T b_t  (da x db).
+// (a, b) = (K, V) gives the KV state of a chunk; (Q, dO) gives the state the
+// dK/dV pass of the backward carries. One CTA per (bh, c); each thread keeps
+// up to 64 state elements in registers.
+// ----------------------------------------------------------------------------
+constexpr int kStateRowsPerTile = 32;
+
+template <typename T>
+__global__ void __launch_bounds__(kSimtThreads)
+chunk_state_kernel(const T* __restrict__ a, const T* __restrict__ b, float* __restrict__ out,
+                   int64_t N, int da, int db, int64_t L, int64_t C) {
+  extern __shared__ float smem[];
+  float* As = smem;                              // [32][da]
+  float* Bs = smem + kStateRowsPerTile * da;     // [32][db]
+  const int64_t unit = blockIdx.x;
+  const int64_t bh = unit / C, c = unit % C;
+  const int64_t t0 = c * L, t1 = imin64(N, t0 + L);
+  const T* ab = a + bh * N * da;
+  const T* bb = b + bh * N * db;
+  const int nel = da * db;
+  float acc[64];
+#pragma unroll
+  for (int r = 0; r < 64; ++r) acc[r] = 0.f;
+
+  for (int64_t s0 = t0; s0 < t1; s0 += kStateRowsPerTile) {
+    const int rows = (int)imin64(kStateRowsPerTile, t1 - s0);
+    for (int i = threadIdx.x; i < kStateRowsPerTile * da; i += blockDim.x) {
+      const int r = i / da, col = i % da;
+      As[i] = r < rows ? to_f32(ab[(s0 + r) * da + col]) : 0.f;
+    }
+    for (int i = threadIdx.x; i < kStateRowsPerTile * db; i += blockDim.x) {
+      const int r = i / db, col = i % db;
+      Bs[i] = r < rows ? to_f32(bb[(s0 + r) * db + col]) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < 64; ++r) {
+      const int idx = threadIdx.x + r * kSimtThreads;
+      if (idx < nel) {
+        const int ci = idx / db, ei = idx % db;
+        float s = acc[r];
+        for (int t = 0; t < rows; ++t) s = fmaf(As[t * da + ci], Bs[t * db + ei], s);
+        acc[r] = s;
+      }
+    }
+    __syncthreads();
+  }
+  float* o = out + (bh * C + c) * (int64_t)nel;
+#pragma unroll
+  for (int r = 0; r < 64; ++r) {
+    const int idx = threadIdx.x + r * kSimtThreads;
+    if (idx < nel) o[idx] = acc[r];
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Scan of chunk states along c, per (bh, element), in place.
+//   mode 0: exclusive prefix  P_c = sum_{c' < c} S_c'   (causal, forward order)
+//   mode 1: exclusive suffix  R_c = sum_{c' > c} S_c'   (causal, reverse order)
+//   mode 2: total into slot 0  T = sum_c S_c             (non-causal)
+// ----------------------------------------------------------------------------
+__global__ void __launch_bounds__(kSimtThreads)
+chunk_scan_kernel(float* __restrict__ s, int64_t C, int nel, int mode) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= nel) return;
+  float* p = s + (int64_t)blockIdx.y * C * nel + e;
+  float run = 0.f;
+  if (mode == 0) {
+    for (int64_t c = 0; c < C; ++c) {
+      const float x = p[c * nel];
+      p[c * nel] = run;
+      run += x;
+    }
+  } else if (mode == 1) {
+    for (int64_t c = C - 1; c >= 0; --c) {
+      const float x = p[c * nel];
+      p[c * nel] = run;
+      run += x;
+    }
+  } else {
+    for (int64_t c = 0; c < C; ++c) run += p[c * nel];
+    p[0] = run;
+  }
+}
+
+// Shared-memory helpers: load `rows` rows of a [*, w] tile, zero the rest.
+template <typename T>
+__device__ __forceinline__ void load_tile(float* dst, const T* src, int rows, int Bk, int w) {
+  for (int i = threadIdx.x; i < Bk * w; i += blockDim.x) {
+    const int r = i / w;
+    dst[i] = r < rows ? to_f32(src[i]) : 0.f;
+  }
+}
+
+__device__ __forceinline__ void load_state(float* dst, const float* src, int nel) {
+  for (int i = threadIdx.x; i < nel; i += blockDim.x) dst[i] = src ? src[i] : 0.f;
+}
+
+// ----------------------------------------------------------------------------
+// Forward block loop (CUDA cores). Per block i of the chunk:
+//   O_i = ((Q_i K_i^T) ⊙ M_B) V_i + Q_i KV ;  KV += K_i^T V_i
+// Non-causal: O_i = Q_i T with T the total K^T V of the sequence.
+// Shared memory: KV [d][dv], Q [Bk][d], K [Bk][d], V [Bk][dv], S [Bk][Bk].
+// ----------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(kSimtThreads)
+fwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
+                T* __restrict__ o, const float* __restrict__ states, int64_t N, int d, int dv,
+                int Bk, int64_t L, int64_t C, int causal) {
+  extern __shared__ float smem[];
+  float* KV = smem;
+  float* Qs = KV + d * dv;
+  float* Ks = Qs + Bk * d;
+  float* Vs = Ks + Bk * d;
+  float* S = Vs + Bk * dv;
+  const int64_t unit = blockIdx.x;
+  const int64_t bh = unit / C, c = unit % C;
+  const int64_t t0 = c * L, t1 = imin64(N, t0 + L);
+  const T* qb = q + bh * N * d;
+  const T* kb = k + bh * N * d;
+  const T* vb = v + bh * N * dv;
+  T* ob = o + bh * N * dv;
+  const int64_t nel = (int64_t)d * dv;
+  const float* init = nullptr;
+  if (!causal) init = states + bh * C * nel;           // total in slot 0
+  else if (states) init = states + (bh * C + c) * nel;  // exclusive prefix
+  load_state(KV, init, (int)nel);
+
+  for (int64_t i0 = t0; i0 < t1; i0 += Bk) {
+    const int rows = (int)imin64(Bk, t1 - i0);
+    load_tile(Qs, qb + i0 * d, rows, Bk, d);
+    if (causal) {
+      load_tile(Ks, kb + i0 * d, rows, Bk, d);
+      load_tile(Vs, vb + i0 * dv, rows, Bk, dv);
+    }
+    __syncthreads();
+    if (causal) {
+      for (int i = threadIdx.x; i < Bk * Bk; i += blockDim.x) {
+        const int t = i / Bk, j = i % Bk;
+        float s = 0.f;
+        if (j <= t)
+          for (int cc = 0; cc < d; ++cc) s = fmaf(Qs[t * d + cc], Ks[j * d + cc], s);
+        S[i] = s;  // M_B: lower-triangular ones, diagonal kept
+      }
+      __syncthreads();
+    }
+    for (int i = threadIdx.x; i < rows * dv; i += blockDim.x) {
+      const int t = i / dv, e = i % dv;
+      float acc = 0.f;
+      if (causal)
+        for (int j = 0; j <= t; ++j) acc = fmaf(S[t * Bk + j], Vs[j * dv + e], acc);
+      for (int cc = 0; cc < d; ++cc) acc = fmaf(Qs[t * d + cc], KV[cc * dv + e], acc);
+      ob[(i0 + t) * dv + e] = from_f32<T>(acc);
+    }
+    __syncthreads();
+    if (causal) {
+      for (int i = threadIdx.x; i < d * dv; i += blockDim.x) {
+        const int cc = i / dv, e = i % dv;
+        float acc = KV[i];
+        for (int t = 0; t < rows; ++t) acc = fmaf(Ks[t * d + cc], Vs[t * dv + e], acc);
+        KV[i] = acc;
+      }
+      __syncthreads();
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Backward, dQ pass (blocks ascending, state KV = sum_{j<i} K_j^T V_j):
+//   dQ_i = ((dO_i V_i^T) ⊙ M_B) K_i + dO_i KV^T ;  KV += K_i^T V_i
+// Non-causal: dQ_i = dO_i T^T with T = K^T V over the whole sequence.
+// Shared memory: KV [d][dv], dO [Bk][dv], V [Bk][dv], K [Bk][d], A [Bk][Bk].
+// ----------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(kSimtThreads)
+bwd_dq_simt_kernel(const T* __restrict__ k, const T* __restrict__ v, const T* __restrict__ dout,
+                   T* __restrict__ dq, const float* __restrict__ states, int64_t N, int d, int dv,
+                   int Bk, int64_t L, int64_t C, int causal) {
+  extern __shared__ float smem[];
+  float* KV = smem;
+  float* dOs = KV + d * dv;
+  float* Vs = dOs + Bk * dv;
+  float* Ks = Vs + Bk * dv;
+  float* A = Ks + Bk * d;
+  const int64_t unit = blockIdx.x;
+  const int64_t bh = unit / C, c = unit % C;
+  const int64_t t0 = c * L, t1 = imin64(N, t0 + L);
+  const T* kb = k + bh * N * d;
+  const T* vb = v + bh * N * dv;
+  const T* gb = dout + bh * N * dv;
+  T* dqb = dq + bh * N * d;
+  const int64_t nel = (int64_t)d * dv;
+  const float* init = nullptr;
+  if (!causal) init = states + bh * C * nel;
+  else if (states) init = states + (bh * C + c) * nel;
+  load_state(KV, init, (int)nel);
+
+  for (int64_t i0 = t0; i0 < t1; i0 += Bk) {
+    const int rows = (int)imin64(Bk, t1 - i0);
+    load_tile(dOs, gb + i0 * dv, rows, Bk, dv);
+    if (causal) {
+      load_tile(Vs, vb + i0 * dv, rows, Bk, dv);
+      load_tile(Ks, kb + i0 * d, rows, Bk, d);
+    }
+    __syncthreads();
+    if (causal) {
+      for (int i = threadIdx.x; i < Bk * Bk; i += blockDim.x) {
+        const int t = i / Bk, j = i % Bk;
+        float s = 0.f;
+        if (j <= t)
+          for (int e = 0; e < dv; ++e) s = fmaf(dOs[t * dv + e], Vs[j * dv + e], s);
+        A[i] = s;
+      }
+      __syncthreads();
+    }
+    for (int i = threadIdx.x; i < rows * d; i += blockDim.x) {
+      const int t = i / d, cc = i % d;
+      float acc = 0.f;
+      if (causal)
+        for (int j = 0; j <= t; ++j) acc = fmaf(A[t * Bk + j], Ks[j * d + cc], acc);
+      for (int e = 0; e < dv; ++e) acc = fmaf(dOs[t * dv + e], KV[cc * dv + e], acc);
+      dqb[(i0 + t) * d + cc] = from_f32<T>(acc);
+    }
+    __syncthreads();
+    if (causal) {
+      for (int i = threadIdx.x; i < d * dv; i += blockDim.x) {
+        const int cc = i / dv, e = i % dv;
+        float acc = KV[i];
+        for (int t = 0; t < rows; ++t) acc = fmaf(Ks[t * d + cc], Vs[t * dv + e], acc);
+        KV[i] = acc;
+      }
+      __syncthreads();
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Backward, dK/dV pass (blocks descending, state U = sum_{l>i} Q_l^T dO_l):
+//   dK_i = ((dO_i V_i^T) ⊙ M_B)^T Q_i + V_i U^T
+//   dV_i = ((Q_i K_i^T) ⊙ M_B)^T dO_i + K_i U ;  U += Q_i^T dO_i
+// Non-causal: dK_i = V_i U^T, dV_i = K_i U with U = Q^T dO over the sequence.
+// Shared memory: U [d][dv], Q, K [Bk][d], V, dO [Bk][dv], A, P [Bk][Bk].
+// ----------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(kSimtThreads)
+bwd_dkdv_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
+                     const T* __restrict__ dout, T* __restrict__ dk, T* __restrict__ dvv,
+                     const float* __restrict__ states, int64_t N, int d, int dv, int Bk,
+                     int64_t L, int64_t C, int causal) {
+  extern __shared__ float smem[];
+  float* U = smem;
+  float* Qs = U + d * dv;
+  float* Ks = Qs + Bk * d;
+  float* Vs = Ks + Bk * d;
+  float* dOs = Vs + Bk * dv;
+  float* A = dOs + Bk * dv;
+  float* P = A + Bk * Bk;
+  const int64_t unit = blockIdx.x;
+  const int64_t bh = unit / C, c = unit % C;
+  const int64_t t0 = c * L, t1 = imin64(N, t0 + L);
+  const T* qb = q + bh * N * d;
+  const T* kb = k + bh * N * d;
+  const T* vb = v + bh * N * dv;
+  const T* gb = dout + bh * N * dv;
+  T* dkb = dk + bh * N * d;
+  T* dvb = dvv + bh * N * dv;
+  const int64_t nel = (int64_t)d * dv;
+  const float* init = nullptr;
+  if (!causal) init = states + bh * C * nel;
+  else if (states) init = states + (bh * C + c) * nel;  // exclusive suffix
+  load_state(U, init, (int)nel);
+
+  const int64_t nblk = (t1 - t0 + Bk - 1) / Bk;
+  for (int64_t bi = nblk - 1; bi >= 0; --bi) {
+    const int64_t i0 = t0 + bi * Bk;
+    const int rows = (int)imin64(Bk, t1 - i0);
+    load_tile(Ks, kb + i0 * d, rows, Bk, d);
+    load_tile(Vs, vb + i0 * dv, rows, Bk, dv);
+    if (causal) {
+      load_tile(Qs, qb + i0 * d, rows, Bk, d);
+      load_tile(dOs, gb + i0 * dv, rows, Bk, dv);
+    }
+    __syncthreads();
+    if (causal) {
+      for (int i = threadIdx.x; i < Bk * Bk; i += blockDim.x) {
+        const int t = i / Bk, j = i % Bk;  // t: query row, j: key row
+        float a = 0.f, p = 0.f;
+        if (j <= t) {
+          for (int e = 0; e < dv; ++e) a = fmaf(dOs[t * dv + e], Vs[j * dv + e], a);
+          for (int cc = 0; cc < d; ++cc) p = fmaf(Qs[t * d + cc], Ks[j * d + cc], p);
+        }
+        A[i] = a;
+        P[i] = p;
+      }
+      __syncthreads();
+    }
+    for (int i = threadIdx.x; i < rows * d; i += blockDim.x) {
+      const int j = i / d, cc = i % d;
+      float acc = 0.f;
+      if (causal)
+        for (int t = j; t < rows; ++t) acc = fmaf(A[t * Bk + j], Qs[t * d + cc], acc);
+      for (int e = 0; e < dv; ++e) acc = fmaf(Vs[j * dv + e], U[cc * dv + e], acc);
+      dkb[(i0 + j) * d + cc] = from_f32<T>(acc);
+    }
+    for (int i = threadIdx.x; i < rows * dv; i += blockDim.x) {
+      const int j = i / dv, e = i % dv;
+      float acc = 0.f;
+      if (causal)
+        for (int t = j; t < rows; ++t) acc = fmaf(P[t * Bk + j], dOs[t * dv + e], acc);
+      for (int cc = 0; cc < d; ++cc) acc = fmaf(Ks[j * d + cc], U[cc * dv + e], acc);
+      dvb[(i0 + j) * dv + e] = from_f32<T>(acc);
+    }
+    __syncthreads();
+    if (causal) {
+      for (int i = threadIdx.x; i < d * dv; i += blockDim.x) {
+        const int cc = i / dv, e = i % dv;
+        float acc = U[i];
+        for (int t = 0; t < rows; ++t) acc = fmaf(Qs[t * d + cc], dOs[t * dv + e], acc);
+        U[i] = acc;
+      }
+      __syncthreads();
+    }
+  }
+}
+
+inline size_t fwd_simt_smem(int d, int dv, int Bk) {
+  return sizeof(float) * ((size_t)d * dv + (size_t)Bk * (2 * d + dv) + (size_t)Bk * Bk);
+}
+inline size_t bwd_dq_simt_smem(int d, int dv, int Bk) {
+  return sizeof(float) * ((size_t)d * dv + (size_t)Bk * (2 * dv + d) + (size_t)Bk * Bk);
+}
+inline size_t bwd_dkdv_simt_smem(int d, int dv, int Bk) {
+  return sizeof(float) * ((size_t)d * dv + (size_t)Bk * (2 * d + 2 * dv) + 2 * (size_t)Bk * Bk);
+}
+inline size_t chunk_state_smem(int da, int db) {
+  return sizeof(float) * (size_t)kStateRowsPerTile * (da + db);
+}
+
+}  // namespace la2

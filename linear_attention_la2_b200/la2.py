@@ -1,0 +1,192 @@
+"""ctypes binding of libla2.so (C ABI in ``include/la2.h``).
+
+Argument marshalling only: every step of the computation runs in the
+library's CUDA kernels. The raw functions keep the C names and argument order
+and return the C status code. ``forward`` / ``backward`` below take torch
+tensors, allocate outputs and the workspace with torch (PyTorch is only the
+allocator and the stream provider here) and raise ``La2Error`` on a non-zero
+status. Importing this module fails loudly when the library is missing.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libla2.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"libla2.so not found at {LIB_PATH}; build it with "
+        "`python -m linear_attention_la2_b200.build` (nvcc, sm_100a)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+LA2_OK = 0
+LA2_ERR_INVALID_ARG = 1
+LA2_ERR_UNSUPPORTED = 2
+LA2_ERR_WORKSPACE = 3
+LA2_ERR_CUDA = 4
+LA2_ERR_TIMEOUT = 5
+LA2_F32 = 0
+LA2_BF16 = 1
+
+_i64 = ctypes.c_int64
+_int = ctypes.c_int
+_vp = ctypes.c_void_p
+_sz = ctypes.c_size_t
+
+_SIGS = {
+    "la2_workspace_size": (_sz, [_i64, _i64, _i64, _i64, _i64, _int, _int, _int, _int]),
+    "la2_forward": (_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _int, _int, _int,
+                           _vp, _sz, _vp]),
+    "la2_backward": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _int,
+                            _int, _int, _vp, _sz, _vp]),
+    "la2_check": (_int, [_vp]),
+    "la2_status_string": (ctypes.c_char_p, [_int]),
+    "la2_set_chunk_len": (_int, [_i64]),
+    "la2_num_chunks": (_i64, [_i64, _i64, _i64, _int, _int]),
+    "la2_set_spin_limit": (_int, [_i64]),
+    "la2_profile_enable": (_int, [_int]),
+    "la2_profile_num_kernels": (_int, []),
+    "la2_profile_kernel_name": (ctypes.c_char_p, [_int]),
+    "la2_profile_collect": (_int, [_int, ctypes.POINTER(_i64), ctypes.POINTER(ctypes.c_double)]),
+    "la2_version": (_int, []),
+}
+
+EXPORTED = tuple(_SIGS)
+
+for _name, (_res, _args) in _SIGS.items():
+    _fn = getattr(_lib, _name)
+    _fn.restype = _res
+    _fn.argtypes = _args
+
+# Raw C entry points, same names and argument order as include/la2.h.
+la2_workspace_size = _lib.la2_workspace_size
+la2_forward = _lib.la2_forward
+la2_backward = _lib.la2_backward
+la2_check = _lib.la2_check
+la2_set_chunk_len = _lib.la2_set_chunk_len
+la2_num_chunks = _lib.la2_num_chunks
+la2_set_spin_limit = _lib.la2_set_spin_limit
+la2_profile_enable = _lib.la2_profile_enable
+la2_profile_num_kernels = _lib.la2_profile_num_kernels
+la2_version = _lib.la2_version
+
+
+def la2_status_string(code: int) -> str:
+    return _lib.la2_status_string(code).decode()
+
+
+def la2_profile_kernel_name(kernel: int) -> str:
+    s = _lib.la2_profile_kernel_name(kernel)
+    return s.decode() if s else ""
+
+
+def la2_profile_collect(kernel: int):
+    n = _i64(0)
+    ms = ctypes.c_double(0.0)
+    st = _lib.la2_profile_collect(kernel, ctypes.byref(n), ctypes.byref(ms))
+    _raise(st)
+    return int(n.value), float(ms.value)
+
+
+class La2Error(RuntimeError):
+    def __init__(self, code: int):
+        super().__init__(la2_status_string(code))
+        self.code = code
+
+
+def _raise(code: int):
+    if code != LA2_OK:
+        raise La2Error(code)
+
+
+# ------------------------------------------------------------ torch helpers
+
+
+def _dtype_code(t):
+    import torch
+
+    if t.dtype == torch.bfloat16:
+        return LA2_BF16
+    if t.dtype == torch.float32:
+        return LA2_F32
+    raise La2Error(LA2_ERR_UNSUPPORTED)
+
+
+def _stream_handle(stream):
+    import torch
+
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return _vp(stream.cuda_stream)
+
+
+def _ptr(t):
+    return _vp(t.data_ptr()) if t is not None and t.numel() > 0 else _vp(0)
+
+
+def workspace_bytes(B, H, N, d, dv, causal, block, dtype_code, is_backward) -> int:
+    n = la2_workspace_size(B, H, N, d, dv, int(causal), block, dtype_code, int(is_backward))
+    if n == ctypes.c_size_t(-1).value:
+        raise La2Error(LA2_ERR_INVALID_ARG)
+    return int(n)
+
+
+def _workspace(nbytes, device):
+    import torch
+
+    if nbytes == 0:
+        return None
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def _check_inputs(*ts):
+    for t in ts:
+        if not t.is_cuda:
+            raise La2Error(LA2_ERR_INVALID_ARG)
+        if not t.is_contiguous():
+            raise La2Error(LA2_ERR_INVALID_ARG)
+
+
+def forward(q, k, v, causal: bool = True, block: int = 64, out=None, workspace=None, stream=None):
+    """O = ((Q K^T) ⊙ M) V for [B,H,N,d] CUDA tensors; returns O."""
+    import torch
+
+    _check_inputs(q, k, v)
+    B, H, N, d = q.shape
+    dv = v.shape[-1]
+    dt = _dtype_code(q)
+    if out is None:
+        out = torch.empty((B, H, N, dv), dtype=q.dtype, device=q.device)
+    need = workspace_bytes(B, H, N, d, dv, causal, block, dt, False)
+    ws = workspace if workspace is not None else _workspace(need, q.device)
+    _raise(la2_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, N, d, dv, int(causal), block, dt,
+                       _ptr(ws), ws.numel() if ws is not None else 0, _stream_handle(stream)))
+    return out
+
+
+def backward(q, k, v, do, causal: bool = True, block: int = 64, outs=None, workspace=None,
+             stream=None):
+    """Gradients (dQ, dK, dV) of <dO, O> for the same op; returns a tuple."""
+    import torch
+
+    _check_inputs(q, k, v, do)
+    B, H, N, d = q.shape
+    dv = v.shape[-1]
+    dt = _dtype_code(q)
+    if outs is None:
+        outs = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
+    dq, dk, dvv = outs
+    need = workspace_bytes(B, H, N, d, dv, causal, block, dt, True)
+    ws = workspace if workspace is not None else _workspace(need, q.device)
+    _raise(la2_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dvv), B, H, N,
+                        d, dv, int(causal), block, dt, _ptr(ws), ws.numel() if ws is not None else 0,
+                        _stream_handle(stream)))
+    return dq, dk, dvv
+
+
+def check(stream=None):
+    _raise(la2_check(_stream_handle(stream)))

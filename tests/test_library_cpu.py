@@ -1,0 +1,121 @@
+"""Host-only checks of libla2.so: it loads, exports what include/la2.h declares,
+and rejects bad arguments before touching the device (no GPU needed)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from linear_attention_la2_b200 import build as la2_build
+
+la2_build.build()
+from linear_attention_la2_b200 import la2  # noqa: E402
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+NULL = ctypes.c_void_p(0)
+
+
+def declared_symbols():
+    names = set()
+    inc = os.path.join(ROOT, "include")
+    for f in os.listdir(inc):
+        if f.endswith(".h"):
+            text = open(os.path.join(inc, f)).read()
+            names.update(re.findall(r"LA2_API[^;(]*?\b(la2_\w+)\s*\(", text))
+    return sorted(names)
+
+
+def test_header_declares_entry_points():
+    names = declared_symbols()
+    for required in ("la2_forward", "la2_backward", "la2_workspace_size", "la2_check",
+                     "la2_status_string"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(la2.LIB_PATH)
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+        assert name in la2.EXPORTED, name
+
+
+def test_status_strings():
+    for code in range(6):
+        s = la2.la2_status_string(code)
+        assert s.startswith("LA2_")
+    assert "unknown" in la2.la2_status_string(99)
+
+
+def _fwd(**kw):
+    args = dict(q=NULL, k=NULL, v=NULL, o=NULL, B=1, H=1, N=16, d=64, dv=64, causal=1, block=64,
+                dt=la2.LA2_F32, ws=NULL, wsb=0, stream=NULL)
+    args.update(kw)
+    return la2.la2_forward(args["q"], args["k"], args["v"], args["o"], args["B"], args["H"],
+                           args["N"], args["d"], args["dv"], args["causal"], args["block"],
+                           args["dt"], args["ws"], args["wsb"], args["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(B=-1), la2.LA2_ERR_INVALID_ARG),
+    (dict(N=-5), la2.LA2_ERR_INVALID_ARG),
+    (dict(d=0), la2.LA2_ERR_INVALID_ARG),
+    (dict(dv=0), la2.LA2_ERR_INVALID_ARG),
+    (dict(causal=2), la2.LA2_ERR_INVALID_ARG),
+    (dict(dt=7), la2.LA2_ERR_INVALID_ARG),
+    (dict(block=0), la2.LA2_ERR_INVALID_ARG),
+    (dict(block=48), la2.LA2_ERR_UNSUPPORTED),
+    (dict(d=129), la2.LA2_ERR_UNSUPPORTED),
+    (dict(dt=la2.LA2_BF16, d=96), la2.LA2_ERR_UNSUPPORTED),
+    (dict(dt=la2.LA2_BF16, block=32), la2.LA2_ERR_UNSUPPORTED),
+    (dict(d=128, dv=128, block=128), la2.LA2_ERR_UNSUPPORTED),  # fp32 tiles exceed smem
+    (dict(), la2.LA2_ERR_INVALID_ARG),  # NULL pointers
+    (dict(q=ctypes.c_void_p(0x1008), k=ctypes.c_void_p(0x2000), v=ctypes.c_void_p(0x3000),
+          o=ctypes.c_void_p(0x4000)), la2.LA2_ERR_INVALID_ARG),  # q not 16-byte aligned
+    (dict(q=ctypes.c_void_p(0x10000), k=ctypes.c_void_p(0x20000), v=ctypes.c_void_p(0x30000),
+          o=ctypes.c_void_p(0x10100)), la2.LA2_ERR_INVALID_ARG),  # o overlaps q
+])
+def test_forward_rejects_bad_arguments(kw, code):
+    assert _fwd(**kw) == code
+
+
+def test_empty_problem_is_a_noop():
+    for kw in (dict(B=0), dict(H=0), dict(N=0)):
+        assert _fwd(**kw) == la2.LA2_OK
+        assert la2.la2_workspace_size(kw.get("B", 1), kw.get("H", 1), kw.get("N", 16), 64, 64, 1,
+                                      64, la2.LA2_F32, 0) == 0
+
+
+def test_backward_rejects_bad_arguments():
+    b = la2.la2_backward
+    assert b(NULL, NULL, NULL, NULL, NULL, NULL, NULL, 1, 1, 16, 64, 64, 1, 64, la2.LA2_F32, NULL, 0,
+             NULL) == la2.LA2_ERR_INVALID_ARG
+    assert b(NULL, NULL, NULL, NULL, NULL, NULL, NULL, 1, 1, 16, 64, 64, 3, 64, la2.LA2_F32, NULL, 0,
+             NULL) == la2.LA2_ERR_INVALID_ARG
+    assert b(NULL, NULL, NULL, NULL, NULL, NULL, NULL, 0, 1, 16, 64, 64, 1, 64, la2.LA2_F32, NULL, 0,
+             NULL) == la2.LA2_OK
+    p = [ctypes.c_void_p(0x100000 * (i + 1)) for i in range(7)]
+    p[4] = ctypes.c_void_p(0x100000 + 64)  # dq overlaps q
+    assert b(*p, 1, 1, 16, 64, 64, 1, 64, la2.LA2_F32, NULL, 0, NULL) == la2.LA2_ERR_INVALID_ARG
+
+
+def test_workspace_size_rejects_bad_arguments():
+    bad = ctypes.c_size_t(-1).value
+    assert la2.la2_workspace_size(1, 1, 16, 64, 64, 5, 64, la2.LA2_F32, 0) == bad
+    assert la2.la2_num_chunks(1, 1, 16, 48, la2.LA2_BF16) == -1
+
+
+def test_settings_validation():
+    assert la2.la2_set_chunk_len(-1) == la2.LA2_ERR_INVALID_ARG
+    assert la2.la2_set_chunk_len(0) == la2.LA2_OK
+    assert la2.la2_set_spin_limit(-3) == la2.LA2_ERR_INVALID_ARG
+    assert la2.la2_set_spin_limit(0) == la2.LA2_OK
+
+
+def test_profiler_names():
+    n = la2.la2_profile_num_kernels()
+    assert n >= 5
+    names = [la2.la2_profile_kernel_name(i) for i in range(n)]
+    assert all(names) and len(set(names)) == n
+    assert la2.la2_profile_kernel_name(n) == ""
+    assert la2.la2_version() > 0
