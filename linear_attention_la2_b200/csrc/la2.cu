@@ -223,6 +223,67 @@ static la2_status backward_simt(const void* q, const void* k, const void* v, con
   return launch_status();
 }
 
+// Tensor-core forward: chunk states (if the sequence is split, or always for
+// the non-causal form), their scan, then the block loop from each chunk's
+// initial state.
+template <int BK>
+static la2_status forward_sm100_bk(const void* q, const void* k, const void* v, void* o,
+                                   int64_t BH, int64_t N, int causal, float* states,
+                                   const Plan& p, int64_t spin, cudaStream_t st) {
+  constexpr int D = 128, DV = 128;
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap_3d(&tq, q, BH, N, D, BK) || !make_tmap_3d(&tk, k, BH, N, D, BK) ||
+      !make_tmap_3d(&tv, v, BH, N, DV, BK))
+    return LA2_ERR_CUDA;
+  sm100::Params prm{};
+  prm.o = static_cast<__nv_bfloat16*>(o);
+  prm.N = N;
+  prm.L = p.L;
+  prm.C = p.C;
+  prm.spin_limit = spin;
+  la2_status s = LA2_OK;
+  const int nel = D * DV;
+  if (causal) {
+    if (p.C > 1) {
+      sm100::Params ps = prm;
+      ps.out_states = states;
+      ps.units_per_seq = p.C - 1;  // the last chunk's state is never needed
+      {
+        LaunchTimer t(K_STATE_TC, st);
+        s = launch_fwd_sm100<BK, D, DV, sm100::MODE_STATE>(tq, tk, tv, ps, BH * (p.C - 1), st);
+      }
+      if (s != LA2_OK) return s;
+      s = run_scan(states, BH, nel, p, 0, st);
+      if (s != LA2_OK) return s;
+      prm.init_states = states;
+    }
+    prm.units_per_seq = p.C;
+    LaunchTimer t(K_FWD_TC, st);
+    return launch_fwd_sm100<BK, D, DV, sm100::MODE_CAUSAL>(tq, tk, tv, prm, BH * p.C, st);
+  }
+  sm100::Params ps = prm;
+  ps.out_states = states;
+  ps.units_per_seq = p.C;
+  {
+    LaunchTimer t(K_STATE_TC, st);
+    s = launch_fwd_sm100<BK, D, DV, sm100::MODE_STATE>(tq, tk, tv, ps, BH * p.C, st);
+  }
+  if (s != LA2_OK) return s;
+  s = run_scan(states, BH, nel, p, 2, st);
+  if (s != LA2_OK) return s;
+  prm.init_states = states;
+  prm.units_per_seq = p.C;
+  LaunchTimer t(K_FWD_TC, st);
+  return launch_fwd_sm100<BK, D, DV, sm100::MODE_NONCAUSAL>(tq, tk, tv, prm, BH * p.C, st);
+}
+
+static la2_status forward_sm100(const void* q, const void* k, const void* v, void* o, int64_t BH,
+                                int64_t N, int causal, int block, float* states, const Plan& p,
+                                int64_t spin, cudaStream_t st) {
+  return block == 64 ? forward_sm100_bk<64>(q, k, v, o, BH, N, causal, states, p, spin, st)
+                     : forward_sm100_bk<128>(q, k, v, o, BH, N, causal, states, p, spin, st);
+}
+
 }  // namespace la2
 
 using namespace la2;
@@ -286,8 +347,7 @@ la2_status la2_forward(const void* q, const void* k, const void* v, void* o, int
   const int64_t BH = B * H;
   float* states = p.need_states ? static_cast<float*>(workspace) : nullptr;
   const int nel = (int)(d * dv);
-  if (p.tc) return sm100_forward(q, k, v, o, BH, N, (int)d, (int)dv, causal, block, states, p.L,
-                                 p.C, spin_limit(), st);
+  if (p.tc) return forward_sm100(q, k, v, o, BH, N, causal, block, states, p, spin_limit(), st);
   if (p.need_states) {
     s = dt == LA2_BF16
             ? run_chunk_states<__nv_bfloat16>(k, v, states, BH, N, (int)d, (int)dv, p, st)
@@ -353,9 +413,6 @@ la2_status la2_backward(const void* q, const void* k, const void* v, const void*
     s = run_scan(s_u, BH, nel, p, causal ? 1 : 2, st);
     if (s != LA2_OK) return s;
   }
-  if (p.tc)
-    return sm100_backward(q, k, v, dout, dq, dk, dvv, BH, N, (int)d, (int)dv, causal, block, s_kv,
-                          s_u, p.L, p.C, spin_limit(), st);
   return dt == LA2_BF16
              ? backward_simt<__nv_bfloat16>(q, k, v, dout, dq, dk, dvv, BH, N, (int)d, (int)dv,
                                             causal, block, s_kv, s_u, p, st)

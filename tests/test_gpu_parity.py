@@ -101,7 +101,7 @@ EDGE = [
     ("f32", 2, 3, 200, 32, 48, 32, 64),       # forced chunk split, ragged tail
     ("f32", 1, 1, 513, 64, 64, 64, 128),      # tail of one row in the last chunk
     ("f32", 1, 1, 300, 128, 128, 16, 0),
-    ("f32", 1, 1, 257, 64, 32, 128, 0),       # block 128 at small d
+    ("f32", 1, 1, 257, 32, 32, 128, 0),       # block 128 at small d
     ("bf16", 1, 1, 1, 128, 128, 64, 0),
     ("bf16", 1, 1, 63, 128, 128, 64, 0),      # N < block
     ("bf16", 1, 2, 65, 128, 128, 64, 0),      # one full block + one row
