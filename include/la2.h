@@ -151,6 +151,33 @@ LA2_API int la2_profile_num_kernels(void);
 LA2_API const char *la2_profile_kernel_name(int kernel);
 LA2_API la2_status la2_profile_collect(int kernel, int64_t *launches, double *total_ms);
 
+/*
+ * la2_forward_noalloc: la2_forward without a workspace argument. The article
+ * has no counterpart; this entry point exists for callers that cannot
+ * allocate device memory at the time they call the op (for example an
+ * operator hosted by a runtime that owns all device memory and offers no
+ * scratch space, or a serving loop that forbids allocations after start-up).
+ *
+ * The chunk states that la2_forward keeps in the caller's workspace live here
+ * in one array of LA2_NOALLOC_SCRATCH_BYTES (32 MiB) compiled into the
+ * library: every GPU on which the library is loaded holds that memory until
+ * the process exits. The first call on each device looks up the array's
+ * device address (cudaGetSymbolAddress, with that device current); make that
+ * first call before any stream capture. A problem whose workspace
+ * (la2_workspace_size(..., is_backward = 0)) exceeds the array returns
+ * LA2_ERR_WORKSPACE without launching anything; other arguments and errors are
+ * as for la2_forward. The call allocates nothing.
+ *
+ * All calls share the one array and it keeps the previous call's contents
+ * (every element a call reads it first writes). Calls that may overlap on the
+ * GPU - on different streams, or from host threads without ordering between
+ * them - race on the array and give wrong results: serialise them.
+ */
+#define LA2_NOALLOC_SCRATCH_BYTES (32u << 20)
+LA2_API la2_status la2_forward_noalloc(const void *q, const void *k, const void *v, void *o,
+                                       int64_t B, int64_t H, int64_t N, int64_t d, int64_t dv,
+                                       int causal, int block, la2_dtype dt, la2_stream_t stream);
+
 /* Library version, (major << 16) | minor. */
 LA2_API int la2_version(void);
 

@@ -477,3 +477,52 @@ la2_status la2_profile_collect(int kernel, int64_t* launches, double* total_ms) 
 int la2_version(void) { return (0 << 16) | 1; }
 
 }  // extern "C"
+
+// ============================================ forward without caller workspace
+//
+// For callers that cannot allocate device memory when they call the op: the
+// chunk states live in one array compiled into this library instead of a
+// caller-provided workspace. Host code cannot use the array's name as a device
+// address (it is only a host-side handle), so each device's address is looked
+// up once with cudaGetSymbolAddress, with that device current.
+
+namespace la2 {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[LA2_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kNoallocMaxDevices = 128;
+static void* g_noalloc_ptr[kNoallocMaxDevices];
+static std::mutex g_noalloc_mu;
+
+// Device address of the scratch array on the current device (set-up on first
+// use per device), or nullptr if the lookup fails.
+static void* noalloc_scratch_current_device() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoallocMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return nullptr;
+    g_noalloc_ptr[dev] = p;
+  }
+  return g_noalloc_ptr[dev];
+}
+
+}  // namespace la2
+
+extern "C" la2_status la2_forward_noalloc(const void* q, const void* k, const void* v, void* o,
+                                          int64_t B, int64_t H, int64_t N, int64_t d, int64_t dv,
+                                          int causal, int block, la2_dtype dt,
+                                          la2_stream_t stream) {
+  const size_t need = la2_workspace_size(B, H, N, d, dv, causal, block, dt, 0);
+  if (need == static_cast<size_t>(-1))  // let the regular entry point name the argument error
+    return la2_forward(q, k, v, o, B, H, N, d, dv, causal, block, dt, nullptr, 0, stream);
+  if (need > static_cast<size_t>(LA2_NOALLOC_SCRATCH_BYTES)) return LA2_ERR_WORKSPACE;
+  void* ws = nullptr;
+  if (need > 0) {
+    ws = noalloc_scratch_current_device();
+    if (!ws) return LA2_ERR_CUDA;
+  }
+  return la2_forward(q, k, v, o, B, H, N, d, dv, causal, block, dt, ws,
+                     static_cast<size_t>(LA2_NOALLOC_SCRATCH_BYTES), stream);
+}

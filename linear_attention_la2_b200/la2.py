@@ -53,6 +53,8 @@ _SIGS = {
     "la2_profile_kernel_name": (ctypes.c_char_p, [_int]),
     "la2_profile_collect": (_int, [_int, ctypes.POINTER(_i64), ctypes.POINTER(ctypes.c_double)]),
     "la2_version": (_int, []),
+    "la2_forward_noalloc": (_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _int, _int,
+                                   _int, _vp]),
 }
 
 EXPORTED = tuple(_SIGS)
@@ -73,6 +75,8 @@ la2_set_spin_limit = _lib.la2_set_spin_limit
 la2_profile_enable = _lib.la2_profile_enable
 la2_profile_num_kernels = _lib.la2_profile_num_kernels
 la2_version = _lib.la2_version
+la2_forward_noalloc = _lib.la2_forward_noalloc
+NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 def la2_status_string(code: int) -> str:
