@@ -114,21 +114,27 @@ LA2_API la2_status la2_check(la2_stream_t stream);
 LA2_API const char *la2_status_string(la2_status s);
 
 /*
- * Chunk plan. Sequences with few (b, h) pairs are split into chunks of
- * `chunk_len` rows that run in parallel from a prefix of per-chunk KV states
+ * Work split override. 0 (the default) lets the library split the work
+ * from B*H, N and the SM count (see la2_plan_ranges). A positive value cuts
+ * every sequence into chunks of `chunk_len` rows (rounded up to a multiple of
+ * `block`) that run in parallel from the sum of the earlier chunks' KV states
  * (a sum, so any split gives the same result up to fp32 rounding order).
- * 0 (the default) lets the library choose from B*H, N and the SM count; a
- * positive value is rounded up to a multiple of `block`. Process-wide; it
- * changes la2_workspace_size for later calls. Returns LA2_ERR_INVALID_ARG
- * for a negative value.
+ * Process-wide; it changes la2_workspace_size for later calls. Returns
+ * LA2_ERR_INVALID_ARG for a negative value.
  */
 LA2_API la2_status la2_set_chunk_len(int64_t chunk_len);
 
 /*
- * Number of chunks per (b, h) sequence the next call with these arguments
- * uses (1 = no split). -1 for arguments the call would reject.
+ * Work split the next call with these arguments uses. The (b, h) sequences are
+ * laid end to end as B*H*ceil(N/block) blocks; the call runs R ranges of that
+ * list in parallel, range r covering blocks [starts[r], starts[r+1]). A range
+ * that starts inside a sequence starts from the KV state of that sequence's
+ * earlier blocks. Returns R and, when cap >= R + 1, writes the R + 1 starts;
+ * returns -1 for arguments the call would reject.
  */
-LA2_API int64_t la2_num_chunks(int64_t B, int64_t H, int64_t N, int block, la2_dtype dt);
+LA2_API int64_t la2_plan_ranges(int64_t B, int64_t H, int64_t N, int64_t d, int64_t dv,
+                                int causal, int block, la2_dtype dt, int is_backward,
+                                int64_t *starts, int64_t cap);
 
 /*
  * Upper bound, in spin iterations, of every device-side wait (mbarrier or

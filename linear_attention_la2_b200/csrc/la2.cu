@@ -17,6 +17,7 @@
 #include "la2_common.cuh"
 #include "la2_simt.cuh"
 #include "la2_sm100.cuh"
+#include "la2_sm100_causal.cuh"
 
 namespace la2 {
 
@@ -79,10 +80,15 @@ constexpr int64_t kDefaultSpinLimit = int64_t(1) << 31;
 
 static int64_t spin_limit() { return g_spin_limit > 0 ? g_spin_limit : kDefaultSpinLimit; }
 
+constexpr int kMaxDevices = 128;
+
 static int device_sm_count() {
+  static int cached[kMaxDevices];
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  if (dev >= 0 && dev < kMaxDevices && cached[dev] > 0) return cached[dev];
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+  if (dev >= 0 && dev < kMaxDevices) cached[dev] = sms;
   return sms;
 }
 
@@ -94,6 +100,8 @@ struct Plan {
   bool tc = false;      // tensor-core (sm_100a) path
   bool need_states = false;
   size_t ws_bytes = 0;
+  bool ranges = false;  // persistent range split (tensor-core causal forward)
+  RangePlan rp;
 };
 
 static bool is_aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -128,8 +136,8 @@ static la2_status check_shape(int64_t B, int64_t H, int64_t N, int64_t d, int64_
   return LA2_OK;
 }
 
-static Plan make_plan(int64_t B, int64_t H, int64_t N, int64_t d, int64_t dv, int causal, int block,
-                      la2_dtype dt, bool is_bwd, int sms) {
+static Plan make_plan_uncached(int64_t B, int64_t H, int64_t N, int64_t d, int64_t dv, int causal,
+                               int block, la2_dtype dt, bool is_bwd, int sms) {
   Plan p;
   const int64_t BH = B * H;
   const int64_t T = (N + block - 1) / block;
@@ -146,11 +154,51 @@ static Plan make_plan(int64_t B, int64_t H, int64_t N, int64_t d, int64_t dv, in
     L = ((T + C - 1) / C) * block;
   }
   L = std::max<int64_t>(L, block);
+  if (p.tc && causal && !is_bwd) {
+    p.ranges = true;
+    p.rp = plan_ranges(BH, N, block, sms, g_chunk_len);
+    p.need_states = p.rp.prefix_mode == 1;
+    p.ws_bytes = p.need_states ? (size_t)p.rp.R * (size_t)d * (size_t)dv * sizeof(float) : 0;
+    return p;
+  }
   p.L = L;
   p.C = std::max<int64_t>(1, (N + L - 1) / L);
   p.need_states = (p.C > 1) || !causal;
   const size_t one = (size_t)BH * (size_t)p.C * (size_t)d * (size_t)dv * sizeof(float);
   p.ws_bytes = p.need_states ? one * (is_bwd ? 2 : 1) : 0;
+  return p;
+}
+
+// Plans are pure functions of the arguments, the split override and the SM
+// count; the range split is a small search, so recent plans are kept.
+struct PlanKey {
+  int64_t B, H, N, d, dv, chunk_len;
+  int causal, block, dt, is_bwd, sms;
+  bool operator==(const PlanKey& o) const {
+    return B == o.B && H == o.H && N == o.N && d == o.d && dv == o.dv && chunk_len == o.chunk_len &&
+           causal == o.causal && block == o.block && dt == o.dt && is_bwd == o.is_bwd && sms == o.sms;
+  }
+};
+
+static Plan make_plan(int64_t B, int64_t H, int64_t N, int64_t d, int64_t dv, int causal, int block,
+                      la2_dtype dt, bool is_bwd, int sms) {
+  constexpr int kSlots = 16;
+  static PlanKey keys[kSlots];
+  static Plan plans[kSlots];
+  static int used = 0, next_slot = 0;
+  static std::mutex mu;
+  const PlanKey k{B, H, N, d, dv, g_chunk_len, causal, block, static_cast<int>(dt), is_bwd ? 1 : 0, sms};
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < used; ++i)
+      if (keys[i] == k) return plans[i];
+  }
+  Plan p = make_plan_uncached(B, H, N, d, dv, causal, block, dt, is_bwd, sms);
+  std::lock_guard<std::mutex> lock(mu);
+  keys[next_slot] = k;
+  plans[next_slot] = p;
+  next_slot = (next_slot + 1) % kSlots;
+  used = used < kSlots ? used + 1 : kSlots;
   return p;
 }
 
@@ -244,22 +292,22 @@ static la2_status forward_sm100_bk(const void* q, const void* k, const void* v, 
   la2_status s = LA2_OK;
   const int nel = D * DV;
   if (causal) {
-    if (p.C > 1) {
-      sm100::Params ps = prm;
-      ps.out_states = states;
-      ps.units_per_seq = p.C - 1;  // the last chunk's state is never needed
-      {
-        LaunchTimer t(K_STATE_TC, st);
-        s = launch_fwd_sm100<BK, D, DV, sm100::MODE_STATE>(tq, tk, tv, ps, BH * (p.C - 1), st);
-      }
+    sm100::RangeTable rt;
+    if (!fill_range_table(p.rp, &rt)) return LA2_ERR_UNSUPPORTED;
+    sm100::CausalParams cp{};
+    cp.o = static_cast<__nv_bfloat16*>(o);
+    cp.agg = states;
+    cp.N = N;
+    cp.spin_limit = spin;
+    const int sms = device_sm_count();
+    const int grid = std::max(1, std::min(p.rp.R, sms));
+    if (p.rp.prefix_mode == 1) {
+      LaunchTimer t(K_STATE_TC, st);
+      s = launch_causal_sm100<BK, D, DV, sm100::KIND_AGG>(tq, tk, tv, rt, cp, grid, st);
       if (s != LA2_OK) return s;
-      s = run_scan(states, BH, nel, p, 0, st);
-      if (s != LA2_OK) return s;
-      prm.init_states = states;
     }
-    prm.units_per_seq = p.C;
     LaunchTimer t(K_FWD_TC, st);
-    return launch_fwd_sm100<BK, D, DV, sm100::MODE_CAUSAL>(tq, tk, tv, prm, BH * p.C, st);
+    return launch_causal_sm100<BK, D, DV, sm100::KIND_MAIN>(tq, tk, tv, rt, cp, grid, st);
   }
   sm100::Params ps = prm;
   ps.out_states = states;
@@ -301,13 +349,27 @@ size_t la2_workspace_size(int64_t B, int64_t H, int64_t N, int64_t d, int64_t dv
   return make_plan(B, H, N, d, dv, causal, block, dt, is_backward != 0, sms).ws_bytes;
 }
 
-int64_t la2_num_chunks(int64_t B, int64_t H, int64_t N, int block, la2_dtype dt) {
-  const int64_t d = 128, dv = 128;
-  if (check_shape(B, H, N, d, dv, 1, block, dt, false) != LA2_OK) return -1;
+int64_t la2_plan_ranges(int64_t B, int64_t H, int64_t N, int64_t d, int64_t dv, int causal,
+                        int block, la2_dtype dt, int is_backward, int64_t* starts, int64_t cap) {
+  if (check_shape(B, H, N, d, dv, causal, block, dt, is_backward != 0) != LA2_OK) return -1;
   if (B == 0 || H == 0 || N == 0) return 0;
   const int sms = device_sm_count();
   if (sms <= 0) return -1;
-  return make_plan(B, H, N, d, dv, 1, block, dt, false, sms).C;
+  const Plan p = make_plan(B, H, N, d, dv, causal, block, dt, is_backward != 0, sms);
+  const int64_t T = (N + block - 1) / block;
+  std::vector<int64_t> v;
+  if (p.ranges) {
+    v = p.rp.starts;
+  } else {
+    const int64_t per = p.L / block;
+    for (int64_t h = 0; h < B * H; ++h)
+      for (int64_t c = 0; c < p.C; ++c) v.push_back(h * T + c * per);
+    v.push_back(B * H * T);
+  }
+  const int64_t R = static_cast<int64_t>(v.size()) - 1;
+  if (starts && cap >= R + 1)
+    for (int64_t i = 0; i <= R; ++i) starts[i] = v[i];
+  return R;
 }
 
 la2_status la2_set_chunk_len(int64_t chunk_len) {
@@ -475,6 +537,13 @@ la2_status la2_profile_collect(int kernel, int64_t* launches, double* total_ms) 
 }
 
 int la2_version(void) { return (0 << 16) | 1; }
+
+#ifdef LA2_TRACE
+// Copies the per-step timestamps of CTA 0 of the last traced launch (16 x 512 u64).
+LA2_API int la2_trace_read(unsigned long long* dst) {
+  return cudaMemcpyFromSymbol(dst, sm100::g_trace, sizeof(sm100::g_trace)) == cudaSuccess ? 0 : 1;
+}
+#endif
 
 }  // extern "C"
 

@@ -87,22 +87,34 @@ chunk_scan_kernel(float* __restrict__ s, int64_t C, int nel, int mode) {
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
   if (e >= nel) return;
   float* p = s + (int64_t)blockIdx.y * C * nel + e;
+  constexpr int U = 8;  // independent loads in flight per thread
   float run = 0.f;
-  if (mode == 0) {
-    for (int64_t c = 0; c < C; ++c) {
-      const float x = p[c * nel];
-      p[c * nel] = run;
-      run += x;
+  if (mode == 2) {
+    for (int64_t c0 = 0; c0 < C; c0 += U) {
+      float x[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) x[u] = c0 + u < C ? p[(c0 + u) * nel] : 0.f;
+#pragma unroll
+      for (int u = 0; u < U; ++u) run += x[u];
     }
-  } else if (mode == 1) {
-    for (int64_t c = C - 1; c >= 0; --c) {
-      const float x = p[c * nel];
-      p[c * nel] = run;
-      run += x;
-    }
-  } else {
-    for (int64_t c = 0; c < C; ++c) run += p[c * nel];
     p[0] = run;
+    return;
+  }
+  for (int64_t i0 = 0; i0 < C; i0 += U) {
+    float x[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t i = i0 + u;
+      const int64_t c = mode == 0 ? i : C - 1 - i;
+      x[u] = i < C ? p[c * nel] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t i = i0 + u;
+      const int64_t c = mode == 0 ? i : C - 1 - i;
+      if (i < C) p[c * nel] = run;
+      run += x[u];
+    }
   }
 }
 

@@ -283,9 +283,12 @@ struct Bars {
 };
 
 // Bounded wait. Returns false (after recording a timeout and raising the
-// CTA abort flag) when the limit is reached or another role aborted.
-__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, int64_t limit,
-                                         volatile int* abort_flag, int where) {
+// CTA abort flag) when the limit is reached or another role aborted. The
+// common case - the phase has already completed - stays inline; the spin loop
+// and its timeout bookkeeping live out of line to keep every role's hot loop
+// small in the instruction cache.
+__device__ __noinline__ bool wait_bar_slow(uint64_t* bar, uint32_t parity, int64_t limit,
+                                           volatile int* abort_flag, int where) {
   int64_t n = 0;
   uint64_t deadline = 0;
   while (!mbar_try_wait(bar, parity)) {
@@ -302,6 +305,12 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, int64_t
     }
   }
   return true;
+}
+
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, int64_t limit,
+                                         volatile int* abort_flag, int where) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return wait_bar_slow(bar, parity, limit, abort_flag, where);
 }
 
 // Drain wait used after an abort: bounded by a fixed budget, never records.
@@ -711,6 +720,20 @@ inline bool sm100_supports(int64_t d, int64_t dv, int block, bool is_bwd) {
   return d == 128 && dv == 128 && (block == 64 || block == 128);
 }
 
+// Raises a kernel's dynamic shared-memory limit once per device (the
+// attribute is per function and per device context). `done` must be a
+// per-kernel flag array: every launcher below passes its own static one.
+template <typename Kernel>
+inline bool smem_attribute_set(Kernel kern, int bytes, bool (&done)[128]) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  if (dev >= 0 && dev < 128 && done[dev]) return true;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    return false;
+  if (dev >= 0 && dev < 128) done[dev] = true;
+  return true;
+}
+
 using PFN_encodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                      const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                      const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -751,9 +774,8 @@ inline la2_status launch_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk,
                                    cudaStream_t st) {
   using CF = sm100::Cfg<BK, D, DV>;
   auto kern = sm100::la2_fwd_sm100_kernel<BK, D, DV, MODE>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, CF::SMEM) !=
-      cudaSuccess)
-    return LA2_ERR_CUDA;
+  static bool attr_done[128];  // one per template instantiation
+  if (!smem_attribute_set(kern, CF::SMEM, attr_done)) return LA2_ERR_CUDA;
   kern<<<static_cast<unsigned>(units), sm100::kThreads, CF::SMEM, st>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? LA2_OK : LA2_ERR_CUDA;
 }

@@ -1,0 +1,803 @@
+// Persistent causal forward for sm_100a (tcgen05 + TMEM + TMA).
+//
+// Article "Lightning Attention-2 新一代注意力机制", section
+// "Lightning Attention-2简介", point 2 (Fig. 3): a block's output is the masked
+// left product inside the block plus the right product of its queries with the
+// KV state accumulated over the earlier blocks; point 3: tiles go HBM -> on-chip
+// -> HBM once.
+//
+// Work decomposition. The B*H sequences are laid end to end as one list of
+// (sequence, block) tasks of Bk rows. The host cuts that list into R contiguous
+// ranges (about one per SM, balanced by a cost model) and CTA j runs ranges
+// j, j+G, ... A range may cross sequence boundaries; it is processed as
+// segments, one per sequence it touches. A segment that starts at block 0
+// starts from a zero state. The first segment of a range may start inside a
+// sequence; its initial state is either
+//   * rebuilt by a pre-pass over the sequence's earlier blocks (K and V only,
+//     KV += K^T V, no output) - one launch, no workspace; or
+//   * the sum of the per-range states that la2_range_state (the same kernel,
+//     KIND_AGG) wrote for the earlier ranges of that sequence.
+//
+// Per main block (one CTA, warp-specialised):
+//   S   = Q K^T           tcgen05 M=Bk N=Bk K=d          TMEM
+//   P   = bf16(S ⊙ M_B)   mask warpgroup                  SMEM (K-major)
+//   KV += K^T V           tcgen05 M=d N=dv K=Bk          TMEM (fp32 state)
+//   O   = Q bf16(KV_old)  tcgen05 M=Bk N=dv K=d          TMEM (snapshot taken before the update)
+//   O  += P V             tcgen05 M=Bk N=dv K=Bk
+// The KV update is issued as soon as the snapshot of the old state is in SMEM,
+// so the next block's snapshot can start while this block's products run, and
+// S of the next block is issued before P V of this one.
+#pragma once
+
+#include "la2_sm100.cuh"
+
+namespace la2 {
+namespace sm100 {
+
+// Optional per-step timestamps of CTA 0 (globaltimer, ns) for pipeline
+// studies: build with -DLA2_TRACE and read them with la2_trace_read().
+#ifdef LA2_TRACE
+constexpr int kTraceEvents = 16, kTraceSteps = 512;
+__device__ unsigned long long g_trace[kTraceEvents][kTraceSteps];
+#define LA2_TRACE_POINT(ev, idx)                                                  \
+  do {                                                                            \
+    if (blockIdx.x == 0 && (idx) < kTraceSteps) g_trace[ev][idx] = globaltimer_ns(); \
+  } while (0)
+#else
+#define LA2_TRACE_POINT(ev, idx) \
+  do {                           \
+  } while (0)
+#endif
+
+// Issue S of the next block before P V of this one (needs a Q ring deeper than 1).
+constexpr bool kPrefetchS = false;
+
+constexpr int kMaxRanges = 1024;
+
+struct RangeTable {
+  int32_t R;            // number of ranges
+  int32_t prefix_mode;  // 0: pre-pass rebuilds a mid-sequence start; 1: sum of range states
+  int64_t T;            // blocks per sequence
+  int64_t starts[kMaxRanges + 1];  // range r = tasks [starts[r], starts[r+1])
+};
+
+struct CausalParams {
+  __nv_bfloat16* o;  // [BH][N][DV]
+  float* agg;        // range states [R][D][DV] (prefix_mode 1, or KIND_AGG output)
+  int64_t N;
+  int64_t spin_limit;
+};
+
+enum Kind : int { KIND_MAIN = 0, KIND_AGG = 1 };
+
+struct Step {
+  int64_t bh;
+  int32_t blk;
+  int32_t range;
+  uint8_t pre;        // K/V-only state step (pre-pass or range state)
+  uint8_t pre_first;  // first state step of a fresh state
+  uint8_t pre_last;   // last state step (its state is consumed next)
+  uint8_t seg_first;  // first main step of a segment
+  uint8_t seg_last;   // last main step of a segment
+  uint8_t init;       // seg_first: 0 zero state, 1 state from the pre-pass, 2 from range states
+};
+
+// Deterministic walk of this CTA's steps; every role runs its own copy.
+template <int KIND>
+struct StepIter {
+  const RangeTable* rt;
+  int32_t r;
+  int64_t f, fend;      // KIND_MAIN: next task / end of the current range
+  int64_t seg_end;      // end of the open segment (0 when none is open)
+  int64_t seg_lo;
+  int64_t bh;           // sequence of task f
+  int64_t blk;          // block of task f inside its sequence
+  uint8_t seg_init;
+  int64_t pre_bh;
+  int32_t pre_blk, pre_end, pre_lo;
+
+  __device__ __forceinline__ void begin(const RangeTable* t) {
+    rt = t;
+    r = static_cast<int32_t>(blockIdx.x) - static_cast<int32_t>(gridDim.x);
+    f = fend = 0;
+    seg_end = 0;
+    seg_lo = 0;
+    bh = blk = 0;
+    seg_init = 0;
+    pre_bh = 0;
+    pre_blk = pre_end = pre_lo = 0;
+  }
+
+  // Next step of this CTA; false when its ranges are exhausted. No recursion
+  // and one division per range, so every role can call it each step.
+  __device__ __forceinline__ bool next(Step& s) {
+    const int64_t T = rt->T;
+    if (pre_blk >= pre_end) {
+      if (KIND == KIND_AGG) {
+        // One state pass per range whose end falls inside a sequence.
+        bool found = false;
+        while (!found) {
+          r += static_cast<int32_t>(gridDim.x);
+          if (r >= rt->R - 1) return false;  // the last range's state is never needed
+          const int64_t e = rt->starts[r + 1];
+          const int64_t hb = (e - 1) / T;
+          if (e - hb * T == T) continue;  // ends on a sequence boundary
+          const int64_t lo = max(rt->starts[r], hb * T);
+          pre_bh = hb;
+          pre_lo = static_cast<int32_t>(lo - hb * T);
+          pre_blk = pre_lo;
+          pre_end = static_cast<int32_t>(e - hb * T);
+          found = true;
+        }
+      } else {
+        if (f >= fend) {
+          do {
+            r += static_cast<int32_t>(gridDim.x);
+            if (r >= rt->R) return false;
+            f = rt->starts[r];
+            fend = rt->starts[r + 1];
+          } while (f >= fend);
+          seg_end = 0;
+          bh = f / T;
+          blk = f - bh * T;
+        }
+        bool main_now = true;
+        if (seg_end == 0) {  // a segment opens at f
+          seg_lo = f;
+          seg_end = min(fend, f + (T - blk));
+          if (blk == 0) {
+            seg_init = 0;
+          } else if (rt->prefix_mode == 0) {
+            seg_init = 1;  // pre-pass over the sequence's earlier blocks first
+            pre_bh = bh;
+            pre_lo = 0;
+            pre_blk = 0;
+            pre_end = static_cast<int32_t>(blk);
+            main_now = false;
+          } else {
+            seg_init = 2;
+          }
+        }
+        if (main_now) {
+          s.bh = bh;
+          s.blk = static_cast<int32_t>(blk);
+          s.range = r;
+          s.pre = 0;
+          s.pre_first = s.pre_last = 0;
+          s.seg_first = f == seg_lo;
+          s.seg_last = f == seg_end - 1;
+          s.init = seg_init;
+          ++f;
+          if (++blk == T) {
+            blk = 0;
+            ++bh;
+          }
+          if (f == seg_end) seg_end = 0;
+          return true;
+        }
+      }
+    }
+    s.bh = pre_bh;
+    s.blk = pre_blk;
+    s.range = r;
+    s.pre = 1;
+    s.pre_first = pre_blk == pre_lo;
+    s.pre_last = pre_blk == pre_end - 1;
+    s.seg_first = s.seg_last = 0;
+    s.init = 0;
+    ++pre_blk;
+    return true;
+  }
+};
+
+template <int BK, int D, int DV>
+struct CCfg {
+  static constexpr int QS = BK == 64 ? 3 : 1;
+  static constexpr int KS = BK == 64 ? 3 : 2;
+  static constexpr int NSB = BK == 64 ? 2 : 1;    // S buffers (TMEM)
+  static constexpr int NPB = BK == 64 ? 2 : 1;    // P buffers (SMEM)
+  static constexpr int NSNAP = BK == 64 ? 2 : 1;  // KV snapshot buffers (SMEM)
+  static constexpr int DP = D / 64;
+  static constexpr int VP = DV / 64;
+  static constexpr int QTILE = BK * D * 2;
+  static constexpr int KTILE = BK * D * 2;
+  static constexpr int VTILE = BK * DV * 2;
+  static constexpr int PTILE = BK * BK * 2;
+  static constexpr int SNAP = D * DV * 2;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + QS * QTILE;
+  static constexpr int OFF_V = OFF_K + KS * KTILE;
+  static constexpr int OFF_P = OFF_V + KS * VTILE;
+  static constexpr int OFF_SNAP = OFF_P + NPB * PTILE;
+  static constexpr int OFF_BAR = OFF_SNAP + NSNAP * SNAP;
+  static constexpr int NBAR = 2 * QS + 2 * KS + 15;
+  static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
+  static constexpr uint32_t COL_KV = 0;
+  static constexpr uint32_t COL_O = 128;  // two buffers of 128 columns
+  static constexpr uint32_t COL_S = 384;  // NSB buffers of BK columns
+  static constexpr uint32_t ID_S = make_idesc(BK, BK, false, false);
+  static constexpr uint32_t ID_QKV = make_idesc(BK, DV, false, true);
+  static constexpr uint32_t ID_UPD = make_idesc(D, DV, true, true);
+  static constexpr uint32_t ID_PV = make_idesc(BK, DV, false, true);
+  static_assert(SMEM <= 227 * 1024, "shared memory budget");
+  static_assert(COL_S + NSB * BK <= kTmemCols, "TMEM budget");
+};
+
+template <int D>
+__device__ __forceinline__ void put_snap_row(uint32_t sbase, int r, const uint32_t* v, int col0) {
+#pragma unroll
+  for (int q4 = 0; q4 < 4; ++q4) {
+    const int col = col0 + q4 * 8;
+    const int panel = col >> 6, cj = (col & 63) >> 3;
+    st_shared_v4(sbase + panel * D * 128 + r * 128 + ((cj ^ (r & 7)) << 4),
+                 pack_bf16x2(__uint_as_float(v[q4 * 8 + 0]), __uint_as_float(v[q4 * 8 + 1])),
+                 pack_bf16x2(__uint_as_float(v[q4 * 8 + 2]), __uint_as_float(v[q4 * 8 + 3])),
+                 pack_bf16x2(__uint_as_float(v[q4 * 8 + 4]), __uint_as_float(v[q4 * 8 + 5])),
+                 pack_bf16x2(__uint_as_float(v[q4 * 8 + 6]), __uint_as_float(v[q4 * 8 + 7])));
+  }
+}
+
+// Row r of the state: sum over the earlier ranges of this sequence of their
+// range states (fp32, HBM), written to TMEM (fp32) and, rounded to bf16, to
+// the snapshot at `sbase`. Cold path (once per range), kept out of line.
+template <int D, int DV>
+__device__ __noinline__ void init_from_ranges(const float* agg, const RangeTable& rt, int32_t range,
+                                              int64_t head0, int r, uint32_t tKV, uint32_t sbase) {
+#pragma unroll 1
+  for (int c32 = 0; c32 < DV / 32; ++c32) {
+    float acc[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) acc[j] = 0.f;
+    if (r >= 0) {
+      for (int rr = range - 1; rr >= 0 && rt.starts[rr + 1] > head0; --rr) {
+        const float4* src = reinterpret_cast<const float4*>(
+            agg + static_cast<int64_t>(rr) * D * DV + static_cast<int64_t>(r) * DV + c32 * 32);
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4) {
+          const float4 x = src[q4];
+          acc[4 * q4] += x.x;
+          acc[4 * q4 + 1] += x.y;
+          acc[4 * q4 + 2] += x.z;
+          acc[4 * q4 + 3] += x.w;
+        }
+      }
+    }
+    uint32_t u[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) u[j] = __float_as_uint(acc[j]);
+    tmem_st32(tKV + c32 * 32, u);
+    if (r >= 0) put_snap_row<D>(sbase, r, u, c32 * 32);
+  }
+  tmem_st_wait();
+}
+
+template <int BK, int D, int DV, int KIND>
+__global__ void __launch_bounds__(kThreads, 1)
+la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
+                        const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v,
+                        const __grid_constant__ RangeTable rt, const CausalParams prm) {
+  using CF = CCfg<BK, D, DV>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int wg = warp >> 2;
+  const int w4 = warp & 3;
+
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + CF::OFF_BAR);
+  uint64_t* q_full = bar;
+  uint64_t* q_empty = q_full + CF::QS;
+  uint64_t* kv_full = q_empty + CF::QS;
+  uint64_t* kv_empty = kv_full + CF::KS;
+  uint64_t* s_full = kv_empty + CF::KS;
+  uint64_t* s_empty = s_full + 2;
+  uint64_t* p_full = s_empty + 2;
+  uint64_t* p_empty = p_full + 2;
+  uint64_t* snap_full = p_empty + 2;
+  uint64_t* snap_free = snap_full + 2;
+  uint64_t* o_full = snap_free + 2;
+  uint64_t* o_empty = o_full + 2;
+  uint64_t* kv_updated = o_empty + 2;
+  uint64_t* seg_ack = kv_updated + 1;
+  uint64_t* drain = seg_ack + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < CF::QS; ++s) { mbar_init(&q_full[s], 1); mbar_init(&q_empty[s], 1); }
+    for (int s = 0; s < CF::KS; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&s_full[s], 1);
+      mbar_init(&s_empty[s], 128);
+      mbar_init(&p_full[s], 128);
+      mbar_init(&p_empty[s], 1);
+      mbar_init(&snap_full[s], 128);
+      mbar_init(&snap_free[s], 1);
+      mbar_init(&o_full[s], 1);
+      mbar_init(&o_empty[s], 128);
+    }
+    mbar_init(kv_updated, 1);
+    mbar_init(seg_ack, 128);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == kWarpProducer && lane == 0) {
+    if (KIND == KIND_MAIN) tma_prefetch(&tm_q);
+    tma_prefetch(&tm_k);
+    tma_prefetch(&tm_v);
+  }
+  if (warp == kWarpMma) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int64_t lim = prm.spin_limit;
+
+  uint8_t* sQ = smem + CF::OFF_Q;
+  uint8_t* sK = smem + CF::OFF_K;
+  uint8_t* sV = smem + CF::OFF_V;
+  uint8_t* sP = smem + CF::OFF_P;
+  uint8_t* sSnap = smem + CF::OFF_SNAP;
+
+  if (warp == kWarpProducer) {
+    // ================================================================ TMA
+    if (lane == 0) {
+      StepIter<KIND> it;
+      it.begin(&rt);
+      Step st;
+      uint32_t g = 0, m = 0;
+      int issued_kv = 0, issued_q = 0;
+      bool ok = true;
+      while (ok && it.next(st)) {
+        const int row = st.blk * BK;
+        const int zz = static_cast<int>(st.bh);
+        const int ks = g % CF::KS;
+        if (!wait_bar(&kv_empty[ks], ((g / CF::KS) & 1) ^ 1, lim, abort_flag, 101)) { ok = false; break; }
+        LA2_TRACE_POINT(0, g);
+        mbar_expect_tx(&kv_full[ks], CF::KTILE + CF::VTILE);
+        for (int p = 0; p < CF::DP; ++p)
+          tma_load_3d(sK + ks * CF::KTILE + p * BK * 128, &tm_k, &kv_full[ks], 64 * p, row, zz);
+        for (int p = 0; p < CF::VP; ++p)
+          tma_load_3d(sV + ks * CF::VTILE + p * BK * 128, &tm_v, &kv_full[ks], 64 * p, row, zz);
+        ++issued_kv;
+        ++g;
+        if (!st.pre) {
+          const int qs = m % CF::QS;
+          if (!wait_bar(&q_empty[qs], ((m / CF::QS) & 1) ^ 1, lim, abort_flag, 102)) { ok = false; break; }
+          LA2_TRACE_POINT(1, m);
+          mbar_expect_tx(&q_full[qs], CF::QTILE);
+          for (int p = 0; p < CF::DP; ++p)
+            tma_load_3d(sQ + qs * CF::QTILE + p * BK * 128, &tm_q, &q_full[qs], 64 * p, row, zz);
+          ++issued_q;
+          ++m;
+        }
+      }
+      if (!ok) {
+        for (int j = max(0, issued_kv - CF::KS); j < issued_kv; ++j)
+          drain_wait(&kv_full[j % CF::KS], (j / CF::KS) & 1);
+        for (int j = max(0, issued_q - CF::QS); j < issued_q; ++j)
+          drain_wait(&q_full[j % CF::QS], (j / CF::QS) & 1);
+      }
+    }
+  } else if (warp == kWarpMma) {
+    // ================================================================ MMA
+    if (lane == 0) {
+      const uint32_t tKV = tmem + CF::COL_KV;
+      StepIter<KIND> it;
+      it.begin(&rt);
+      Step st, nx;
+      bool have = it.next(st);
+      uint32_t g = 0, m = 0, sn = 0, acks = 0;
+      bool ack_pending = false, s_ready = false, ok = true;
+
+      auto wait_ack = [&]() -> bool {
+        if (!ack_pending) return true;
+        if (!wait_bar(seg_ack, acks & 1, lim, abort_flag, 110)) return false;
+        ++acks;
+        ack_pending = false;
+        return true;
+      };
+      // Descriptor templates (start address 0); a tile's descriptor is the
+      // template plus its address >> 4, and a k-step adds its byte offset >> 4.
+      const uint64_t dK_mn = make_desc(0, BK * 128, 1024);   // MN-major, panels of BK rows
+      const uint64_t dKm = make_desc(0, 16, 1024);           // K-major
+      const uint64_t dSnap = make_desc(0, D * 128, 1024);    // MN-major, panels of D rows
+      const uint32_t sK0 = smem_u32(sK), sV0 = smem_u32(sV), sQ0 = smem_u32(sQ);
+      const uint32_t sP0 = smem_u32(sP), sS0 = smem_u32(sSnap);
+      auto update = [&](uint32_t slot, bool accumulate) {
+        const uint64_t a = dK_mn + ((sK0 + slot * CF::KTILE) >> 4);
+        const uint64_t b = dK_mn + ((sV0 + slot * CF::VTILE) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk)
+          mma_bf16_ss(tKV, a + kk * (2048 >> 4), b + kk * (2048 >> 4), CF::ID_UPD,
+                      (accumulate || kk > 0) ? 1u : 0u);
+      };
+      // S(mm) = Q K^T into S buffer mm % NSB; Q slot mm % QS, K slot gg % KS.
+      auto issue_s = [&](uint32_t mm, uint32_t gg) -> bool {
+        LA2_TRACE_POINT(5, mm);
+        if (!wait_bar(&q_full[mm % CF::QS], (mm / CF::QS) & 1, lim, abort_flag, 111)) return false;
+        if (!wait_bar(&kv_full[gg % CF::KS], (gg / CF::KS) & 1, lim, abort_flag, 112)) return false;
+        if (!wait_bar(&s_empty[mm % CF::NSB], ((mm / CF::NSB) & 1) ^ 1, lim, abort_flag, 113)) return false;
+        tc_fence_after();
+        const uint64_t a = dKm + ((sQ0 + (mm % CF::QS) * CF::QTILE) >> 4);
+        const uint64_t b = dKm + ((sK0 + (gg % CF::KS) * CF::KTILE) >> 4);
+        const uint32_t tS = tmem + CF::COL_S + (mm % CF::NSB) * BK;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = ((kk >> 2) * BK * 128 + (kk & 3) * 32) >> 4;
+          mma_bf16_ss(tS, a + off, b + off, CF::ID_S, kk > 0);
+        }
+        mma_commit(&s_full[mm % CF::NSB]);
+        LA2_TRACE_POINT(6, mm);
+        return true;
+      };
+
+      while (have && ok) {
+        const bool have_nx = it.next(nx);
+        const uint32_t ks = g % CF::KS;
+        if (st.pre) {
+          if (!wait_bar(&kv_full[ks], (g / CF::KS) & 1, lim, abort_flag, 114)) { ok = false; break; }
+          if (!wait_ack()) { ok = false; break; }
+          tc_fence_after();
+          update(ks, !st.pre_first);
+          if (st.pre_last) {
+            mma_commit(kv_updated);
+            if (KIND == KIND_AGG) ack_pending = true;
+          }
+          mma_commit(&kv_empty[ks]);
+        } else {
+          if (!s_ready && !issue_s(m, g)) { ok = false; break; }
+          s_ready = false;
+          const bool needs_snap = !(st.seg_first && st.init == 0);
+          const uint32_t sb = sn % CF::NSNAP;
+          if (needs_snap &&
+              !wait_bar(&snap_full[sb], (sn / CF::NSNAP) & 1, lim, abort_flag, 115)) { ok = false; break; }
+          if (!wait_ack()) { ok = false; break; }
+          LA2_TRACE_POINT(2, m);
+          const uint32_t ob = m & 1;
+          const uint32_t tO = tmem + CF::COL_O + ob * 128;
+          if (!wait_bar(&o_empty[ob], ((m >> 1) & 1) ^ 1, lim, abort_flag, 116)) { ok = false; break; }
+          tc_fence_after();
+          if (needs_snap) {
+            const uint64_t a = dKm + ((sQ0 + (m % CF::QS) * CF::QTILE) >> 4);
+            const uint64_t b = dSnap + ((sS0 + sb * CF::SNAP) >> 4);
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = ((kk >> 2) * BK * 128 + (kk & 3) * 32) >> 4;
+              mma_bf16_ss(tO, a + off, b + kk * (2048 >> 4), CF::ID_QKV, kk > 0);
+            }
+            mma_commit(&snap_free[sb]);
+            ++sn;
+          }
+          mma_commit(&q_empty[m % CF::QS]);
+          update(ks, needs_snap);
+          mma_commit(kv_updated);
+          if (st.seg_last) ack_pending = true;
+          const uint32_t pb = m % CF::NPB;
+          LA2_TRACE_POINT(3, m);
+          if (!wait_bar(&p_full[pb], (m / CF::NPB) & 1, lim, abort_flag, 117)) { ok = false; break; }
+          LA2_TRACE_POINT(4, m);
+          tc_fence_after();
+          {
+            const uint64_t a = dKm + ((sP0 + pb * CF::PTILE) >> 4);
+            const uint64_t b = dK_mn + ((sV0 + ks * CF::VTILE) >> 4);
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              const uint32_t off = ((kk >> 2) * BK * 128 + (kk & 3) * 32) >> 4;
+              mma_bf16_ss(tO, a + off, b + kk * (2048 >> 4), CF::ID_PV,
+                          (needs_snap || kk > 0) ? 1u : 0u);
+            }
+          }
+          mma_commit(&o_full[ob]);
+          mma_commit(&p_empty[pb]);
+          mma_commit(&kv_empty[ks]);
+          ++m;
+        }
+        ++g;
+        st = nx;
+        have = have_nx;
+      }
+      mma_commit(drain);
+      drain_wait(drain, 0);
+    }
+  } else if (wg == kWgMask) {
+    // ================================================ mask + convert S -> P
+    if (KIND == KIND_MAIN) {
+      const int r = acc_row<BK>(w4, lane);
+      const uint32_t lane_off = static_cast<uint32_t>(32 * w4) << 16;
+      StepIter<KIND> it;
+      it.begin(&rt);
+      Step st;
+      uint32_t m = 0;
+      while (it.next(st)) {
+        if (st.pre) continue;
+        const uint32_t sbuf = m % CF::NSB, pb = m % CF::NPB;
+        const uint32_t tS = tmem + CF::COL_S + sbuf * BK + lane_off;
+        if (!__all_sync(0xffffffffu, wait_bar(&s_full[sbuf], (m / CF::NSB) & 1, lim, abort_flag, 120))) break;
+        if (threadIdx.x % 128 == 0) LA2_TRACE_POINT(7, m);
+        if (!__all_sync(0xffffffffu, wait_bar(&p_empty[pb], ((m / CF::NPB) & 1) ^ 1, lim, abort_flag, 121))) break;
+        tc_fence_after();
+        const uint32_t pbase = smem_u32(sP + pb * CF::PTILE);
+#pragma unroll
+        for (int c32 = 0; c32 < BK / 32; ++c32) {
+          uint32_t v[32];
+          tmem_ld32(tS + c32 * 32, v);
+          tmem_ld_wait();
+          if (r >= 0) {
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              uint32_t w[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int col = c32 * 32 + q4 * 8 + 2 * e;
+                const float a = (col <= r) ? __uint_as_float(v[q4 * 8 + 2 * e]) : 0.f;
+                const float bb = (col + 1 <= r) ? __uint_as_float(v[q4 * 8 + 2 * e + 1]) : 0.f;
+                w[e] = pack_bf16x2(a, bb);
+              }
+              const int ch = c32 * 4 + q4;
+              const int panel = ch >> 3, cj = ch & 7;
+              st_shared_v4(pbase + panel * BK * 128 + r * 128 + ((cj ^ (r & 7)) << 4), w[0], w[1],
+                           w[2], w[3]);
+            }
+          }
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        mbar_arrive(&s_empty[sbuf]);
+        mbar_arrive(&p_full[pb]);
+        if (threadIdx.x % 128 == 0) LA2_TRACE_POINT(8, m);
+        ++m;
+      }
+    }
+  } else if (wg == kWgState) {
+    // ==================================================== KV state (snapshot)
+    const int r = acc_row<D>(w4, lane);  // state row
+    const uint32_t lane_off = static_cast<uint32_t>(32 * w4) << 16;
+    const uint32_t tKV = tmem + CF::COL_KV + lane_off;
+    StepIter<KIND> it;
+    it.begin(&rt);
+    Step st;
+    uint32_t sn = 0, kvu = 0;
+    bool ok = true;
+
+    auto wait_kvu = [&]() -> bool {
+      const bool w = __all_sync(0xffffffffu, wait_bar(kv_updated, kvu & 1, lim, abort_flag, 130));
+      ++kvu;
+      if (w) tc_fence_after();
+      return w;
+    };
+    auto snap_from_tmem = [&]() -> bool {
+      const uint32_t sb = sn % CF::NSNAP;
+      const uint32_t sbase = smem_u32(sSnap + sb * CF::SNAP);
+#pragma unroll
+      for (int c32 = 0; c32 < DV / 32; ++c32) {
+        uint32_t v[32];
+        tmem_ld32(tKV + c32 * 32, v);
+        tmem_ld_wait();
+        if (c32 == 0 &&
+            !__all_sync(0xffffffffu,
+                        wait_bar(&snap_free[sb], ((sn / CF::NSNAP) & 1) ^ 1, lim, abort_flag, 131)))
+          return false;
+        if (r >= 0) put_snap_row<D>(sbase, r, v, c32 * 32);
+      }
+      fence_proxy_async();
+      tc_fence_before();
+      mbar_arrive(&snap_full[sb]);
+      ++sn;
+      return true;
+    };
+    // Initial state = sum of the states of the earlier ranges of this sequence.
+    auto snap_from_ranges = [&](const Step& s) -> bool {
+      const uint32_t sb = sn % CF::NSNAP;
+      if (!__all_sync(0xffffffffu,
+                      wait_bar(&snap_free[sb], ((sn / CF::NSNAP) & 1) ^ 1, lim, abort_flag, 132)))
+        return false;
+      init_from_ranges<D, DV>(prm.agg, rt, s.range, s.bh * rt.T, r, tKV,
+                              smem_u32(sSnap + sb * CF::SNAP));
+      fence_proxy_async();
+      tc_fence_before();
+      mbar_arrive(&snap_full[sb]);
+      ++sn;
+      return true;
+    };
+
+    while (ok && it.next(st)) {
+      if (KIND == KIND_AGG) {
+        if (!st.pre_last) continue;
+        if (!wait_kvu()) break;
+        float* dst = prm.agg + static_cast<int64_t>(st.range) * D * DV;
+#pragma unroll
+        for (int c32 = 0; c32 < DV / 32; ++c32) {
+          uint32_t v[32];
+          tmem_ld32(tKV + c32 * 32, v);
+          tmem_ld_wait();
+          if (r >= 0) {
+            float4* p4 = reinterpret_cast<float4*>(dst + static_cast<int64_t>(r) * DV + c32 * 32);
+#pragma unroll
+            for (int q4 = 0; q4 < 8; ++q4)
+              p4[q4] = make_float4(__uint_as_float(v[4 * q4]), __uint_as_float(v[4 * q4 + 1]),
+                                   __uint_as_float(v[4 * q4 + 2]), __uint_as_float(v[4 * q4 + 3]));
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(seg_ack);
+        continue;
+      }
+      if (st.pre) continue;
+      if (st.seg_first) {
+        if (st.init == 1) {
+          if (!wait_kvu() || !snap_from_tmem()) break;
+        } else if (st.init == 2) {
+          if (!snap_from_ranges(st)) break;
+        }
+      } else {
+        if (!wait_kvu()) break;
+        if (threadIdx.x % 128 == 0) LA2_TRACE_POINT(9, sn);
+        if (!snap_from_tmem()) break;
+        if (threadIdx.x % 128 == 0) LA2_TRACE_POINT(10, sn - 1);
+      }
+      if (st.seg_last) {
+        if (!wait_kvu()) break;
+        tc_fence_before();
+        mbar_arrive(seg_ack);
+      }
+    }
+  } else if (wg == kWgEpilogue) {
+    // ========================================== O: TMEM -> bf16 -> HBM
+    if (KIND == KIND_MAIN) {
+      const int r = acc_row<BK>(w4, lane);
+      const uint32_t lane_off = static_cast<uint32_t>(32 * w4) << 16;
+      StepIter<KIND> it;
+      it.begin(&rt);
+      Step st;
+      uint32_t m = 0;
+      while (it.next(st)) {
+        if (st.pre) continue;
+        const uint32_t ob = m & 1;
+        const uint32_t tO = tmem + CF::COL_O + ob * 128 + lane_off;
+        if (!__all_sync(0xffffffffu, wait_bar(&o_full[ob], (m >> 1) & 1, lim, abort_flag, 140))) break;
+        if (threadIdx.x % 128 == 0) LA2_TRACE_POINT(11, m);
+        tc_fence_after();
+        const int64_t row = static_cast<int64_t>(st.blk) * BK + r;
+        const bool valid = r >= 0 && row < prm.N;
+        uint4* dst = reinterpret_cast<uint4*>(prm.o + (st.bh * prm.N + (valid ? row : 0)) * DV);
+#pragma unroll
+        for (int c32 = 0; c32 < DV / 32; ++c32) {
+          uint32_t v[32];
+          tmem_ld32(tO + c32 * 32, v);
+          tmem_ld_wait();
+          if (valid) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              dst[c32 * 4 + q] = make_uint4(
+                  pack_bf16x2(__uint_as_float(v[8 * q]), __uint_as_float(v[8 * q + 1])),
+                  pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3])),
+                  pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5])),
+                  pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7])));
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&o_empty[ob]);
+        if (threadIdx.x % 128 == 0) LA2_TRACE_POINT(12, m);
+        ++m;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kWarpMma) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace sm100
+
+// ------------------------------------------------------------------ host side
+
+// Cost model of the range split (in units of one main block): a pre-pass
+// block reads only K and V and issues one small MMA group.
+constexpr double kPrepassCost = 0.25;
+constexpr double kRangeStateCost = 0.35;  // separate state launch, per block
+constexpr double kLaunchCost = 1.0;       // one extra launch, in main blocks
+
+struct RangePlan {
+  int R = 0;
+  int prefix_mode = 0;
+  int64_t T = 0;
+  std::vector<int64_t> starts;
+  double makespan = 0.0;
+};
+
+// Greedy split of `total` tasks into ranges of cost <= tau; a range that
+// starts at block b of a sequence pays b pre-pass blocks. Returns the count.
+inline int greedy_ranges(int64_t total, int64_t T, double tau, std::vector<int64_t>* starts) {
+  int64_t f = 0;
+  int n = 0;
+  if (starts) starts->clear();
+  while (f < total) {
+    const int64_t blk = f % T;
+    const double budget = tau - static_cast<double>(blk) * kPrepassCost;
+    int64_t take = budget >= 1.0 ? static_cast<int64_t>(budget) : 1;
+    if (starts) starts->push_back(f);
+    f = std::min(total, f + take);
+    ++n;
+    if (n > sm100::kMaxRanges) return n;
+  }
+  if (starts) starts->push_back(total);
+  return n;
+}
+
+inline RangePlan plan_ranges(int64_t BH, int64_t N, int block, int sms, int64_t forced_len) {
+  RangePlan p;
+  const int64_t T = (N + block - 1) / block;
+  const int64_t total = BH * T;
+  p.T = T;
+  if (forced_len > 0) {
+    // fixed ranges of forced_len rows, never crossing a sequence; states from range sums
+    const int64_t per = std::max<int64_t>(1, forced_len / block);
+    p.prefix_mode = 1;
+    for (int64_t h = 0; h < BH; ++h)
+      for (int64_t b = 0; b < T; b += per) p.starts.push_back(h * T + b);
+    p.starts.push_back(total);
+    p.R = static_cast<int>(p.starts.size()) - 1;
+    return p;
+  }
+  const int G = std::max(1, sms);
+  // (a) pre-pass plan: smallest makespan tau whose greedy split fits in G ranges
+  double lo = std::max(1.0, static_cast<double>(total) / G), hi = static_cast<double>(total) + T;
+  for (int it = 0; it < 40; ++it) {
+    const double mid = 0.5 * (lo + hi);
+    if (greedy_ranges(total, T, mid, nullptr) <= G) hi = mid;
+    else lo = mid;
+  }
+  std::vector<int64_t> pre_starts;
+  const int n_pre = greedy_ranges(total, T, hi, &pre_starts);
+  const double tau_pre = hi;
+  // (b) range-state plan: equal split; a separate launch computes range states
+  const int n_eq = static_cast<int>(std::min<int64_t>(G, total));
+  const double tau_eq = static_cast<double>(total) / n_eq * (1.0 + kRangeStateCost) + kLaunchCost;
+  if (tau_pre <= tau_eq && n_pre <= sm100::kMaxRanges) {
+    p.prefix_mode = 0;
+    p.starts = pre_starts;
+    p.R = n_pre;
+    p.makespan = tau_pre;
+  } else {
+    p.prefix_mode = 1;
+    p.starts.resize(n_eq + 1);
+    for (int j = 0; j <= n_eq; ++j) p.starts[j] = total * j / n_eq;
+    p.R = n_eq;
+    p.makespan = tau_eq;
+  }
+  return p;
+}
+
+inline bool fill_range_table(const RangePlan& p, sm100::RangeTable* t) {
+  if (p.R < 1 || p.R > sm100::kMaxRanges) return false;
+  t->R = p.R;
+  t->prefix_mode = p.prefix_mode;
+  t->T = p.T;
+  for (int i = 0; i <= p.R; ++i) t->starts[i] = p.starts[i];
+  return true;
+}
+
+template <int BK, int D, int DV, int KIND>
+inline la2_status launch_causal_sm100(const CUtensorMap& tq, const CUtensorMap& tk,
+                                      const CUtensorMap& tv, const sm100::RangeTable& rt,
+                                      const sm100::CausalParams& p, int grid, cudaStream_t st) {
+  using CF = sm100::CCfg<BK, D, DV>;
+  auto kern = sm100::la2_causal_sm100_kernel<BK, D, DV, KIND>;
+  static bool attr_done[128];  // one per template instantiation
+  if (!smem_attribute_set(kern, CF::SMEM, attr_done)) return LA2_ERR_CUDA;
+  kern<<<static_cast<unsigned>(grid), sm100::kThreads, CF::SMEM, st>>>(tq, tk, tv, rt, p);
+  return cudaGetLastError() == cudaSuccess ? LA2_OK : LA2_ERR_CUDA;
+}
+
+}  // namespace la2

@@ -46,7 +46,8 @@ _SIGS = {
     "la2_check": (_int, [_vp]),
     "la2_status_string": (ctypes.c_char_p, [_int]),
     "la2_set_chunk_len": (_int, [_i64]),
-    "la2_num_chunks": (_i64, [_i64, _i64, _i64, _int, _int]),
+    "la2_plan_ranges": (_i64, [_i64, _i64, _i64, _i64, _i64, _int, _int, _int, _int,
+                               ctypes.POINTER(_i64), _i64]),
     "la2_set_spin_limit": (_int, [_i64]),
     "la2_profile_enable": (_int, [_int]),
     "la2_profile_num_kernels": (_int, []),
@@ -70,13 +71,24 @@ la2_forward = _lib.la2_forward
 la2_backward = _lib.la2_backward
 la2_check = _lib.la2_check
 la2_set_chunk_len = _lib.la2_set_chunk_len
-la2_num_chunks = _lib.la2_num_chunks
+la2_plan_ranges = _lib.la2_plan_ranges
 la2_set_spin_limit = _lib.la2_set_spin_limit
 la2_profile_enable = _lib.la2_profile_enable
 la2_profile_num_kernels = _lib.la2_profile_num_kernels
 la2_version = _lib.la2_version
 la2_forward_noalloc = _lib.la2_forward_noalloc
 NOALLOC_SCRATCH_BYTES = 32 << 20
+
+
+def plan_ranges(B, H, N, d, dv, causal, block, dtype_code, is_backward=False):
+    """Range starts (in blocks of the flattened B*H*ceil(N/block) list) the
+    library will use for these arguments."""
+    R = la2_plan_ranges(B, H, N, d, dv, int(causal), block, dtype_code, int(is_backward), None, 0)
+    if R < 0:
+        raise La2Error(LA2_ERR_INVALID_ARG)
+    buf = (_i64 * (R + 1))()
+    la2_plan_ranges(B, H, N, d, dv, int(causal), block, dtype_code, int(is_backward), buf, R + 1)
+    return list(buf)
 
 
 def la2_status_string(code: int) -> str:

@@ -173,9 +173,11 @@ def _sampled_and_blocked(la2, w, heads_full=None):
     against the float64 block algorithm (pinned to the left product)."""
     ins = la2_inputs.make_inputs(w)
     got = run_forward(la2, ins, True, w.block)
-    nchunk = la2.la2_num_chunks(w.B, w.H, w.N, w.block, 1)
-    chunk = -(-w.N // nchunk) if nchunk > 1 else None
-    rows = la2_inputs.sample_rows(w.N, w.block, w.seed, chunk=chunk)
+    T = -(-w.N // w.block)
+    starts = la2.plan_ranges(w.B, w.H, w.N, w.d, w.dv, True, w.block, la2.LA2_BF16)
+    # rows on both sides of every range boundary inside a sequence
+    edges = {r for f in starts[1:-1] if f % T for r in ((f % T) * w.block - 1, (f % T) * w.block)}
+    rows = sorted(set(la2_inputs.sample_rows(w.N, w.block, w.seed)) | edges)
     ref_rows = oracle.forward_rows(ins["q"], ins["k"], ins["v"], rows, True)
     assert rel(got[:, :, rows], ref_rows) <= TOL["bf16"]
     for r_i, r in enumerate(rows[:: max(1, len(rows) // 64)]):

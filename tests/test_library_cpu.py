@@ -102,7 +102,7 @@ def test_backward_rejects_bad_arguments():
 def test_workspace_size_rejects_bad_arguments():
     bad = ctypes.c_size_t(-1).value
     assert la2.la2_workspace_size(1, 1, 16, 64, 64, 5, 64, la2.LA2_F32, 0) == bad
-    assert la2.la2_num_chunks(1, 1, 16, 48, la2.LA2_BF16) == -1
+    assert la2.la2_plan_ranges(1, 1, 16, 128, 128, 1, 48, la2.LA2_BF16, 0, None, 0) == -1
 
 
 def test_settings_validation():
