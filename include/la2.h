@@ -119,8 +119,10 @@ LA2_API const char *la2_status_string(la2_status s);
  * every sequence into chunks of `chunk_len` rows (rounded up to a multiple of
  * `block`) that run in parallel from the sum of the earlier chunks' KV states
  * (a sum, so any split gives the same result up to fp32 rounding order).
- * Process-wide; it changes la2_workspace_size for later calls. Returns
- * LA2_ERR_INVALID_ARG for a negative value.
+ * Process-wide; it changes la2_workspace_size for later calls. A forced split
+ * of the tensor-core causal forward into more than 160 chunks in total gives
+ * LA2_ERR_UNSUPPORTED at the call. Returns LA2_ERR_INVALID_ARG for a negative
+ * value.
  */
 LA2_API la2_status la2_set_chunk_len(int64_t chunk_len);
 

@@ -52,7 +52,7 @@ __device__ unsigned long long g_trace[kTraceEvents][kTraceSteps];
 // Issue S of the next block before P V of this one (needs a Q ring deeper than 1).
 constexpr bool kPrefetchS = false;
 
-constexpr int kMaxRanges = 1024;
+constexpr int kMaxRanges = 160;  // the range table travels as a kernel parameter (< 4 KB)
 
 struct RangeTable {
   int32_t R;            // number of ranges
