@@ -331,12 +331,24 @@ def bench_workload(args, w, dev, la2, world, rank, local, hbm, peak_kind, main):
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
     st = la2._stream_handle(stream)
 
+    if w.backward:  # one step = forward + backward of the same batch
+        dO = I.make_inputs(w, with_grad_out=True)["do"].to(dev)
+        grads = tuple(torch.empty_like(sets[0][0]) for _ in range(3))
+        wsb_bytes = la2.workspace_bytes(w.B, w.H, w.N, w.d, w.dv, True, w.block, dt, True)
+        wsb = torch.empty(max(wsb_bytes, 1), dtype=torch.uint8, device=dev)
+
     def step(i):
         q, k, v, o = sets[i % nsets]
         rc = la2.la2_forward(la2._ptr(q), la2._ptr(k), la2._ptr(v), la2._ptr(o), w.B, w.H, w.N, w.d,
                              w.dv, 1, w.block, dt, la2._ptr(ws), ws_bytes, st)
         if rc != 0:
             raise la2.La2Error(rc)
+        if w.backward:
+            rc = la2.la2_backward(la2._ptr(q), la2._ptr(k), la2._ptr(v), la2._ptr(dO),
+                                  la2._ptr(grads[0]), la2._ptr(grads[1]), la2._ptr(grads[2]), w.B,
+                                  w.H, w.N, w.d, w.dv, 1, w.block, dt, la2._ptr(wsb), wsb_bytes, st)
+            if rc != 0:
+                raise la2.La2Error(rc)
 
     for i in range(args.warmup):
         step(i)
@@ -399,7 +411,10 @@ def bench_workload(args, w, dev, la2, world, rank, local, hbm, peak_kind, main):
     }
     if clocks:
         line["clocks"] = clocks
-    if main and not args.no_e2e:
+    if w.backward:
+        line["metric"] = "causal linear-attn fwd+bwd tokens/s (B·H·N/s), 1 B200"
+        line["config"]["workload"] += " (+ backward)"
+    if main and not args.no_e2e and not w.backward:
         line["e2e"] = e2e_measure(args, w, dev, la2, world, base, ws, ws_bytes, dt)
     if main and rank == 0 and world == 1 and not args.no_cpu_baseline:
         r, sample, cores = cpu_oracle_rate(w, budget_s=10.0)

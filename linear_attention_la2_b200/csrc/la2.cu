@@ -18,6 +18,7 @@
 #include "la2_simt.cuh"
 #include "la2_sm100.cuh"
 #include "la2_sm100_causal.cuh"
+#include "la2_sm100_bwd.cuh"
 
 namespace la2 {
 
@@ -128,9 +129,10 @@ static la2_status check_shape(int64_t B, int64_t H, int64_t N, int64_t d, int64_
     if (d > 128 || dv > 128) return LA2_ERR_UNSUPPORTED;
     if (block != 16 && block != 32 && block != 64 && block != 128) return LA2_ERR_UNSUPPORTED;
   }
-  const size_t smem = is_bwd ? std::max(bwd_dq_simt_smem((int)d, (int)dv, block),
-                                        bwd_dkdv_simt_smem((int)d, (int)dv, block))
-                             : fwd_simt_smem((int)d, (int)dv, block);
+  const size_t es = dt == LA2_BF16 ? 2 : 4;
+  const size_t smem = is_bwd ? std::max(bwd_dq_simt_smem((int)d, (int)dv, block, es),
+                                        bwd_dkdv_simt_smem((int)d, (int)dv, block, es))
+                             : fwd_simt_smem((int)d, (int)dv, block, es);
   const bool tc = (dt == LA2_BF16) && sm100_supports(d, dv, block, is_bwd);
   if (!tc && smem > 227 * 1024) return LA2_ERR_UNSUPPORTED;
   return LA2_OK;
@@ -230,7 +232,7 @@ template <typename T>
 static la2_status forward_simt(const void* q, const void* k, const void* v, void* o, int64_t BH,
                                int64_t N, int d, int dv, int causal, int block, float* states,
                                const Plan& p, cudaStream_t st) {
-  const size_t smem = fwd_simt_smem(d, dv, block);
+  const size_t smem = fwd_simt_smem(d, dv, block, sizeof(T));
   if (cudaFuncSetAttribute(fwd_simt_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
     return LA2_ERR_CUDA;
@@ -246,8 +248,8 @@ static la2_status backward_simt(const void* q, const void* k, const void* v, con
                                 void* dq, void* dk, void* dvv, int64_t BH, int64_t N, int d,
                                 int dv, int causal, int block, float* s_kv, float* s_u,
                                 const Plan& p, cudaStream_t st) {
-  const size_t smem_q = bwd_dq_simt_smem(d, dv, block);
-  const size_t smem_kv = bwd_dkdv_simt_smem(d, dv, block);
+  const size_t smem_q = bwd_dq_simt_smem(d, dv, block, sizeof(T));
+  const size_t smem_kv = bwd_dkdv_simt_smem(d, dv, block, sizeof(T));
   if (cudaFuncSetAttribute(bwd_dq_simt_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem_q) != cudaSuccess ||
       cudaFuncSetAttribute(bwd_dkdv_simt_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -323,6 +325,73 @@ static la2_status forward_sm100_bk(const void* q, const void* k, const void* v, 
   prm.units_per_seq = p.C;
   LaunchTimer t(K_FWD_TC, st);
   return launch_fwd_sm100<BK, D, DV, sm100::MODE_NONCAUSAL>(tq, tk, tv, prm, BH * p.C, st);
+}
+
+// Tensor-core backward: chunk states K^T V (prefix for dQ) and Q^T dO
+// (suffix for dK, dV), their scans, then the dQ pass (the block loop with
+// dO, V, K in the Q, K, V slots) and the reverse dK/dV pass.
+template <int BK>
+static la2_status backward_sm100_bk(const void* q, const void* k, const void* v, const void* dout,
+                                    void* dq, void* dk, void* dvv, int64_t BH, int64_t N,
+                                    int causal, float* s_kv, float* s_u, const Plan& p,
+                                    int64_t spin, cudaStream_t st) {
+  constexpr int D = 128, DV = 128;
+  CUtensorMap tq, tk, tv, tdo;
+  if (!make_tmap_3d(&tq, q, BH, N, D, BK) || !make_tmap_3d(&tk, k, BH, N, D, BK) ||
+      !make_tmap_3d(&tv, v, BH, N, DV, BK) || !make_tmap_3d(&tdo, dout, BH, N, DV, BK))
+    return LA2_ERR_CUDA;
+  la2_status s = LA2_OK;
+  const int nel = D * DV;
+  const bool states = p.need_states;
+  if (states) {
+    sm100::Params ps{};
+    ps.N = N;
+    ps.L = p.L;
+    ps.C = p.C;
+    ps.units_per_seq = p.C;
+    ps.spin_limit = spin;
+    {
+      LaunchTimer t(K_STATE_TC, st);
+      ps.out_states = s_kv;  // K^T V per chunk
+      s = launch_fwd_sm100<BK, D, DV, sm100::MODE_STATE>(tq, tk, tv, ps, BH * p.C, st);
+    }
+    if (s != LA2_OK) return s;
+    {
+      LaunchTimer t(K_STATE_TC, st);
+      ps.out_states = s_u;  // Q^T dO per chunk
+      s = launch_fwd_sm100<BK, D, DV, sm100::MODE_STATE>(tq, tq, tdo, ps, BH * p.C, st);
+    }
+    if (s != LA2_OK) return s;
+    s = run_scan(s_kv, BH, nel, p, causal ? 0 : 2, st);
+    if (s != LA2_OK) return s;
+    s = run_scan(s_u, BH, nel, p, causal ? 1 : 2, st);
+    if (s != LA2_OK) return s;
+  }
+  sm100::Params pq{};
+  pq.o = static_cast<__nv_bfloat16*>(dq);
+  pq.init_states = states ? s_kv : nullptr;
+  pq.N = N;
+  pq.L = p.L;
+  pq.C = p.C;
+  pq.units_per_seq = p.C;
+  pq.spin_limit = spin;
+  {
+    LaunchTimer t(K_BWD_DQ_TC, st);
+    s = causal ? launch_fwd_sm100<BK, D, DV, sm100::MODE_CAUSAL, true>(tdo, tv, tk, pq, BH * p.C, st)
+               : launch_fwd_sm100<BK, D, DV, sm100::MODE_NONCAUSAL, true>(tdo, tv, tk, pq, BH * p.C, st);
+  }
+  if (s != LA2_OK) return s;
+  sm100::BwdParams pb{};
+  pb.dk = static_cast<__nv_bfloat16*>(dk);
+  pb.dv = static_cast<__nv_bfloat16*>(dvv);
+  pb.init_u = states ? s_u : nullptr;
+  pb.N = N;
+  pb.L = p.L;
+  pb.C = p.C;
+  pb.spin_limit = spin;
+  pb.causal = causal;
+  LaunchTimer t(K_BWD_DKDV_TC, st);
+  return launch_bwd_dkdv_sm100<BK>(tq, tk, tv, tdo, pb, BH * p.C, st);
 }
 
 static la2_status forward_sm100(const void* q, const void* k, const void* v, void* o, int64_t BH,
@@ -462,6 +531,11 @@ la2_status la2_backward(const void* q, const void* k, const void* v, const void*
   const int nel = (int)(d * dv);
   float* s_kv = p.need_states ? static_cast<float*>(workspace) : nullptr;
   float* s_u = p.need_states ? s_kv + (size_t)BH * p.C * nel : nullptr;
+  if (p.tc)
+    return block == 64 ? backward_sm100_bk<64>(q, k, v, dout, dq, dk, dvv, BH, N, causal, s_kv, s_u,
+                                                p, spin_limit(), st)
+                       : backward_sm100_bk<128>(q, k, v, dout, dq, dk, dvv, BH, N, causal, s_kv,
+                                                 s_u, p, spin_limit(), st);
   if (p.need_states) {
     const bool bf = dt == LA2_BF16;
     s = bf ? run_chunk_states<__nv_bfloat16>(k, v, s_kv, BH, N, (int)d, (int)dv, p, st)

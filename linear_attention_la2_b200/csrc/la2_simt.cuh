@@ -119,11 +119,13 @@ chunk_scan_kernel(float* __restrict__ s, int64_t C, int nel, int mode) {
 }
 
 // Shared-memory helpers: load `rows` rows of a [*, w] tile, zero the rest.
+// Tiles stay in the input type T (fp32 inputs: fp32; bf16 inputs: bf16);
+// every product is accumulated in fp32.
 template <typename T>
-__device__ __forceinline__ void load_tile(float* dst, const T* src, int rows, int Bk, int w) {
+__device__ __forceinline__ void load_tile(T* dst, const T* src, int rows, int Bk, int w) {
   for (int i = threadIdx.x; i < Bk * w; i += blockDim.x) {
     const int r = i / w;
-    dst[i] = r < rows ? to_f32(src[i]) : 0.f;
+    dst[i] = r < rows ? src[i] : from_f32<T>(0.f);
   }
 }
 
@@ -144,10 +146,10 @@ fwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
                 int Bk, int64_t L, int64_t C, int causal) {
   extern __shared__ float smem[];
   float* KV = smem;
-  float* Qs = KV + d * dv;
-  float* Ks = Qs + Bk * d;
-  float* Vs = Ks + Bk * d;
-  float* S = Vs + Bk * dv;
+  T* Qs = reinterpret_cast<T*>(KV + d * dv);
+  T* Ks = Qs + Bk * d;
+  T* Vs = Ks + Bk * d;
+  T* S = Vs + Bk * dv;  // masked (Q K^T) block, rounded to T
   const int64_t unit = blockIdx.x;
   const int64_t bh = unit / C, c = unit % C;
   const int64_t t0 = c * L, t1 = imin64(N, t0 + L);
@@ -174,8 +176,8 @@ fwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
         const int t = i / Bk, j = i % Bk;
         float s = 0.f;
         if (j <= t)
-          for (int cc = 0; cc < d; ++cc) s = fmaf(Qs[t * d + cc], Ks[j * d + cc], s);
-        S[i] = s;  // M_B: lower-triangular ones, diagonal kept
+          for (int cc = 0; cc < d; ++cc) s = fmaf(to_f32(Qs[t * d + cc]), to_f32(Ks[j * d + cc]), s);
+        S[i] = from_f32<T>(s);  // M_B: lower-triangular ones, diagonal kept
       }
       __syncthreads();
     }
@@ -183,8 +185,8 @@ fwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
       const int t = i / dv, e = i % dv;
       float acc = 0.f;
       if (causal)
-        for (int j = 0; j <= t; ++j) acc = fmaf(S[t * Bk + j], Vs[j * dv + e], acc);
-      for (int cc = 0; cc < d; ++cc) acc = fmaf(Qs[t * d + cc], KV[cc * dv + e], acc);
+        for (int j = 0; j <= t; ++j) acc = fmaf(to_f32(S[t * Bk + j]), to_f32(Vs[j * dv + e]), acc);
+      for (int cc = 0; cc < d; ++cc) acc = fmaf(to_f32(Qs[t * d + cc]), KV[cc * dv + e], acc);
       ob[(i0 + t) * dv + e] = from_f32<T>(acc);
     }
     __syncthreads();
@@ -192,7 +194,7 @@ fwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
       for (int i = threadIdx.x; i < d * dv; i += blockDim.x) {
         const int cc = i / dv, e = i % dv;
         float acc = KV[i];
-        for (int t = 0; t < rows; ++t) acc = fmaf(Ks[t * d + cc], Vs[t * dv + e], acc);
+        for (int t = 0; t < rows; ++t) acc = fmaf(to_f32(Ks[t * d + cc]), to_f32(Vs[t * dv + e]), acc);
         KV[i] = acc;
       }
       __syncthreads();
@@ -213,10 +215,10 @@ bwd_dq_simt_kernel(const T* __restrict__ k, const T* __restrict__ v, const T* __
                    int Bk, int64_t L, int64_t C, int causal) {
   extern __shared__ float smem[];
   float* KV = smem;
-  float* dOs = KV + d * dv;
-  float* Vs = dOs + Bk * dv;
-  float* Ks = Vs + Bk * dv;
-  float* A = Ks + Bk * d;
+  T* dOs = reinterpret_cast<T*>(KV + d * dv);
+  T* Vs = dOs + Bk * dv;
+  T* Ks = Vs + Bk * dv;
+  T* A = Ks + Bk * d;  // masked (dO V^T) block, rounded to T
   const int64_t unit = blockIdx.x;
   const int64_t bh = unit / C, c = unit % C;
   const int64_t t0 = c * L, t1 = imin64(N, t0 + L);
@@ -243,8 +245,8 @@ bwd_dq_simt_kernel(const T* __restrict__ k, const T* __restrict__ v, const T* __
         const int t = i / Bk, j = i % Bk;
         float s = 0.f;
         if (j <= t)
-          for (int e = 0; e < dv; ++e) s = fmaf(dOs[t * dv + e], Vs[j * dv + e], s);
-        A[i] = s;
+          for (int e = 0; e < dv; ++e) s = fmaf(to_f32(dOs[t * dv + e]), to_f32(Vs[j * dv + e]), s);
+        A[i] = from_f32<T>(s);
       }
       __syncthreads();
     }
@@ -252,8 +254,8 @@ bwd_dq_simt_kernel(const T* __restrict__ k, const T* __restrict__ v, const T* __
       const int t = i / d, cc = i % d;
       float acc = 0.f;
       if (causal)
-        for (int j = 0; j <= t; ++j) acc = fmaf(A[t * Bk + j], Ks[j * d + cc], acc);
-      for (int e = 0; e < dv; ++e) acc = fmaf(dOs[t * dv + e], KV[cc * dv + e], acc);
+        for (int j = 0; j <= t; ++j) acc = fmaf(to_f32(A[t * Bk + j]), to_f32(Ks[j * d + cc]), acc);
+      for (int e = 0; e < dv; ++e) acc = fmaf(to_f32(dOs[t * dv + e]), KV[cc * dv + e], acc);
       dqb[(i0 + t) * d + cc] = from_f32<T>(acc);
     }
     __syncthreads();
@@ -261,7 +263,7 @@ bwd_dq_simt_kernel(const T* __restrict__ k, const T* __restrict__ v, const T* __
       for (int i = threadIdx.x; i < d * dv; i += blockDim.x) {
         const int cc = i / dv, e = i % dv;
         float acc = KV[i];
-        for (int t = 0; t < rows; ++t) acc = fmaf(Ks[t * d + cc], Vs[t * dv + e], acc);
+        for (int t = 0; t < rows; ++t) acc = fmaf(to_f32(Ks[t * d + cc]), to_f32(Vs[t * dv + e]), acc);
         KV[i] = acc;
       }
       __syncthreads();
@@ -284,12 +286,12 @@ bwd_dkdv_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* 
                      int64_t L, int64_t C, int causal) {
   extern __shared__ float smem[];
   float* U = smem;
-  float* Qs = U + d * dv;
-  float* Ks = Qs + Bk * d;
-  float* Vs = Ks + Bk * d;
-  float* dOs = Vs + Bk * dv;
-  float* A = dOs + Bk * dv;
-  float* P = A + Bk * Bk;
+  T* Qs = reinterpret_cast<T*>(U + d * dv);
+  T* Ks = Qs + Bk * d;
+  T* Vs = Ks + Bk * d;
+  T* dOs = Vs + Bk * dv;
+  T* A = dOs + Bk * dv;  // masked (dO V^T) block, rounded to T
+  T* P = A + Bk * Bk;    // masked (Q K^T) block, rounded to T
   const int64_t unit = blockIdx.x;
   const int64_t bh = unit / C, c = unit % C;
   const int64_t t0 = c * L, t1 = imin64(N, t0 + L);
@@ -321,11 +323,11 @@ bwd_dkdv_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* 
         const int t = i / Bk, j = i % Bk;  // t: query row, j: key row
         float a = 0.f, p = 0.f;
         if (j <= t) {
-          for (int e = 0; e < dv; ++e) a = fmaf(dOs[t * dv + e], Vs[j * dv + e], a);
-          for (int cc = 0; cc < d; ++cc) p = fmaf(Qs[t * d + cc], Ks[j * d + cc], p);
+          for (int e = 0; e < dv; ++e) a = fmaf(to_f32(dOs[t * dv + e]), to_f32(Vs[j * dv + e]), a);
+          for (int cc = 0; cc < d; ++cc) p = fmaf(to_f32(Qs[t * d + cc]), to_f32(Ks[j * d + cc]), p);
         }
-        A[i] = a;
-        P[i] = p;
+        A[i] = from_f32<T>(a);
+        P[i] = from_f32<T>(p);
       }
       __syncthreads();
     }
@@ -333,16 +335,16 @@ bwd_dkdv_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* 
       const int j = i / d, cc = i % d;
       float acc = 0.f;
       if (causal)
-        for (int t = j; t < rows; ++t) acc = fmaf(A[t * Bk + j], Qs[t * d + cc], acc);
-      for (int e = 0; e < dv; ++e) acc = fmaf(Vs[j * dv + e], U[cc * dv + e], acc);
+        for (int t = j; t < rows; ++t) acc = fmaf(to_f32(A[t * Bk + j]), to_f32(Qs[t * d + cc]), acc);
+      for (int e = 0; e < dv; ++e) acc = fmaf(to_f32(Vs[j * dv + e]), U[cc * dv + e], acc);
       dkb[(i0 + j) * d + cc] = from_f32<T>(acc);
     }
     for (int i = threadIdx.x; i < rows * dv; i += blockDim.x) {
       const int j = i / dv, e = i % dv;
       float acc = 0.f;
       if (causal)
-        for (int t = j; t < rows; ++t) acc = fmaf(P[t * Bk + j], dOs[t * dv + e], acc);
-      for (int cc = 0; cc < d; ++cc) acc = fmaf(Ks[j * d + cc], U[cc * dv + e], acc);
+        for (int t = j; t < rows; ++t) acc = fmaf(to_f32(P[t * Bk + j]), to_f32(dOs[t * dv + e]), acc);
+      for (int cc = 0; cc < d; ++cc) acc = fmaf(to_f32(Ks[j * d + cc]), U[cc * dv + e], acc);
       dvb[(i0 + j) * dv + e] = from_f32<T>(acc);
     }
     __syncthreads();
@@ -350,7 +352,7 @@ bwd_dkdv_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* 
       for (int i = threadIdx.x; i < d * dv; i += blockDim.x) {
         const int cc = i / dv, e = i % dv;
         float acc = U[i];
-        for (int t = 0; t < rows; ++t) acc = fmaf(Qs[t * d + cc], dOs[t * dv + e], acc);
+        for (int t = 0; t < rows; ++t) acc = fmaf(to_f32(Qs[t * d + cc]), to_f32(dOs[t * dv + e]), acc);
         U[i] = acc;
       }
       __syncthreads();
@@ -358,14 +360,14 @@ bwd_dkdv_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* 
   }
 }
 
-inline size_t fwd_simt_smem(int d, int dv, int Bk) {
-  return sizeof(float) * ((size_t)d * dv + (size_t)Bk * (2 * d + dv) + (size_t)Bk * Bk);
+inline size_t fwd_simt_smem(int d, int dv, int Bk, size_t es) {
+  return sizeof(float) * (size_t)d * dv + es * ((size_t)Bk * (2 * d + dv) + (size_t)Bk * Bk);
 }
-inline size_t bwd_dq_simt_smem(int d, int dv, int Bk) {
-  return sizeof(float) * ((size_t)d * dv + (size_t)Bk * (2 * dv + d) + (size_t)Bk * Bk);
+inline size_t bwd_dq_simt_smem(int d, int dv, int Bk, size_t es) {
+  return sizeof(float) * (size_t)d * dv + es * ((size_t)Bk * (2 * dv + d) + (size_t)Bk * Bk);
 }
-inline size_t bwd_dkdv_simt_smem(int d, int dv, int Bk) {
-  return sizeof(float) * ((size_t)d * dv + (size_t)Bk * (2 * d + 2 * dv) + 2 * (size_t)Bk * Bk);
+inline size_t bwd_dkdv_simt_smem(int d, int dv, int Bk, size_t es) {
+  return sizeof(float) * (size_t)d * dv + es * ((size_t)Bk * (2 * d + 2 * dv) + 2 * (size_t)Bk * Bk);
 }
 inline size_t chunk_state_smem(int da, int db) {
   return sizeof(float) * (size_t)kStateRowsPerTile * (da + db);

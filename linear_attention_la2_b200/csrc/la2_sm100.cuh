@@ -247,6 +247,7 @@ struct Cfg {
   // instruction descriptors
   static constexpr uint32_t ID_S = make_idesc(BK, BK, false, false);
   static constexpr uint32_t ID_QKV = make_idesc(BK, DV, false, true);
+  static constexpr uint32_t ID_QKV_KMAJOR = make_idesc(BK, DV, false, false);
   static constexpr uint32_t ID_UPD = make_idesc(D, DV, true, true);
   static constexpr uint32_t ID_PV = make_idesc(BK, DV, false, true);
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
@@ -332,7 +333,12 @@ __device__ __forceinline__ int acc_row(int w4, int t) {
 
 // ------------------------------------------------------------------- kernel
 
-template <int BK, int D, int DV, int MODE>
+// DQ = true turns the block loop into the dQ pass of the backward
+// (d = dv): the Q, K, V slots hold dO, V, K, so S = dO V^T, the masked
+// product P K gives the intra-block part of dQ, the state update is
+// KV += K^T V from the swapped slots, and the inter-block part is dO KV^T
+// (the bf16 snapshot read K-major).
+template <int BK, int D, int DV, int MODE, bool DQ = false>
 __global__ void __launch_bounds__(kThreads, 1)
 la2_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_k,
@@ -502,8 +508,13 @@ la2_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           const uint32_t sa = smem_u32(sSnap);
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * BK * 128 + (kk & 3) * 32;
-            mma_bf16_ss(tO, make_desc(qa + off, 16, 1024), make_desc(sa + kk * 2048, D * 128, 1024),
-                        CF::ID_QKV, kk > 0);
+            if constexpr (DQ)  // B[n=c][k=e] = KV[c][e]: snapshot rows read K-major
+              mma_bf16_ss(tO, make_desc(qa + off, 16, 1024),
+                          make_desc(sa + (kk >> 2) * D * 128 + (kk & 3) * 32, 16, 1024),
+                          CF::ID_QKV_KMAJOR, kk > 0);
+            else
+              mma_bf16_ss(tO, make_desc(qa + off, 16, 1024), make_desc(sa + kk * 2048, D * 128, 1024),
+                          CF::ID_QKV, kk > 0);
           }
         }
         mma_commit(&b.q_empty[qs]);
@@ -513,8 +524,8 @@ la2_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         }
         // KV += K_i^T V_i (after the snapshot of the old state was taken)
         for (int kk = 0; kk < BK / 16; ++kk)
-          mma_bf16_ss(tKV, make_desc(ka + kk * 2048, BK * 128, 1024),
-                      make_desc(va + kk * 2048, BK * 128, 1024), CF::ID_UPD,
+          mma_bf16_ss(tKV, make_desc((DQ ? va : ka) + kk * 2048, BK * 128, 1024),
+                      make_desc((DQ ? ka : va) + kk * 2048, BK * 128, 1024), CF::ID_UPD,
                       (have_snap || kk > 0) ? 1u : 0u);
         mma_commit(b.kv_updated);
         // O_i += P_i V_i
@@ -716,7 +727,7 @@ la2_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
 // --------------------------------------------------------------- host side
 
 inline bool sm100_supports(int64_t d, int64_t dv, int block, bool is_bwd) {
-  if (is_bwd) return false;
+  (void)is_bwd;
   return d == 128 && dv == 128 && (block == 64 || block == 128);
 }
 
@@ -768,12 +779,12 @@ inline bool make_tmap_3d(CUtensorMap* m, const void* base, int64_t BH, int64_t N
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BK, int D, int DV, int MODE>
+template <int BK, int D, int DV, int MODE, bool DQ = false>
 inline la2_status launch_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk,
                                    const CUtensorMap& tv, const sm100::Params& p, int64_t units,
                                    cudaStream_t st) {
   using CF = sm100::Cfg<BK, D, DV>;
-  auto kern = sm100::la2_fwd_sm100_kernel<BK, D, DV, MODE>;
+  auto kern = sm100::la2_fwd_sm100_kernel<BK, D, DV, MODE, DQ>;
   static bool attr_done[128];  // one per template instantiation
   if (!smem_attribute_set(kern, CF::SMEM, attr_done)) return LA2_ERR_CUDA;
   kern<<<static_cast<unsigned>(units), sm100::kThreads, CF::SMEM, st>>>(tq, tk, tv, p);

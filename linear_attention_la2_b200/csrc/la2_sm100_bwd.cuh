@@ -1,0 +1,399 @@
+// dK / dV pass of the backward on sm_100a (tcgen05 + TMEM + TMA).
+//
+// Gradients of L = <dO, O> for O = ((Q K^T) ⊙ M) V (article "Lightning
+// Attention-2 新一代注意力机制", section "Lightning Attention-2简介", point 1;
+// the article names its backward algorithm without printing it). Split along
+// the blocks of point 2, with U = sum over later blocks l of Q_l^T dO_l
+// (d x dv, fp32, kept in TMEM) walking the blocks of a chunk in reverse:
+//   S^T = K_i Q_i^T,  A^T = V_i dO_i^T            (masked: query t >= key j)
+//   dV_i = K_i U + (S^T ⊙ M)  dO_i
+//   dK_i = V_i U^T + (A^T ⊙ M) Q_i
+//   U   += Q_i^T dO_i                             (after U was read for block i)
+// Non-causal: dV_i = K_i U, dK_i = V_i U^T with U = Q^T dO over the sequence.
+//
+// One CTA per (b, h, chunk); 512 threads: warp 0 TMA, warp 1 MMA issuer
+// (+ TMEM), warps 4-7 mask S^T, A^T -> bf16 P^T, Pd^T (SMEM), warps 8-11 the
+// bf16 snapshot of U, warps 12-15 dK, dV -> HBM. A^T lives in the columns of
+// the dK accumulator until the mask warpgroup has read it.
+#pragma once
+
+#include "la2_sm100.cuh"
+
+namespace la2 {
+namespace sm100 {
+
+template <int BK, int D, int DV>
+struct BCfg {
+  static_assert(D == 128 && DV == 128, "tensor-core backward: d = dv = 128");
+  static constexpr int NS = BK == 64 ? 2 : 1;  // stages of (Q, K, V, dO)
+  static constexpr int TILE = BK * 128 * 2;    // one [BK x 128] bf16 tile
+  static constexpr int STAGE = 4 * TILE;
+  static constexpr int PTILE = BK * BK * 2;
+  static constexpr int SNAP = D * DV * 2;
+  static constexpr int OFF_ST = 0;
+  static constexpr int OFF_PT = OFF_ST + NS * STAGE;
+  static constexpr int OFF_PDT = OFF_PT + PTILE;
+  static constexpr int OFF_SNAP = OFF_PDT + PTILE;
+  static constexpr int OFF_BAR = OFF_SNAP + SNAP;
+  static constexpr int NBAR = 2 * NS + 12;
+  static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
+  // TMEM columns: U, dV, dK (A^T aliases dK), S^T
+  static constexpr uint32_t COL_U = 0, COL_DV = 128, COL_DK = 256, COL_ST = 384;
+  static constexpr uint32_t ID_ST = make_idesc(BK, BK, false, false);   // K Q^T, V dO^T
+  static constexpr uint32_t ID_MN = make_idesc(BK, 128, false, true);   // X[K-major] * Y[MN-major]
+  static constexpr uint32_t ID_KM = make_idesc(BK, 128, false, false);  // X[K-major] * Y[K-major]
+  static constexpr uint32_t ID_UPD = make_idesc(D, DV, true, true);     // Q^T dO
+  static_assert(SMEM <= 227 * 1024, "shared memory budget");
+};
+
+struct BwdParams {
+  __nv_bfloat16* dk;       // [BH][N][D]
+  __nv_bfloat16* dv;       // [BH][N][DV]
+  const float* init_u;     // [BH][C][D][DV]: suffix (causal) or total in slot 0 (non-causal)
+  int64_t N, L, C;
+  int64_t spin_limit;
+  int causal;
+};
+
+template <int BK, int D, int DV>
+__global__ void __launch_bounds__(kThreads, 1)
+la2_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
+                          const __grid_constant__ CUtensorMap tm_k,
+                          const __grid_constant__ CUtensorMap tm_v,
+                          const __grid_constant__ CUtensorMap tm_do, const BwdParams prm) {
+  using CF = BCfg<BK, D, DV>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, wg = warp >> 2, w4 = warp & 3;
+
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + CF::OFF_BAR);
+  uint64_t* st_full = bar;
+  uint64_t* st_empty = st_full + CF::NS;
+  uint64_t* s_full = st_empty + CF::NS;   // S^T and A^T written
+  uint64_t* s_read = s_full + 1;          // mask warpgroup has read both
+  uint64_t* p_full = s_read + 1;          // P^T and Pd^T written
+  uint64_t* p_empty = p_full + 1;
+  uint64_t* snap_full = p_empty + 1;
+  uint64_t* u_updated = snap_full + 1;
+  uint64_t* g_full = u_updated + 1;       // dK, dV complete
+  uint64_t* g_empty = g_full + 1;
+  uint64_t* drain = g_empty + 1;
+  uint64_t* spare = drain + 1;
+  (void)spare;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + CF::NBAR);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int64_t unit = blockIdx.x;
+  const int64_t bh = unit / prm.C, c = unit % prm.C;
+  const int64_t t0 = c * prm.L, t1 = min(prm.N, t0 + prm.L);
+  const int nblk = static_cast<int>((t1 - t0 + BK - 1) / BK);
+  const bool causal = prm.causal != 0;
+  const bool has_init = !causal || (prm.init_u && c + 1 < prm.C);
+  const float* init = nullptr;
+  if (!causal) init = prm.init_u + bh * prm.C * static_cast<int64_t>(D * DV);
+  else if (has_init) init = prm.init_u + (bh * prm.C + c) * static_cast<int64_t>(D * DV);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < CF::NS; ++s) { mbar_init(&st_full[s], 1); mbar_init(&st_empty[s], 1); }
+    mbar_init(s_full, 1);
+    mbar_init(s_read, 128);
+    mbar_init(p_full, 128);
+    mbar_init(p_empty, 1);
+    mbar_init(snap_full, 128);
+    mbar_init(u_updated, 1);
+    mbar_init(g_full, 1);
+    mbar_init(g_empty, 128);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == kWarpProducer && lane == 0) {
+    tma_prefetch(&tm_q);
+    tma_prefetch(&tm_k);
+    tma_prefetch(&tm_v);
+    tma_prefetch(&tm_do);
+  }
+  if (warp == kWarpMma) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int64_t lim = prm.spin_limit;
+  uint8_t* sStage = smem + CF::OFF_ST;
+  uint8_t* sPT = smem + CF::OFF_PT;
+  uint8_t* sPdT = smem + CF::OFF_PDT;
+  uint8_t* sSnap = smem + CF::OFF_SNAP;
+  // tile t of stage s: 0 = Q, 1 = K, 2 = V, 3 = dO ([BK rows x 128], two 64-column panels)
+  auto tile = [&](int s, int t) { return sStage + s * CF::STAGE + t * CF::TILE; };
+
+  if (warp == kWarpProducer) {
+    if (lane == 0) {
+      int issued = 0;
+      bool ok = true;
+      for (int s = 0; s < nblk && ok; ++s) {
+        const int i = nblk - 1 - s;  // reverse block order
+        const int row = static_cast<int>(t0 + static_cast<int64_t>(i) * BK);
+        const int slot = s % CF::NS;
+        if (!wait_bar(&st_empty[slot], ((s / CF::NS) & 1) ^ 1, lim, abort_flag, 201)) { ok = false; break; }
+        mbar_expect_tx(&st_full[slot], causal ? 4 * CF::TILE : 2 * CF::TILE);
+        const CUtensorMap* maps[4] = {&tm_q, &tm_k, &tm_v, &tm_do};
+        for (int t = 0; t < 4; ++t) {
+          if (!causal && (t == 0 || t == 3)) continue;  // non-causal needs only K and V
+          for (int p = 0; p < 2; ++p)
+            tma_load_3d(tile(slot, t) + p * BK * 128, maps[t], &st_full[slot], 64 * p, row,
+                        static_cast<int>(bh));
+        }
+        ++issued;
+      }
+      if (!ok)
+        for (int j = max(0, issued - CF::NS); j < issued; ++j) drain_wait(&st_full[j % CF::NS], (j / CF::NS) & 1);
+    }
+  } else if (warp == kWarpMma) {
+    if (lane == 0) {
+      const uint64_t dKm = make_desc(0, 16, 1024);
+      const uint64_t dMN = make_desc(0, BK * 128, 1024);
+      const uint64_t dSnapMN = make_desc(0, D * 128, 1024);
+      const uint32_t tU = tmem + CF::COL_U, tDV = tmem + CF::COL_DV, tDK = tmem + CF::COL_DK;
+      const uint32_t tST = tmem + CF::COL_ST;
+      const uint32_t snap0 = smem_u32(sSnap), pt0 = smem_u32(sPT), pdt0 = smem_u32(sPdT);
+      int snap_ph = 0;
+      bool ok = true;
+      for (int s = 0; s < nblk && ok; ++s) {
+        const int slot = s % CF::NS;
+        const uint32_t aq = smem_u32(tile(slot, 0)), ak = smem_u32(tile(slot, 1));
+        const uint32_t av = smem_u32(tile(slot, 2)), ado = smem_u32(tile(slot, 3));
+        if (!wait_bar(&st_full[slot], (s / CF::NS) & 1, lim, abort_flag, 210)) { ok = false; break; }
+        // the dK/dV accumulators (and the A^T scratch inside dK) must be free
+        if (!wait_bar(g_empty, (s & 1) ^ 1, lim, abort_flag, 211)) { ok = false; break; }
+        const bool have_u = s > 0 || has_init;
+        if (causal) {
+          if (!wait_bar(s_read, (s & 1) ^ 1, lim, abort_flag, 212)) { ok = false; break; }
+          tc_fence_after();
+          // S^T = K Q^T and A^T = V dO^T (both K-major operands, K = 128)
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = ((kk >> 2) * BK * 128 + (kk & 3) * 32) >> 4;
+            mma_bf16_ss(tST, dKm + (ak >> 4) + off, dKm + (aq >> 4) + off, CF::ID_ST, kk > 0);
+          }
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = ((kk >> 2) * BK * 128 + (kk & 3) * 32) >> 4;
+            mma_bf16_ss(tDK, dKm + (av >> 4) + off, dKm + (ado >> 4) + off, CF::ID_ST, kk > 0);
+          }
+          mma_commit(s_full);
+        }
+        if (have_u && (causal || s == 0)) {
+          if (!wait_bar(snap_full, snap_ph, lim, abort_flag, 213)) { ok = false; break; }
+          snap_ph ^= 1;
+        }
+        tc_fence_after();
+        if (have_u) {
+          // dV = K U: A = K (K-major, K = d), B[n=e][k=c] = U[c][e] (snapshot, MN-major)
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = ((kk >> 2) * BK * 128 + (kk & 3) * 32) >> 4;
+            mma_bf16_ss(tDV, dKm + (ak >> 4) + off, dSnapMN + (snap0 >> 4) + kk * (2048 >> 4), CF::ID_MN,
+                        kk > 0);
+          }
+        }
+        if (causal) {
+          // U += Q^T dO (after the snapshot of the old U was taken)
+          for (int kk = 0; kk < BK / 16; ++kk)
+            mma_bf16_ss(tU, dMN + (aq >> 4) + kk * (2048 >> 4), dMN + (ado >> 4) + kk * (2048 >> 4),
+                        CF::ID_UPD, (have_u || kk > 0) ? 1u : 0u);
+          // dK region: A^T must have been read by the mask warpgroup
+          if (!wait_bar(s_read, s & 1, lim, abort_flag, 214)) { ok = false; break; }
+          tc_fence_after();
+        }
+        if (have_u) {
+          // dK = V U^T: A = V (K-major, K = dv), B[n=c][k=e] = U[c][e] (snapshot, K-major)
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = ((kk >> 2) * BK * 128 + (kk & 3) * 32) >> 4;
+            const uint32_t soff = ((kk >> 2) * D * 128 + (kk & 3) * 32) >> 4;
+            mma_bf16_ss(tDK, dKm + (av >> 4) + off, dKm + (snap0 >> 4) + soff, CF::ID_KM, kk > 0);
+          }
+        }
+        // U is updated and no issued MMA reads the snapshot any more: the
+        // state warpgroup may take the next one
+        if (causal) mma_commit(u_updated);
+        if (causal) {
+          if (!wait_bar(p_full, s & 1, lim, abort_flag, 215)) { ok = false; break; }
+          tc_fence_after();
+          // dV += P^T dO ; dK += Pd^T Q  (A = masked tiles, K-major, K = BK; B MN-major)
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint32_t off = ((kk >> 2) * BK * 128 + (kk & 3) * 32) >> 4;
+            mma_bf16_ss(tDV, dKm + (pt0 >> 4) + off, dMN + (ado >> 4) + kk * (2048 >> 4), CF::ID_MN,
+                        (have_u || kk > 0) ? 1u : 0u);
+          }
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint32_t off = ((kk >> 2) * BK * 128 + (kk & 3) * 32) >> 4;
+            mma_bf16_ss(tDK, dKm + (pdt0 >> 4) + off, dMN + (aq >> 4) + kk * (2048 >> 4), CF::ID_MN,
+                        (have_u || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(p_empty);
+        }
+        mma_commit(g_full);
+        mma_commit(&st_empty[slot]);
+      }
+      mma_commit(drain);
+      drain_wait(drain, 0);
+    }
+  } else if (wg == kWgMask) {
+    // S^T, A^T (TMEM, rows = keys j, columns = queries t) -> keep t >= j -> bf16 P^T, Pd^T
+    if (causal) {
+      const int r = acc_row<BK>(w4, lane);
+      const uint32_t lane_off = static_cast<uint32_t>(32 * w4) << 16;
+      const uint32_t bases[2] = {smem_u32(sPT), smem_u32(sPdT)};
+      const uint32_t srcs[2] = {tmem + CF::COL_ST + lane_off, tmem + CF::COL_DK + lane_off};
+      for (int s = 0; s < nblk; ++s) {
+        if (!__all_sync(0xffffffffu, wait_bar(s_full, s & 1, lim, abort_flag, 220))) break;
+        if (!__all_sync(0xffffffffu, wait_bar(p_empty, (s & 1) ^ 1, lim, abort_flag, 221))) break;
+        tc_fence_after();
+        for (int which = 0; which < 2; ++which) {
+#pragma unroll
+          for (int c32 = 0; c32 < BK / 32; ++c32) {
+            uint32_t v[32];
+            tmem_ld32(srcs[which] + c32 * 32, v);
+            tmem_ld_wait();
+            if (r >= 0) {
+#pragma unroll
+              for (int q4 = 0; q4 < 4; ++q4) {
+                uint32_t w[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const int col = c32 * 32 + q4 * 8 + 2 * e;
+                  const float a = (col >= r) ? __uint_as_float(v[q4 * 8 + 2 * e]) : 0.f;
+                  const float b = (col + 1 >= r) ? __uint_as_float(v[q4 * 8 + 2 * e + 1]) : 0.f;
+                  w[e] = pack_bf16x2(a, b);
+                }
+                const int ch = c32 * 4 + q4;
+                const int panel = ch >> 3, cj = ch & 7;
+                st_shared_v4(bases[which] + panel * BK * 128 + r * 128 + ((cj ^ (r & 7)) << 4), w[0],
+                             w[1], w[2], w[3]);
+              }
+            }
+          }
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        mbar_arrive(s_read);
+        mbar_arrive(p_full);
+      }
+    }
+  } else if (wg == kWgState) {
+    // bf16 snapshot of U (rows c, 64-column panels); initial U from HBM
+    const int r = acc_row<D>(w4, lane);
+    const uint32_t lane_off = static_cast<uint32_t>(32 * w4) << 16;
+    const uint32_t tU = tmem + CF::COL_U + lane_off;
+    const uint32_t sbase = smem_u32(sSnap);
+    auto put_row = [&](const uint32_t* v, int col0) {
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        const int col = col0 + q4 * 8;
+        const int panel = col >> 6, cj = (col & 63) >> 3;
+        st_shared_v4(sbase + panel * D * 128 + r * 128 + ((cj ^ (r & 7)) << 4),
+                     pack_bf16x2(__uint_as_float(v[q4 * 8 + 0]), __uint_as_float(v[q4 * 8 + 1])),
+                     pack_bf16x2(__uint_as_float(v[q4 * 8 + 2]), __uint_as_float(v[q4 * 8 + 3])),
+                     pack_bf16x2(__uint_as_float(v[q4 * 8 + 4]), __uint_as_float(v[q4 * 8 + 5])),
+                     pack_bf16x2(__uint_as_float(v[q4 * 8 + 6]), __uint_as_float(v[q4 * 8 + 7])));
+      }
+    };
+    if (has_init) {
+#pragma unroll 1
+      for (int c32 = 0; c32 < DV / 32; ++c32) {
+        uint32_t u[32];
+        const float4* src = reinterpret_cast<const float4*>(init + static_cast<int64_t>(r) * DV + c32 * 32);
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4) {
+          const float4 x = src[q4];
+          u[4 * q4] = __float_as_uint(x.x);
+          u[4 * q4 + 1] = __float_as_uint(x.y);
+          u[4 * q4 + 2] = __float_as_uint(x.z);
+          u[4 * q4 + 3] = __float_as_uint(x.w);
+        }
+        if (causal) tmem_st32(tU + c32 * 32, u);
+        put_row(u, c32 * 32);
+      }
+      if (causal) tmem_st_wait();
+      fence_proxy_async();
+      tc_fence_before();
+      mbar_arrive(snap_full);
+    }
+    if (causal) {
+      for (int s = 0; s + 1 < nblk; ++s) {
+        if (!__all_sync(0xffffffffu, wait_bar(u_updated, s & 1, lim, abort_flag, 230))) break;
+        // the snapshot buffer is free: every MMA reading it was issued before
+        // the update whose completion u_updated reports
+        tc_fence_after();
+#pragma unroll
+        for (int c32 = 0; c32 < DV / 32; ++c32) {
+          uint32_t v[32];
+          tmem_ld32(tU + c32 * 32, v);
+          tmem_ld_wait();
+          put_row(v, c32 * 32);
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        mbar_arrive(snap_full);
+      }
+    }
+  } else if (wg == kWgEpilogue) {
+    // dV, dK (TMEM, fp32) -> bf16 -> HBM rows
+    const int r = acc_row<BK>(w4, lane);
+    const uint32_t lane_off = static_cast<uint32_t>(32 * w4) << 16;
+    for (int s = 0; s < nblk; ++s) {
+      const int i = nblk - 1 - s;
+      if (!__all_sync(0xffffffffu, wait_bar(g_full, s & 1, lim, abort_flag, 240))) break;
+      tc_fence_after();
+      const int64_t row = t0 + static_cast<int64_t>(i) * BK + r;
+      const bool valid = r >= 0 && row < t1;
+      for (int which = 0; which < 2; ++which) {
+        __nv_bfloat16* outp = which == 0 ? prm.dv : prm.dk;
+        const int W = which == 0 ? DV : D;
+        const uint32_t src = tmem + (which == 0 ? CF::COL_DV : CF::COL_DK) + lane_off;
+        uint4* dst = reinterpret_cast<uint4*>(outp + (bh * prm.N + (valid ? row : 0)) * W);
+#pragma unroll
+        for (int c32 = 0; c32 < 128 / 32; ++c32) {
+          uint32_t v[32];
+          tmem_ld32(src + c32 * 32, v);
+          tmem_ld_wait();
+          if (valid) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              dst[c32 * 4 + q] = make_uint4(
+                  pack_bf16x2(__uint_as_float(v[8 * q]), __uint_as_float(v[8 * q + 1])),
+                  pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3])),
+                  pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5])),
+                  pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7])));
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(g_empty);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kWarpMma) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace sm100
+
+template <int BK>
+inline la2_status launch_bwd_dkdv_sm100(const CUtensorMap& tq, const CUtensorMap& tk,
+                                        const CUtensorMap& tv, const CUtensorMap& tdo,
+                                        const sm100::BwdParams& p, int64_t units, cudaStream_t st) {
+  using CF = sm100::BCfg<BK, 128, 128>;
+  auto kern = sm100::la2_bwd_dkdv_sm100_kernel<BK, 128, 128>;
+  static bool attr_done[128];
+  if (!smem_attribute_set(kern, CF::SMEM, attr_done)) return LA2_ERR_CUDA;
+  kern<<<static_cast<unsigned>(units), sm100::kThreads, CF::SMEM, st>>>(tq, tk, tv, tdo, p);
+  return cudaGetLastError() == cudaSuccess ? LA2_OK : LA2_ERR_CUDA;
+}
+
+}  // namespace la2
