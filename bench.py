@@ -288,6 +288,11 @@ def run_gpu(args):
     return 0
 
 
+def whole_job_rate(units_per_rank, steps, world, ms_max):
+    """Units all ranks processed per second, timed by the slowest rank."""
+    return units_per_rank * steps * world / (ms_max / 1e3)
+
+
 def _max_over_ranks(x, world, dev):
     if world == 1:
         return x
@@ -384,9 +389,8 @@ def bench_workload(args, w, dev, la2, world, rank, local, hbm, peak_kind, main):
             launches += n
     dom = max(per_kernel, key=lambda k: per_kernel[k]["ms"]) if per_kernel else None
 
-    tokens = w.tokens * args.steps * world
-    value = tokens / (ms_max / 1e3)
-    tflops = flops_per_token(w) * tokens / (ms_max / 1e3) / 1e12
+    value = whole_job_rate(w.tokens, args.steps, world, ms_max)
+    tflops = flops_per_token(w) * value / 1e12
     roofline = None
     if dom:
         avg_ms = per_kernel[dom]["ms"] / per_kernel[dom]["launches"]
@@ -457,7 +461,7 @@ def e2e_measure(args, w, dev, la2, world, base, ws, ws_bytes, dt):
     ms = _max_over_ranks(e0.elapsed_time(e1), world, dev)
     h2d = (hq.numel() + hk.numel() + hv.numel()) * hq.element_size()
     d2h = ho.numel() * ho.element_size()
-    return {"value": w.tokens * args.steps * world / (ms / 1e3), "unit": "tokens/s",
+    return {"value": whole_job_rate(w.tokens, args.steps, world, ms), "unit": "tokens/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
 
