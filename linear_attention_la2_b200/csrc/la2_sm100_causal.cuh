@@ -387,7 +387,9 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
   } else if (warp == kWarpMma) {
     // ================================================================ MMA
-    if (lane == 0) {
+    // The whole warp runs the issue loop (warp-uniform bookkeeping); one
+    // elected lane issues each tcgen05 instruction.
+    {
       const uint32_t tKV = tmem + CF::COL_KV;
       StepIter<KIND> it;
       it.begin(&rt);
@@ -395,10 +397,13 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       bool have = it.next(st);
       uint32_t g = 0, m = 0, sn = 0, acks = 0;
       bool ack_pending = false, s_ready = false, ok = true;
+      auto wait_w = [&](uint64_t* b, uint32_t par, int where) -> bool {
+        return __all_sync(0xffffffffu, wait_bar(b, par, lim, abort_flag, where));
+      };
 
       auto wait_ack = [&]() -> bool {
         if (!ack_pending) return true;
-        if (!wait_bar(seg_ack, acks & 1, lim, abort_flag, 110)) return false;
+        if (!wait_w(seg_ack, acks & 1, 110)) return false;
         ++acks;
         ack_pending = false;
         return true;
@@ -415,15 +420,15 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         const uint64_t b = dK_mn + ((sV0 + slot * CF::VTILE) >> 4);
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk)
-          mma_bf16_ss(tKV, a + kk * (2048 >> 4), b + kk * (2048 >> 4), CF::ID_UPD,
+          mma_bf16_ss_warp(tKV, a + kk * (2048 >> 4), b + kk * (2048 >> 4), CF::ID_UPD,
                       (accumulate || kk > 0) ? 1u : 0u);
       };
       // S(mm) = Q K^T into S buffer mm % NSB; Q slot mm % QS, K slot gg % KS.
       auto issue_s = [&](uint32_t mm, uint32_t gg) -> bool {
         LA2_TRACE_POINT(5, mm);
-        if (!wait_bar(&q_full[mm % CF::QS], (mm / CF::QS) & 1, lim, abort_flag, 111)) return false;
-        if (!wait_bar(&kv_full[gg % CF::KS], (gg / CF::KS) & 1, lim, abort_flag, 112)) return false;
-        if (!wait_bar(&s_empty[mm % CF::NSB], ((mm / CF::NSB) & 1) ^ 1, lim, abort_flag, 113)) return false;
+        if (!wait_w(&q_full[mm % CF::QS], (mm / CF::QS) & 1, 111)) return false;
+        if (!wait_w(&kv_full[gg % CF::KS], (gg / CF::KS) & 1, 112)) return false;
+        if (!wait_w(&s_empty[mm % CF::NSB], ((mm / CF::NSB) & 1) ^ 1, 113)) return false;
         tc_fence_after();
         const uint64_t a = dKm + ((sQ0 + (mm % CF::QS) * CF::QTILE) >> 4);
         const uint64_t b = dKm + ((sK0 + (gg % CF::KS) * CF::KTILE) >> 4);
@@ -431,9 +436,9 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = ((kk >> 2) * BK * 128 + (kk & 3) * 32) >> 4;
-          mma_bf16_ss(tS, a + off, b + off, CF::ID_S, kk > 0);
+          mma_bf16_ss_warp(tS, a + off, b + off, CF::ID_S, kk > 0);
         }
-        mma_commit(&s_full[mm % CF::NSB]);
+        mma_commit_warp(&s_full[mm % CF::NSB]);
         LA2_TRACE_POINT(6, mm);
         return true;
       };
@@ -442,27 +447,27 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         const bool have_nx = it.next(nx);
         const uint32_t ks = g % CF::KS;
         if (st.pre) {
-          if (!wait_bar(&kv_full[ks], (g / CF::KS) & 1, lim, abort_flag, 114)) { ok = false; break; }
+          if (!wait_w(&kv_full[ks], (g / CF::KS) & 1, 114)) { ok = false; break; }
           if (!wait_ack()) { ok = false; break; }
           tc_fence_after();
           update(ks, !st.pre_first);
           if (st.pre_last) {
-            mma_commit(kv_updated);
+            mma_commit_warp(kv_updated);
             if (KIND == KIND_AGG) ack_pending = true;
           }
-          mma_commit(&kv_empty[ks]);
+          mma_commit_warp(&kv_empty[ks]);
         } else {
           if (!s_ready && !issue_s(m, g)) { ok = false; break; }
           s_ready = false;
           const bool needs_snap = !(st.seg_first && st.init == 0);
           const uint32_t sb = sn % CF::NSNAP;
           if (needs_snap &&
-              !wait_bar(&snap_full[sb], (sn / CF::NSNAP) & 1, lim, abort_flag, 115)) { ok = false; break; }
+              !wait_w(&snap_full[sb], (sn / CF::NSNAP) & 1, 115)) { ok = false; break; }
           if (!wait_ack()) { ok = false; break; }
           LA2_TRACE_POINT(2, m);
           const uint32_t ob = m & 1;
           const uint32_t tO = tmem + CF::COL_O + ob * 128;
-          if (!wait_bar(&o_empty[ob], ((m >> 1) & 1) ^ 1, lim, abort_flag, 116)) { ok = false; break; }
+          if (!wait_w(&o_empty[ob], ((m >> 1) & 1) ^ 1, 116)) { ok = false; break; }
           tc_fence_after();
           if (needs_snap) {
             const uint64_t a = dKm + ((sQ0 + (m % CF::QS) * CF::QTILE) >> 4);
@@ -470,18 +475,18 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               const uint32_t off = ((kk >> 2) * BK * 128 + (kk & 3) * 32) >> 4;
-              mma_bf16_ss(tO, a + off, b + kk * (2048 >> 4), CF::ID_QKV, kk > 0);
+              mma_bf16_ss_warp(tO, a + off, b + kk * (2048 >> 4), CF::ID_QKV, kk > 0);
             }
-            mma_commit(&snap_free[sb]);
+            mma_commit_warp(&snap_free[sb]);
             ++sn;
           }
-          mma_commit(&q_empty[m % CF::QS]);
+          mma_commit_warp(&q_empty[m % CF::QS]);
           update(ks, needs_snap);
-          mma_commit(kv_updated);
+          mma_commit_warp(kv_updated);
           if (st.seg_last) ack_pending = true;
           const uint32_t pb = m % CF::NPB;
           LA2_TRACE_POINT(3, m);
-          if (!wait_bar(&p_full[pb], (m / CF::NPB) & 1, lim, abort_flag, 117)) { ok = false; break; }
+          if (!wait_w(&p_full[pb], (m / CF::NPB) & 1, 117)) { ok = false; break; }
           LA2_TRACE_POINT(4, m);
           tc_fence_after();
           {
@@ -490,20 +495,20 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk) {
               const uint32_t off = ((kk >> 2) * BK * 128 + (kk & 3) * 32) >> 4;
-              mma_bf16_ss(tO, a + off, b + kk * (2048 >> 4), CF::ID_PV,
+              mma_bf16_ss_warp(tO, a + off, b + kk * (2048 >> 4), CF::ID_PV,
                           (needs_snap || kk > 0) ? 1u : 0u);
             }
           }
-          mma_commit(&o_full[ob]);
-          mma_commit(&p_empty[pb]);
-          mma_commit(&kv_empty[ks]);
+          mma_commit_warp(&o_full[ob]);
+          mma_commit_warp(&p_empty[pb]);
+          mma_commit_warp(&kv_empty[ks]);
           ++m;
         }
         ++g;
         st = nx;
         have = have_nx;
       }
-      mma_commit(drain);
+      mma_commit_warp(drain);
       drain_wait(drain, 0);
     }
   } else if (wg == kWgMask) {
