@@ -197,6 +197,10 @@ struct CCfg {
   static constexpr int NSB = BK == 64 ? 2 : 1;    // S buffers (TMEM)
   static constexpr int NPB = BK == 64 ? 2 : 1;    // P buffers (SMEM)
   static constexpr int NSNAP = BK == 64 ? 2 : 1;  // KV snapshot buffers (SMEM)
+  // Q rides in the K/V ring (one barrier per step) when the rings are as deep.
+  static constexpr bool QWITHKV = QS == KS;
+  // With two P buffers the P-free signal is the O-full commit of the same block.
+  static constexpr bool MERGE_OP = NPB == 2;
   static constexpr int DP = D / 64;
   static constexpr int VP = DV / 64;
   static constexpr int QTILE = BK * D * 2;
@@ -210,7 +214,7 @@ struct CCfg {
   static constexpr int OFF_P = OFF_V + KS * VTILE;
   static constexpr int OFF_SNAP = OFF_P + NPB * PTILE;
   static constexpr int OFF_BAR = OFF_SNAP + NSNAP * SNAP;
-  static constexpr int NBAR = 2 * QS + 2 * KS + 15;
+  static constexpr int NBAR = 2 * QS + 2 * KS + 15;  // rings + 6 pairs + 3 singles
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
   static constexpr uint32_t COL_KV = 0;
   static constexpr uint32_t COL_O = 128;  // two buffers of 128 columns
@@ -292,8 +296,7 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   uint64_t* kv_full = q_empty + CF::QS;
   uint64_t* kv_empty = kv_full + CF::KS;
   uint64_t* s_full = kv_empty + CF::KS;
-  uint64_t* s_empty = s_full + 2;
-  uint64_t* p_full = s_empty + 2;
+  uint64_t* p_full = s_full + 2;
   uint64_t* p_empty = p_full + 2;
   uint64_t* snap_full = p_empty + 2;
   uint64_t* snap_free = snap_full + 2;
@@ -310,7 +313,6 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     for (int s = 0; s < CF::KS; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&s_full[s], 1);
-      mbar_init(&s_empty[s], 128);
       mbar_init(&p_full[s], 128);
       mbar_init(&p_empty[s], 1);
       mbar_init(&snap_full[s], 128);
@@ -360,14 +362,18 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         const int ks = g % CF::KS;
         if (!wait_bar(&kv_empty[ks], ((g / CF::KS) & 1) ^ 1, lim, abort_flag, 101)) { ok = false; break; }
         LA2_TRACE_POINT(0, g);
-        mbar_expect_tx(&kv_full[ks], CF::KTILE + CF::VTILE);
+        const bool q_here = CF::QWITHKV && !st.pre;
+        mbar_expect_tx(&kv_full[ks], CF::KTILE + CF::VTILE + (q_here ? CF::QTILE : 0));
         for (int p = 0; p < CF::DP; ++p)
           tma_load_3d(sK + ks * CF::KTILE + p * BK * 128, &tm_k, &kv_full[ks], 64 * p, row, zz);
         for (int p = 0; p < CF::VP; ++p)
           tma_load_3d(sV + ks * CF::VTILE + p * BK * 128, &tm_v, &kv_full[ks], 64 * p, row, zz);
+        if (q_here)
+          for (int p = 0; p < CF::DP; ++p)
+            tma_load_3d(sQ + ks * CF::QTILE + p * BK * 128, &tm_q, &kv_full[ks], 64 * p, row, zz);
         ++issued_kv;
         ++g;
-        if (!st.pre) {
+        if (!CF::QWITHKV && !st.pre) {
           const int qs = m % CF::QS;
           if (!wait_bar(&q_empty[qs], ((m / CF::QS) & 1) ^ 1, lim, abort_flag, 102)) { ok = false; break; }
           LA2_TRACE_POINT(1, m);
@@ -423,14 +429,18 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           mma_bf16_ss_warp(tKV, a + kk * (2048 >> 4), b + kk * (2048 >> 4), CF::ID_UPD,
                       (accumulate || kk > 0) ? 1u : 0u);
       };
-      // S(mm) = Q K^T into S buffer mm % NSB; Q slot mm % QS, K slot gg % KS.
+      auto qslot = [](uint32_t mm, uint32_t gg) -> uint32_t {
+        return CF::QWITHKV ? gg % CF::KS : mm % CF::QS;
+      };
+      // S(mm) = Q K^T into S buffer mm % NSB; Q slot qslot(mm, gg), K slot gg % KS.
       auto issue_s = [&](uint32_t mm, uint32_t gg) -> bool {
         LA2_TRACE_POINT(5, mm);
-        if (!wait_w(&q_full[mm % CF::QS], (mm / CF::QS) & 1, 111)) return false;
+        if (!CF::QWITHKV && !wait_w(&q_full[mm % CF::QS], (mm / CF::QS) & 1, 111)) return false;
         if (!wait_w(&kv_full[gg % CF::KS], (gg / CF::KS) & 1, 112)) return false;
-        if (!wait_w(&s_empty[mm % CF::NSB], ((mm / CF::NSB) & 1) ^ 1, 113)) return false;
+        // S buffer mm % NSB is free: the mask role read S(mm - NSB) before it
+        // arrived on p_full(mm - 1), which this warp waited for before PV(mm - 1).
         tc_fence_after();
-        const uint64_t a = dKm + ((sQ0 + (mm % CF::QS) * CF::QTILE) >> 4);
+        const uint64_t a = dKm + ((sQ0 + qslot(mm, gg) * CF::QTILE) >> 4);
         const uint64_t b = dKm + ((sK0 + (gg % CF::KS) * CF::KTILE) >> 4);
         const uint32_t tS = tmem + CF::COL_S + (mm % CF::NSB) * BK;
 #pragma unroll
@@ -470,7 +480,7 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           if (!wait_w(&o_empty[ob], ((m >> 1) & 1) ^ 1, 116)) { ok = false; break; }
           tc_fence_after();
           if (needs_snap) {
-            const uint64_t a = dKm + ((sQ0 + (m % CF::QS) * CF::QTILE) >> 4);
+            const uint64_t a = dKm + ((sQ0 + qslot(m, g) * CF::QTILE) >> 4);
             const uint64_t b = dSnap + ((sS0 + sb * CF::SNAP) >> 4);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
@@ -480,7 +490,7 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
             mma_commit_warp(&snap_free[sb]);
             ++sn;
           }
-          mma_commit_warp(&q_empty[m % CF::QS]);
+          if (!CF::QWITHKV) mma_commit_warp(&q_empty[m % CF::QS]);
           update(ks, needs_snap);
           mma_commit_warp(kv_updated);
           if (st.seg_last) ack_pending = true;
@@ -500,7 +510,7 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
             }
           }
           mma_commit_warp(&o_full[ob]);
-          mma_commit_warp(&p_empty[pb]);
+          if (!CF::MERGE_OP) mma_commit_warp(&p_empty[pb]);
           mma_commit_warp(&kv_empty[ks]);
           ++m;
         }
@@ -526,7 +536,9 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         const uint32_t tS = tmem + CF::COL_S + sbuf * BK + lane_off;
         if (!__all_sync(0xffffffffu, wait_bar(&s_full[sbuf], (m / CF::NSB) & 1, lim, abort_flag, 120))) break;
         if (threadIdx.x % 128 == 0) LA2_TRACE_POINT(7, m);
-        if (!__all_sync(0xffffffffu, wait_bar(&p_empty[pb], ((m / CF::NPB) & 1) ^ 1, lim, abort_flag, 121))) break;
+        // P buffer pb is free once PV(m - NPB) completed (o_full doubles as the signal).
+        uint64_t* p_free = CF::MERGE_OP ? o_full : p_empty;
+        if (!__all_sync(0xffffffffu, wait_bar(&p_free[pb], ((m / CF::NPB) & 1) ^ 1, lim, abort_flag, 121))) break;
         tc_fence_after();
         const uint32_t pbase = smem_u32(sP + pb * CF::PTILE);
 #pragma unroll
@@ -554,7 +566,6 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         }
         fence_proxy_async();
         tc_fence_before();
-        mbar_arrive(&s_empty[sbuf]);
         mbar_arrive(&p_full[pb]);
         if (threadIdx.x % 128 == 0) LA2_TRACE_POINT(8, m);
         ++m;
