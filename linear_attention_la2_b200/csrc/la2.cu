@@ -296,6 +296,10 @@ static la2_status forward_sm100_bk(const void* q, const void* k, const void* v, 
   if (causal) {
     sm100::RangeTable rt;
     if (!fill_range_table(p.rp, &rt)) return LA2_ERR_UNSUPPORTED;
+    // O tiles leave through per-warp TMA stores of 16 rows at Bk=64.
+    CUtensorMap to = tq;
+    if (sm100::CCfg<BK, D, DV>::TMA_STORE && !make_tmap_3d(&to, o, BH, N, DV, 16))
+      return LA2_ERR_CUDA;
     sm100::CausalParams cp{};
     cp.o = static_cast<__nv_bfloat16*>(o);
     cp.agg = states;
@@ -305,11 +309,11 @@ static la2_status forward_sm100_bk(const void* q, const void* k, const void* v, 
     const int grid = std::max(1, std::min(p.rp.R, sms));
     if (p.rp.prefix_mode == 1) {
       LaunchTimer t(K_STATE_TC, st);
-      s = launch_causal_sm100<BK, D, DV, sm100::KIND_AGG>(tq, tk, tv, rt, cp, grid, st);
+      s = launch_causal_sm100<BK, D, DV, sm100::KIND_AGG>(tq, tk, tv, to, rt, cp, grid, st);
       if (s != LA2_OK) return s;
     }
     LaunchTimer t(K_FWD_TC, st);
-    return launch_causal_sm100<BK, D, DV, sm100::KIND_MAIN>(tq, tk, tv, rt, cp, grid, st);
+    return launch_causal_sm100<BK, D, DV, sm100::KIND_MAIN>(tq, tk, tv, to, rt, cp, grid, st);
   }
   sm100::Params ps = prm;
   ps.out_states = states;

@@ -196,7 +196,14 @@ struct CCfg {
   static constexpr int KS = BK == 64 ? 3 : 2;
   static constexpr int NSB = BK == 64 ? 2 : 1;    // S buffers (TMEM)
   static constexpr int NPB = BK == 64 ? 2 : 1;    // P buffers (SMEM)
-  static constexpr int NSNAP = BK == 64 ? 2 : 1;  // KV snapshot buffers (SMEM)
+  // One snapshot buffer suffices: the state role writes snapshot m+1 only after
+  // update(m) completed, and update(m) is issued after QKV(m) read snapshot m.
+  static constexpr int NSNAP = 1;
+  // Bk=64: O leaves through a swizzled staging tile and per-warp TMA stores
+  // (plain row stores from the epilogue crowd the SM's memory-instruction
+  // queue that the MMA warp's barrier and tcgen05 instructions also use).
+  static constexpr bool TMA_STORE = BK == 64;
+  static constexpr int OSTAGE = TMA_STORE ? 2 : 0;
   // Q rides in the K/V ring (one barrier per step) when the rings are as deep.
   static constexpr bool QWITHKV = QS == KS;
   // With two P buffers the P-free signal is the O-full commit of the same block.
@@ -208,12 +215,14 @@ struct CCfg {
   static constexpr int VTILE = BK * DV * 2;
   static constexpr int PTILE = BK * BK * 2;
   static constexpr int SNAP = D * DV * 2;
+  static constexpr int OTILE = BK * DV * 2;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + QS * QTILE;
   static constexpr int OFF_V = OFF_K + KS * KTILE;
   static constexpr int OFF_P = OFF_V + KS * VTILE;
   static constexpr int OFF_SNAP = OFF_P + NPB * PTILE;
-  static constexpr int OFF_BAR = OFF_SNAP + NSNAP * SNAP;
+  static constexpr int OFF_OST = OFF_SNAP + NSNAP * SNAP;
+  static constexpr int OFF_BAR = OFF_OST + OSTAGE * OTILE;
   static constexpr int NBAR = 2 * QS + 2 * KS + 15;  // rings + 6 pairs + 3 singles
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
   static constexpr uint32_t COL_KV = 0;
@@ -280,6 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v,
+                        const __grid_constant__ CUtensorMap tm_o,
                         const __grid_constant__ RangeTable rt, const CausalParams prm) {
   using CF = CCfg<BK, D, DV>;
   extern __shared__ uint8_t smem_raw[];
@@ -328,6 +338,7 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   }
   if (warp == kWarpProducer && lane == 0) {
     if (KIND == KIND_MAIN) tma_prefetch(&tm_q);
+    if (KIND == KIND_MAIN && CF::TMA_STORE) tma_prefetch(&tm_o);
     tma_prefetch(&tm_k);
     tma_prefetch(&tm_v);
   }
@@ -680,6 +691,47 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (!__all_sync(0xffffffffu, wait_bar(&o_full[ob], (m >> 1) & 1, lim, abort_flag, 140))) break;
         if (threadIdx.x % 128 == 0) LA2_TRACE_POINT(11, m);
         tc_fence_after();
+        if constexpr (CF::TMA_STORE) {
+          // Warp w4 owns rows 16*w4 .. 16*w4+15 of the block: it stages them
+          // (128B-swizzled, panels of 64 columns) and stores them itself.
+          uint8_t* stage = smem + CF::OFF_OST + ob * CF::OTILE + w4 * 16 * 128;
+          if (lane == 0) bulk_wait_group_read<1>();  // this warp's store of block m-2 has read it
+          __syncwarp();
+          const int rl = lane & 15;
+#pragma unroll
+          for (int c32 = 0; c32 < DV / 32; ++c32) {
+            uint32_t v[32];
+            tmem_ld32(tO + c32 * 32, v);
+            tmem_ld_wait();
+            if (r >= 0) {
+              const uint32_t base = smem_u32(stage + (c32 >> 1) * BK * 128) + rl * 128;
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const int cj = (c32 & 1) * 4 + q;
+                st_shared_v4(base + ((cj ^ (rl & 7)) << 4),
+                             pack_bf16x2(__uint_as_float(v[8 * q]), __uint_as_float(v[8 * q + 1])),
+                             pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3])),
+                             pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5])),
+                             pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7])));
+              }
+            }
+          }
+          tc_fence_before();
+          mbar_arrive(&o_empty[ob]);
+          fence_proxy_async();
+          __syncwarp();
+          const int64_t y = static_cast<int64_t>(st.blk) * BK + 16 * w4;
+          if (lane == 0 && y < prm.N) {  // rows past N are clipped by the tensor map
+#pragma unroll
+            for (int p = 0; p < DV / 64; ++p)
+              tma_store_3d(&tm_o, stage + p * BK * 128, 64 * p, static_cast<int>(y),
+                           static_cast<int>(st.bh));
+            bulk_commit_group();
+          }
+          if (threadIdx.x % 128 == 0) LA2_TRACE_POINT(12, m);
+          ++m;
+          continue;
+        }
         const int64_t row = static_cast<int64_t>(st.blk) * BK + r;
         const bool valid = r >= 0 && row < prm.N;
         uint4* dst = reinterpret_cast<uint4*>(prm.o + (st.bh * prm.N + (valid ? row : 0)) * DV);
@@ -703,6 +755,7 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (threadIdx.x % 128 == 0) LA2_TRACE_POINT(12, m);
         ++m;
       }
+      if (CF::TMA_STORE && lane == 0) bulk_wait_group<0>();  // stores done before exit
     }
   }
 
@@ -806,13 +859,14 @@ inline bool fill_range_table(const RangePlan& p, sm100::RangeTable* t) {
 
 template <int BK, int D, int DV, int KIND>
 inline la2_status launch_causal_sm100(const CUtensorMap& tq, const CUtensorMap& tk,
-                                      const CUtensorMap& tv, const sm100::RangeTable& rt,
+                                      const CUtensorMap& tv, const CUtensorMap& to,
+                                      const sm100::RangeTable& rt,
                                       const sm100::CausalParams& p, int grid, cudaStream_t st) {
   using CF = sm100::CCfg<BK, D, DV>;
   auto kern = sm100::la2_causal_sm100_kernel<BK, D, DV, KIND>;
   static bool attr_done[128];  // one per template instantiation
   if (!smem_attribute_set(kern, CF::SMEM, attr_done)) return LA2_ERR_CUDA;
-  kern<<<static_cast<unsigned>(grid), sm100::kThreads, CF::SMEM, st>>>(tq, tk, tv, rt, p);
+  kern<<<static_cast<unsigned>(grid), sm100::kThreads, CF::SMEM, st>>>(tq, tk, tv, to, rt, p);
   return cudaGetLastError() == cudaSuccess ? LA2_OK : LA2_ERR_CUDA;
 }
 
