@@ -63,7 +63,7 @@ struct RangeTable {
 
 struct CausalParams {
   __nv_bfloat16* o;  // [BH][N][DV]
-  float* agg;        // range states [R][D][DV] (prefix_mode 1, or KIND_AGG output)
+  float* agg;        // range states [R][D*DV] (prefix_mode 1, or KIND_AGG output); see agg_f4
   int64_t N;
   int64_t spin_limit;
 };
@@ -253,6 +253,15 @@ __device__ __forceinline__ void put_snap_row(uint32_t sbase, int r, const uint32
 // Row r of the state: sum over the earlier ranges of this sequence of their
 // range states (fp32, HBM), written to TMEM (fp32) and, rounded to bf16, to
 // the snapshot at `sbase`. Cold path (once per range), kept out of line.
+// A range state (D x DV fp32) is stored column-chunk-major: float4 j (columns
+// 4j..4j+3) of row r at float4 index j*D + r. The 32 threads of a warp own 32
+// consecutive rows, so each 16-byte access of the warp covers 512 contiguous
+// bytes (row-major rows would put the warp's accesses 4*DV bytes apart).
+template <int D>
+__device__ __forceinline__ int64_t agg_f4(int r, int j) {
+  return static_cast<int64_t>(j) * D + r;
+}
+
 template <int D, int DV>
 __device__ __noinline__ void init_from_ranges(const float* agg, const RangeTable& rt, int32_t range,
                                               int64_t head0, int r, uint32_t tKV, uint32_t sbase) {
@@ -263,11 +272,10 @@ __device__ __noinline__ void init_from_ranges(const float* agg, const RangeTable
     for (int j = 0; j < 32; ++j) acc[j] = 0.f;
     if (r >= 0) {
       for (int rr = range - 1; rr >= 0 && rt.starts[rr + 1] > head0; --rr) {
-        const float4* src = reinterpret_cast<const float4*>(
-            agg + static_cast<int64_t>(rr) * D * DV + static_cast<int64_t>(r) * DV + c32 * 32);
+        const float4* src = reinterpret_cast<const float4*>(agg + static_cast<int64_t>(rr) * D * DV);
 #pragma unroll
         for (int q4 = 0; q4 < 8; ++q4) {
-          const float4 x = src[q4];
+          const float4 x = src[agg_f4<D>(r, c32 * 8 + q4)];
           acc[4 * q4] += x.x;
           acc[4 * q4 + 1] += x.y;
           acc[4 * q4 + 2] += x.z;
@@ -280,6 +288,63 @@ __device__ __noinline__ void init_from_ranges(const float* agg, const RangeTable
     for (int j = 0; j < 32; ++j) u[j] = __float_as_uint(acc[j]);
     tmem_st32(tKV + c32 * 32, u);
     if (r >= 0) put_snap_row<D>(sbase, r, u, c32 * 32);
+  }
+  tmem_st_wait();
+}
+
+// Initial state of the CTA's first range when it starts inside a sequence
+// (range-state mode): the sum of the states of the sequence's earlier ranges.
+// Run once at CTA start by the three consumer warpgroups together; warp w4 of
+// each owns TMEM lanes (state rows) 32*w4 .. 32*w4+31 and warpgroup `part`
+// (0..2) sums the 32-column chunks {0, 3}, {1} or {2} of those rows, two
+// ranges' loads in flight per round.
+template <int D, int DV>
+__device__ __noinline__ void init_state_coop(const float* agg, const RangeTable& rt, int32_t range,
+                                             int64_t head0, int part, int w4, int lane,
+                                             uint32_t tKV, uint32_t sbase) {
+  static_assert(D == 128 && DV == 128, "one TMEM lane per state row, four column chunks");
+  int nprev = 0;
+  while (range - 1 - nprev >= 0 && rt.starts[range - nprev] > head0) ++nprev;
+  const int r = 32 * w4 + lane;
+  const uint32_t lane_off = static_cast<uint32_t>(32 * w4) << 16;
+  for (int c = part; c < DV / 32; c += 3) {
+    float acc[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) acc[j] = 0.f;
+    int i = 0;
+    for (; i + 2 <= nprev; i += 2) {
+      const float4* s0 = reinterpret_cast<const float4*>(agg + static_cast<int64_t>(range - 1 - i) * D * DV);
+      const float4* s1 = s0 - static_cast<int64_t>(D) * DV / 4;
+      float4 x[8], y[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        x[q] = s0[agg_f4<D>(r, c * 8 + q)];
+        y[q] = s1[agg_f4<D>(r, c * 8 + q)];
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        acc[4 * q] += x[q].x + y[q].x;
+        acc[4 * q + 1] += x[q].y + y[q].y;
+        acc[4 * q + 2] += x[q].z + y[q].z;
+        acc[4 * q + 3] += x[q].w + y[q].w;
+      }
+    }
+    if (i < nprev) {
+      const float4* s0 = reinterpret_cast<const float4*>(agg + static_cast<int64_t>(range - 1 - i) * D * DV);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const float4 x = s0[agg_f4<D>(r, c * 8 + q)];
+        acc[4 * q] += x.x;
+        acc[4 * q + 1] += x.y;
+        acc[4 * q + 2] += x.z;
+        acc[4 * q + 3] += x.w;
+      }
+    }
+    uint32_t u[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) u[j] = __float_as_uint(acc[j]);
+    tmem_st32(tKV + lane_off + c * 32, u);
+    put_snap_row<D>(sbase, r, u, c * 32);
   }
   tmem_st_wait();
 }
@@ -351,6 +416,27 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int64_t lim = prm.spin_limit;
+
+  // Range-state mode: a CTA's range (at most one per CTA) that starts inside
+  // a sequence gets its initial state from the consumer warpgroups before
+  // they take up their roles. The producer warp holds its first loads until
+  // then: behind a full TMA ring the state loads would queue for microseconds.
+  bool first_init_ready = false;
+  if (KIND == KIND_MAIN && rt.prefix_mode == 1 && static_cast<int32_t>(blockIdx.x) < rt.R) {
+    const int64_t f0 = rt.starts[blockIdx.x];
+    const int64_t head0 = (f0 / rt.T) * rt.T;
+    if (f0 != head0 && (wg >= 1 || warp == kWarpProducer)) {
+      if (wg >= 1) {
+        init_state_coop<D, DV>(prm.agg, rt, static_cast<int32_t>(blockIdx.x), head0, wg - 1, w4,
+                               lane, tmem + CF::COL_KV, smem_u32(smem + CF::OFF_SNAP));
+        first_init_ready = true;
+        fence_proxy_async();
+        tc_fence_before();
+      }
+      named_bar_sync(1, 416);  // warps 4..15 and the producer warp
+      tc_fence_after();
+    }
+  }
 
   uint8_t* sQ = smem + CF::OFF_Q;
   uint8_t* sK = smem + CF::OFF_K;
@@ -645,10 +731,10 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           tmem_ld32(tKV + c32 * 32, v);
           tmem_ld_wait();
           if (r >= 0) {
-            float4* p4 = reinterpret_cast<float4*>(dst + static_cast<int64_t>(r) * DV + c32 * 32);
+            float4* p4 = reinterpret_cast<float4*>(dst);
 #pragma unroll
             for (int q4 = 0; q4 < 8; ++q4)
-              p4[q4] = make_float4(__uint_as_float(v[4 * q4]), __uint_as_float(v[4 * q4 + 1]),
+              p4[agg_f4<D>(r, c32 * 8 + q4)] = make_float4(__uint_as_float(v[4 * q4]), __uint_as_float(v[4 * q4 + 1]),
                                    __uint_as_float(v[4 * q4 + 2]), __uint_as_float(v[4 * q4 + 3]));
           }
         }
@@ -661,7 +747,14 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (st.init == 1) {
           if (!wait_kvu() || !snap_from_tmem()) break;
         } else if (st.init == 2) {
-          if (!snap_from_ranges(st)) break;
+          if (first_init_ready) {  // built at CTA start into TMEM and snapshot 0
+            first_init_ready = false;
+            tc_fence_before();
+            mbar_arrive(&snap_full[sn % CF::NSNAP]);
+            ++sn;
+          } else if (!snap_from_ranges(st)) {
+            break;
+          }
         }
       } else {
         if (!wait_kvu()) break;
@@ -771,11 +864,12 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
 
 // ------------------------------------------------------------------ host side
 
-// Cost model of the range split (in units of one main block): a pre-pass
-// block reads only K and V and issues one small MMA group.
-constexpr double kPrepassCost = 0.25;
-constexpr double kRangeStateCost = 0.35;  // separate state launch, per block
-constexpr double kLaunchCost = 1.0;       // one extra launch, in main blocks
+// Cost model of the range split, in units of one main block (measured on a
+// loaded B200 at Bk=64: main block ~1.2 us, pre-pass block ~0.6 us; a pre-pass
+// block moves half the bytes and its loads stay latency-bound).
+constexpr double kPrepassCost = 0.5;
+constexpr double kRangeStateCost = 0.5;  // separate state launch, per block
+constexpr double kLaunchCost = 3.0;      // extra launch + initial-state sum, in main blocks
 
 struct RangePlan {
   int R = 0;
