@@ -102,6 +102,7 @@ struct Plan {
   bool need_states = false;
   size_t ws_bytes = 0;
   bool ranges = false;  // persistent range split (tensor-core causal forward)
+  bool dq_ranges = false;  // tensor-core causal backward: dQ through the range split
   RangePlan rp;
 };
 
@@ -156,18 +157,30 @@ static Plan make_plan_uncached(int64_t B, int64_t H, int64_t N, int64_t d, int64
     L = ((T + C - 1) / C) * block;
   }
   L = std::max<int64_t>(L, block);
-  if (p.tc && causal && !is_bwd) {
+  const size_t state_bytes = (size_t)d * (size_t)dv * sizeof(float);
+  if (p.tc && causal) {
     p.ranges = true;
     p.rp = plan_ranges(BH, N, block, sms, g_chunk_len);
-    p.need_states = p.rp.prefix_mode == 1;
-    p.ws_bytes = p.need_states ? (size_t)p.rp.R * (size_t)d * (size_t)dv * sizeof(float) : 0;
-    return p;
+    if (!is_bwd) {
+      p.need_states = p.rp.prefix_mode == 1;
+      p.ws_bytes = p.need_states ? (size_t)p.rp.R * state_bytes : 0;
+      return p;
+    }
   }
   p.L = L;
   p.C = std::max<int64_t>(1, (N + L - 1) / L);
   p.need_states = (p.C > 1) || !causal;
-  const size_t one = (size_t)BH * (size_t)p.C * (size_t)d * (size_t)dv * sizeof(float);
+  const size_t one = (size_t)BH * (size_t)p.C * state_bytes;
   p.ws_bytes = p.need_states ? one * (is_bwd ? 2 : 1) : 0;
+  if (p.tc && causal && is_bwd) {
+    // Workspace: [U chunk states | K^T V chunk states or the dQ pass's range
+    // states, whichever is larger]. The dQ pass takes the range split when
+    // its table can hold the ranges, else the chunk path.
+    p.dq_ranges = p.rp.R >= 1 && p.rp.R <= sm100::kMaxRanges;
+    const size_t agg = p.dq_ranges && p.rp.prefix_mode == 1 ? (size_t)p.rp.R * state_bytes : 0;
+    const size_t kv = p.need_states ? one : 0;
+    p.ws_bytes = (p.need_states ? one : 0) + std::max(agg, kv);
+  }
   return p;
 }
 
@@ -273,13 +286,51 @@ static la2_status backward_simt(const void* q, const void* k, const void* v, con
   return launch_status();
 }
 
-// Tensor-core forward: chunk states (if the sequence is split, or always for
-// the non-causal form), their scan, then the block loop from each chunk's
-// initial state.
+// Causal O = ((Q K^T) ⊙ M) V on the persistent range-split kernel: the
+// (b, h, block) task list cut into at most one range per SM; a range that
+// starts inside a sequence gets its initial state from a pre-pass over the
+// sequence's earlier blocks or from the range states of a separate pass.
+// Also the dQ pass of the backward, with (dO, V, K) in the (Q, K, V) slots.
+template <int BK>
+static la2_status causal_range_split(const void* q, const void* k, const void* v, void* o,
+                                     int64_t BH, int64_t N, float* range_states,
+                                     const RangePlan& rp, int64_t spin, cudaStream_t st,
+                                     int kid_states, int kid_main) {
+  constexpr int D = 128, DV = 128;
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap_3d(&tq, q, BH, N, D, BK) || !make_tmap_3d(&tk, k, BH, N, D, BK) ||
+      !make_tmap_3d(&tv, v, BH, N, DV, BK))
+    return LA2_ERR_CUDA;
+  sm100::RangeTable rt;
+  if (!fill_range_table(rp, &rt)) return LA2_ERR_UNSUPPORTED;
+  // O tiles leave through per-warp TMA stores of 16 rows at Bk=64.
+  CUtensorMap to = tq;
+  if (sm100::CCfg<BK, D, DV>::TMA_STORE && !make_tmap_3d(&to, o, BH, N, DV, 16))
+    return LA2_ERR_CUDA;
+  sm100::CausalParams cp{};
+  cp.o = static_cast<__nv_bfloat16*>(o);
+  cp.agg = range_states;
+  cp.N = N;
+  cp.spin_limit = spin;
+  const int sms = device_sm_count();
+  const int grid = std::max(1, std::min(rp.R, sms));
+  if (rp.prefix_mode == 1) {
+    LaunchTimer t(kid_states, st);
+    const la2_status s = launch_causal_sm100<BK, D, DV, sm100::KIND_AGG>(tq, tk, tv, to, rt, cp, grid, st);
+    if (s != LA2_OK) return s;
+  }
+  LaunchTimer t(kid_main, st);
+  return launch_causal_sm100<BK, D, DV, sm100::KIND_MAIN>(tq, tk, tv, to, rt, cp, grid, st);
+}
+
+// Tensor-core forward. Causal: the range split above. Non-causal: chunk
+// states, their total, then every block against the total state.
 template <int BK>
 static la2_status forward_sm100_bk(const void* q, const void* k, const void* v, void* o,
                                    int64_t BH, int64_t N, int causal, float* states,
                                    const Plan& p, int64_t spin, cudaStream_t st) {
+  if (causal)
+    return causal_range_split<BK>(q, k, v, o, BH, N, states, p.rp, spin, st, K_STATE_TC, K_FWD_TC);
   constexpr int D = 128, DV = 128;
   CUtensorMap tq, tk, tv;
   if (!make_tmap_3d(&tq, q, BH, N, D, BK) || !make_tmap_3d(&tk, k, BH, N, D, BK) ||
@@ -293,42 +344,22 @@ static la2_status forward_sm100_bk(const void* q, const void* k, const void* v, 
   prm.spin_limit = spin;
   la2_status s = LA2_OK;
   const int nel = D * DV;
-  if (causal) {
-    sm100::RangeTable rt;
-    if (!fill_range_table(p.rp, &rt)) return LA2_ERR_UNSUPPORTED;
-    // O tiles leave through per-warp TMA stores of 16 rows at Bk=64.
-    CUtensorMap to = tq;
-    if (sm100::CCfg<BK, D, DV>::TMA_STORE && !make_tmap_3d(&to, o, BH, N, DV, 16))
-      return LA2_ERR_CUDA;
-    sm100::CausalParams cp{};
-    cp.o = static_cast<__nv_bfloat16*>(o);
-    cp.agg = states;
-    cp.N = N;
-    cp.spin_limit = spin;
-    const int sms = device_sm_count();
-    const int grid = std::max(1, std::min(p.rp.R, sms));
-    if (p.rp.prefix_mode == 1) {
-      LaunchTimer t(K_STATE_TC, st);
-      s = launch_causal_sm100<BK, D, DV, sm100::KIND_AGG>(tq, tk, tv, to, rt, cp, grid, st);
-      if (s != LA2_OK) return s;
-    }
-    LaunchTimer t(K_FWD_TC, st);
-    return launch_causal_sm100<BK, D, DV, sm100::KIND_MAIN>(tq, tk, tv, to, rt, cp, grid, st);
-  }
   sm100::Params ps = prm;
   ps.out_states = states;
   ps.units_per_seq = p.C;
   {
     LaunchTimer t(K_STATE_TC, st);
-    s = launch_fwd_sm100<BK, D, DV, sm100::MODE_STATE>(tq, tk, tv, ps, BH * p.C, st);
+    s = launch_fwd_sm100<BK, D, DV, sm100::MODE_STATE>(tq, tk, tv, tq, ps, BH * p.C, st);
   }
   if (s != LA2_OK) return s;
   s = run_scan(states, BH, nel, p, 2, st);
   if (s != LA2_OK) return s;
   prm.init_states = states;
   prm.units_per_seq = p.C;
+  CUtensorMap to_nc = tq;
+  if (sm100::Cfg<BK, D, DV>::TMA_STORE && !make_tmap_3d(&to_nc, o, BH, N, DV, 16)) return LA2_ERR_CUDA;
   LaunchTimer t(K_FWD_TC, st);
-  return launch_fwd_sm100<BK, D, DV, sm100::MODE_NONCAUSAL>(tq, tk, tv, prm, BH * p.C, st);
+  return launch_fwd_sm100<BK, D, DV, sm100::MODE_NONCAUSAL>(tq, tk, tv, to_nc, prm, BH * p.C, st);
 }
 
 // Tensor-core backward: chunk states K^T V (prefix for dQ) and Q^T dO
@@ -347,6 +378,12 @@ static la2_status backward_sm100_bk(const void* q, const void* k, const void* v,
   la2_status s = LA2_OK;
   const int nel = D * DV;
   const bool states = p.need_states;
+  const bool dq_split = causal && p.dq_ranges;
+  if (dq_split) {
+    // dQ = ((dO V^T) ⊙ M) K: the causal forward with (dO, V, K) as (Q, K, V).
+    s = causal_range_split<BK>(dout, v, k, dq, BH, N, s_kv, p.rp, spin, st, K_STATE_TC, K_BWD_DQ_TC);
+    if (s != LA2_OK) return s;
+  }
   if (states) {
     sm100::Params ps{};
     ps.N = N;
@@ -354,37 +391,47 @@ static la2_status backward_sm100_bk(const void* q, const void* k, const void* v,
     ps.C = p.C;
     ps.units_per_seq = p.C;
     ps.spin_limit = spin;
-    {
+    if (!dq_split) {
       LaunchTimer t(K_STATE_TC, st);
       ps.out_states = s_kv;  // K^T V per chunk
-      s = launch_fwd_sm100<BK, D, DV, sm100::MODE_STATE>(tq, tk, tv, ps, BH * p.C, st);
+      s = launch_fwd_sm100<BK, D, DV, sm100::MODE_STATE>(tq, tk, tv, tq, ps, BH * p.C, st);
     }
     if (s != LA2_OK) return s;
     {
       LaunchTimer t(K_STATE_TC, st);
       ps.out_states = s_u;  // Q^T dO per chunk
-      s = launch_fwd_sm100<BK, D, DV, sm100::MODE_STATE>(tq, tq, tdo, ps, BH * p.C, st);
+      s = launch_fwd_sm100<BK, D, DV, sm100::MODE_STATE>(tq, tq, tdo, tq, ps, BH * p.C, st);
     }
     if (s != LA2_OK) return s;
-    s = run_scan(s_kv, BH, nel, p, causal ? 0 : 2, st);
-    if (s != LA2_OK) return s;
+    if (!dq_split) {
+      s = run_scan(s_kv, BH, nel, p, causal ? 0 : 2, st);
+      if (s != LA2_OK) return s;
+    }
     s = run_scan(s_u, BH, nel, p, causal ? 1 : 2, st);
     if (s != LA2_OK) return s;
   }
-  sm100::Params pq{};
-  pq.o = static_cast<__nv_bfloat16*>(dq);
-  pq.init_states = states ? s_kv : nullptr;
-  pq.N = N;
-  pq.L = p.L;
-  pq.C = p.C;
-  pq.units_per_seq = p.C;
-  pq.spin_limit = spin;
-  {
-    LaunchTimer t(K_BWD_DQ_TC, st);
-    s = causal ? launch_fwd_sm100<BK, D, DV, sm100::MODE_CAUSAL, true>(tdo, tv, tk, pq, BH * p.C, st)
-               : launch_fwd_sm100<BK, D, DV, sm100::MODE_NONCAUSAL, true>(tdo, tv, tk, pq, BH * p.C, st);
+  // Otherwise (non-causal, or a forced split beyond the range table) the
+  // block loop over chunks from the scanned K^T V prefix (or total) states.
+  if (!dq_split) {
+    sm100::Params pq{};
+    pq.o = static_cast<__nv_bfloat16*>(dq);
+    pq.init_states = states ? s_kv : nullptr;
+    pq.N = N;
+    pq.L = p.L;
+    pq.C = p.C;
+    pq.units_per_seq = p.C;
+    pq.spin_limit = spin;
+    CUtensorMap tdq = tq;
+    if (sm100::Cfg<BK, D, DV>::TMA_STORE && !make_tmap_3d(&tdq, dq, BH, N, D, 16)) return LA2_ERR_CUDA;
+    {
+      LaunchTimer t(K_BWD_DQ_TC, st);
+      s = causal
+              ? launch_fwd_sm100<BK, D, DV, sm100::MODE_CAUSAL, true>(tdo, tv, tk, tdq, pq, BH * p.C, st)
+              : launch_fwd_sm100<BK, D, DV, sm100::MODE_NONCAUSAL, true>(tdo, tv, tk, tdq, pq, BH * p.C,
+                                                                        st);
+    }
+    if (s != LA2_OK) return s;
   }
-  if (s != LA2_OK) return s;
   sm100::BwdParams pb{};
   pb.dk = static_cast<__nv_bfloat16*>(dk);
   pb.dv = static_cast<__nv_bfloat16*>(dvv);
@@ -394,8 +441,12 @@ static la2_status backward_sm100_bk(const void* q, const void* k, const void* v,
   pb.C = p.C;
   pb.spin_limit = spin;
   pb.causal = causal;
+  CUtensorMap tdk = tq, tdv = tq;
+  if (sm100::BCfg<BK, D, DV>::TMA_STORE &&
+      (!make_tmap_3d(&tdk, dk, BH, N, D, 16) || !make_tmap_3d(&tdv, dvv, BH, N, DV, 16)))
+    return LA2_ERR_CUDA;
   LaunchTimer t(K_BWD_DKDV_TC, st);
-  return launch_bwd_dkdv_sm100<BK>(tq, tk, tv, tdo, pb, BH * p.C, st);
+  return launch_bwd_dkdv_sm100<BK>(tq, tk, tv, tdo, tdk, tdv, pb, BH * p.C, st);
 }
 
 static la2_status forward_sm100(const void* q, const void* k, const void* v, void* o, int64_t BH,
@@ -535,11 +586,19 @@ la2_status la2_backward(const void* q, const void* k, const void* v, const void*
   const int nel = (int)(d * dv);
   float* s_kv = p.need_states ? static_cast<float*>(workspace) : nullptr;
   float* s_u = p.need_states ? s_kv + (size_t)BH * p.C * nel : nullptr;
-  if (p.tc)
-    return block == 64 ? backward_sm100_bk<64>(q, k, v, dout, dq, dk, dvv, BH, N, causal, s_kv, s_u,
-                                                p, spin_limit(), st)
-                       : backward_sm100_bk<128>(q, k, v, dout, dq, dk, dvv, BH, N, causal, s_kv,
+  if (p.tc) {
+    float* second = nullptr;  // K^T V chunk states, or the dQ pass's range states
+    if (p.need_states) {
+      s_u = static_cast<float*>(workspace);
+      second = s_u + (size_t)BH * p.C * nel;
+    } else if (p.ws_bytes > 0) {
+      second = static_cast<float*>(workspace);
+    }
+    return block == 64 ? backward_sm100_bk<64>(q, k, v, dout, dq, dk, dvv, BH, N, causal, second,
+                                                s_u, p, spin_limit(), st)
+                       : backward_sm100_bk<128>(q, k, v, dout, dq, dk, dvv, BH, N, causal, second,
                                                  s_u, p, spin_limit(), st);
+  }
   if (p.need_states) {
     const bool bf = dt == LA2_BF16;
     s = bf ? run_chunk_states<__nv_bfloat16>(k, v, s_kv, BH, N, (int)d, (int)dv, p, st)

@@ -280,7 +280,11 @@ struct Cfg {
   static constexpr int OFF_V = OFF_K + KS * KTILE;
   static constexpr int OFF_P = OFF_V + KS * VTILE;
   static constexpr int OFF_SNAP = OFF_P + PTILE;
-  static constexpr int OFF_BAR = OFF_SNAP + SNAP;
+  // Bk=64: O leaves through two swizzled staging tiles and per-warp TMA stores.
+  static constexpr bool TMA_STORE = BK == 64;
+  static constexpr int OTILE = BK * DV * 2;
+  static constexpr int OFF_OST = OFF_SNAP + SNAP;
+  static constexpr int OFF_BAR = OFF_OST + (TMA_STORE ? 2 * OTILE : 0);
   static constexpr int NBAR = 2 * QS + 2 * KS + 16;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;  // + alignment slack
   // TMEM columns
@@ -340,15 +344,17 @@ __device__ __noinline__ bool wait_bar_slow(uint64_t* bar, uint32_t parity, int64
   uint64_t deadline = 0;
   while (!mbar_try_wait(bar, parity)) {
     ++n;
+    bool expired = n >= limit;
     if ((n & 63) == 0) {
       if (*abort_flag) return false;
       const uint64_t now = globaltimer_ns();
       if (deadline == 0) deadline = now + 20ull * 1000ull * 1000ull * 1000ull;  // 20 s
-      if (n >= limit || now > deadline) {
-        record_error(DEV_ERR_TIMEOUT, where);
-        *abort_flag = 1;
-        return false;
-      }
+      expired = expired || now > deadline;
+    }
+    if (expired) {
+      record_error(DEV_ERR_TIMEOUT, where);
+      *abort_flag = 1;
+      return false;
     }
   }
   return true;
@@ -366,6 +372,15 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   while (!mbar_try_wait(bar, parity)) {
     if (globaltimer_ns() > deadline) return;
   }
+}
+
+// A fp32 state (D x DV) in HBM is stored column-chunk-major: float4 j
+// (columns 4j..4j+3) of row r at float4 index j*D + r. The 32 threads of a
+// warp own 32 consecutive rows of a TMEM accumulator, so each of their
+// 16-byte accesses covers 512 contiguous bytes.
+template <int D>
+__device__ __forceinline__ int64_t state_f4(int r, int j) {
+  return static_cast<int64_t>(j) * D + r;
 }
 
 // Row of an M-row accumulator held by thread `t` of warpgroup-warp `w4`
@@ -388,7 +403,8 @@ template <int BK, int D, int DV, int MODE, bool DQ = false>
 __global__ void __launch_bounds__(kThreads, 1)
 la2_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_k,
-                     const __grid_constant__ CUtensorMap tm_v, const Params prm) {
+                     const __grid_constant__ CUtensorMap tm_v,
+                     const __grid_constant__ CUtensorMap tm_o, const Params prm) {
   using CF = Cfg<BK, D, DV>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -451,6 +467,7 @@ la2_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     tma_prefetch(&tm_q);
     tma_prefetch(&tm_k);
     tma_prefetch(&tm_v);
+    if (MODE != MODE_STATE && CF::TMA_STORE) tma_prefetch(&tm_o);
   }
   if (warp == kWarpMma) {
     tmem_alloc(b.tmem_base, kTmemCols);
@@ -504,7 +521,12 @@ la2_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
   } else if (warp == kWarpMma) {
     // ================================================================ MMA
-    if (lane == 0) {
+    // The whole warp runs the issue loop; one elected lane issues each
+    // tcgen05 instruction (warp-uniform bookkeeping).
+    {
+      auto wait_w = [&](uint64_t* bar, uint32_t par, int where) -> bool {
+        return __all_sync(0xffffffffu, wait_bar(bar, par, lim, b.abort_flag, where));
+      };
       const uint32_t tKV = tmem + CF::COL_KV;
       int snap_ph = 0;
       bool ok = true;
@@ -514,39 +536,39 @@ la2_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         const uint32_t ka = smem_u32(sK + ks * CF::KTILE);
         const uint32_t va = smem_u32(sV + ks * CF::VTILE);
         if constexpr (MODE == MODE_STATE) {
-          if (!wait_bar(&b.kv_full[ks], (i / CF::KS) & 1, lim, b.abort_flag, 10)) { ok = false; break; }
+          if (!wait_w(&b.kv_full[ks], (i / CF::KS) & 1, 10)) { ok = false; break; }
           tc_fence_after();
           for (int kk = 0; kk < BK / 16; ++kk)
-            mma_bf16_ss(tKV, make_desc(ka + kk * 2048, BK * 128, 1024),
+            mma_bf16_ss_warp(tKV, make_desc(ka + kk * 2048, BK * 128, 1024),
                         make_desc(va + kk * 2048, BK * 128, 1024), CF::ID_UPD, (i > 0 || kk > 0));
-          mma_commit(&b.kv_empty[ks]);
+          mma_commit_warp(&b.kv_empty[ks]);
           continue;
         }
-        if (!wait_bar(&b.q_full[qs], (i / CF::QS) & 1, lim, b.abort_flag, 11)) { ok = false; break; }
+        if (!wait_w(&b.q_full[qs], (i / CF::QS) & 1, 11)) { ok = false; break; }
         if (MODE == MODE_CAUSAL &&
-            !wait_bar(&b.kv_full[ks], (i / CF::KS) & 1, lim, b.abort_flag, 12)) { ok = false; break; }
+            !wait_w(&b.kv_full[ks], (i / CF::KS) & 1, 12)) { ok = false; break; }
         tc_fence_after();
         const int sb = CF::NSB == 2 ? (i & 1) : 0;
         const int s_use = CF::NSB == 2 ? (i >> 1) : i;
         const uint32_t tS = tmem + (sb ? CF::COL_S1 : CF::COL_S0);
         if (MODE == MODE_CAUSAL) {
           // S_i = Q_i K_i^T
-          if (!wait_bar(&b.s_empty[sb], (s_use & 1) ^ 1, lim, b.abort_flag, 13)) { ok = false; break; }
+          if (!wait_w(&b.s_empty[sb], (s_use & 1) ^ 1, 13)) { ok = false; break; }
           tc_fence_after();
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * BK * 128 + (kk & 3) * 32;
-            mma_bf16_ss(tS, make_desc(qa + off, 16, 1024), make_desc(ka + off, 16, 1024), CF::ID_S,
+            mma_bf16_ss_warp(tS, make_desc(qa + off, 16, 1024), make_desc(ka + off, 16, 1024), CF::ID_S,
                         kk > 0);
           }
-          mma_commit(&b.s_full[sb]);
+          mma_commit_warp(&b.s_full[sb]);
         }
         // O_i = Q_i * bf16(KV)
         const int ob = i & 1;
         const uint32_t tO = tmem + (ob ? CF::COL_O1 : CF::COL_O0);
-        if (!wait_bar(&b.o_empty[ob], ((i >> 1) & 1) ^ 1, lim, b.abort_flag, 14)) { ok = false; break; }
+        if (!wait_w(&b.o_empty[ob], ((i >> 1) & 1) ^ 1, 14)) { ok = false; break; }
         const bool have_snap = (i > 0) || has_init;
         if (have_snap && (MODE == MODE_CAUSAL || i == 0)) {
-          if (!wait_bar(b.snap_full, snap_ph, lim, b.abort_flag, 15)) { ok = false; break; }
+          if (!wait_w(b.snap_full, snap_ph, 15)) { ok = false; break; }
           snap_ph ^= 1;
         }
         tc_fence_after();
@@ -555,41 +577,41 @@ la2_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * BK * 128 + (kk & 3) * 32;
             if constexpr (DQ)  // B[n=c][k=e] = KV[c][e]: snapshot rows read K-major
-              mma_bf16_ss(tO, make_desc(qa + off, 16, 1024),
+              mma_bf16_ss_warp(tO, make_desc(qa + off, 16, 1024),
                           make_desc(sa + (kk >> 2) * D * 128 + (kk & 3) * 32, 16, 1024),
                           CF::ID_QKV_KMAJOR, kk > 0);
             else
-              mma_bf16_ss(tO, make_desc(qa + off, 16, 1024), make_desc(sa + kk * 2048, D * 128, 1024),
+              mma_bf16_ss_warp(tO, make_desc(qa + off, 16, 1024), make_desc(sa + kk * 2048, D * 128, 1024),
                           CF::ID_QKV, kk > 0);
           }
         }
-        mma_commit(&b.q_empty[qs]);
+        mma_commit_warp(&b.q_empty[qs]);
         if constexpr (MODE == MODE_NONCAUSAL) {
-          mma_commit(&b.o_full[ob]);
+          mma_commit_warp(&b.o_full[ob]);
           continue;
         }
         // KV += K_i^T V_i (after the snapshot of the old state was taken)
         for (int kk = 0; kk < BK / 16; ++kk)
-          mma_bf16_ss(tKV, make_desc((DQ ? va : ka) + kk * 2048, BK * 128, 1024),
+          mma_bf16_ss_warp(tKV, make_desc((DQ ? va : ka) + kk * 2048, BK * 128, 1024),
                       make_desc((DQ ? ka : va) + kk * 2048, BK * 128, 1024), CF::ID_UPD,
                       (have_snap || kk > 0) ? 1u : 0u);
-        mma_commit(b.kv_updated);
+        mma_commit_warp(b.kv_updated);
         // O_i += P_i V_i
-        if (!wait_bar(b.p_full, i & 1, lim, b.abort_flag, 16)) { ok = false; break; }
+        if (!wait_w(b.p_full, i & 1, 16)) { ok = false; break; }
         tc_fence_after();
         const uint32_t pa = smem_u32(sP);
         for (int kk = 0; kk < BK / 16; ++kk) {
           const uint32_t off = (kk >> 2) * BK * 128 + (kk & 3) * 32;
-          mma_bf16_ss(tO, make_desc(pa + off, 16, 1024), make_desc(va + kk * 2048, BK * 128, 1024),
+          mma_bf16_ss_warp(tO, make_desc(pa + off, 16, 1024), make_desc(va + kk * 2048, BK * 128, 1024),
                       CF::ID_PV, (have_snap || kk > 0) ? 1u : 0u);
         }
-        mma_commit(&b.o_full[ob]);
-        mma_commit(b.p_empty);
-        mma_commit(&b.kv_empty[ks]);
+        mma_commit_warp(&b.o_full[ob]);
+        mma_commit_warp(b.p_empty);
+        mma_commit_warp(&b.kv_empty[ks]);
       }
-      if (MODE == MODE_STATE && ok) mma_commit(b.kv_updated);
+      if (MODE == MODE_STATE && ok) mma_commit_warp(b.kv_updated);
       // All MMAs issued by this thread must finish before TMEM is released.
-      mma_commit(b.drain);
+      mma_commit_warp(b.drain);
       drain_wait(b.drain, 0);
     }
   } else if (wg == kWgMask) {
@@ -656,7 +678,7 @@ la2_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
     };
     if (MODE == MODE_STATE) {
-      // Chunk state out: TMEM (fp32) -> HBM, row-major [D][DV].
+      // Chunk state out: TMEM (fp32) -> HBM, column-chunk-major (state_f4).
       if (__all_sync(0xffffffffu, wait_bar(b.kv_updated, 0, lim, b.abort_flag, 30))) {
         tc_fence_after();
         float* dst = prm.out_states + (bh * prm.C + c) * (int64_t)(D * DV);
@@ -666,10 +688,10 @@ la2_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           tmem_ld32(tKV + c32 * 32, v);
           tmem_ld_wait();
           if (r >= 0) {
-            float4* p4 = reinterpret_cast<float4*>(dst + (int64_t)r * DV + c32 * 32);
+            float4* p4 = reinterpret_cast<float4*>(dst);
 #pragma unroll
             for (int q4 = 0; q4 < 8; ++q4)
-              p4[q4] = make_float4(__uint_as_float(v[4 * q4]), __uint_as_float(v[4 * q4 + 1]),
+              p4[state_f4<D>(r, c32 * 8 + q4)] = make_float4(__uint_as_float(v[4 * q4]), __uint_as_float(v[4 * q4 + 1]),
                                    __uint_as_float(v[4 * q4 + 2]), __uint_as_float(v[4 * q4 + 3]));
           }
         }
@@ -682,10 +704,10 @@ la2_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           float vals[32];
           uint32_t u[32];
           if (r >= 0) {
-            const float4* src = reinterpret_cast<const float4*>(init + (int64_t)r * DV + c32 * 32);
+            const float4* src = reinterpret_cast<const float4*>(init);
 #pragma unroll
             for (int q4 = 0; q4 < 8; ++q4) {
-              const float4 x = src[q4];
+              const float4 x = src[state_f4<D>(r, c32 * 8 + q4)];
               vals[4 * q4] = x.x; vals[4 * q4 + 1] = x.y; vals[4 * q4 + 2] = x.z; vals[4 * q4 + 3] = x.w;
             }
           } else {
@@ -736,6 +758,47 @@ la2_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         const uint32_t tO = tmem + (buf ? CF::COL_O1 : CF::COL_O0) + lane_off;
         if (!__all_sync(0xffffffffu, wait_bar(&b.o_full[buf], (i >> 1) & 1, lim, b.abort_flag, 40))) break;
         tc_fence_after();
+        if constexpr (CF::TMA_STORE) {
+          // Warp w4 stages its 16 rows (128B-swizzled 64-column panels) and
+          // stores them with TMA; rows past the chunk end are not written.
+          uint8_t* stage = smem + CF::OFF_OST + buf * CF::OTILE + w4 * 16 * 128;
+          if (lane == 0) bulk_wait_group_read<1>();  // this warp's store of block i-2 has read it
+          __syncwarp();
+          const int rl = lane & 15;
+#pragma unroll
+          for (int c32 = 0; c32 < DV / 32; ++c32) {
+            uint32_t v[32];
+            tmem_ld32(tO + c32 * 32, v);
+            tmem_ld_wait();
+            if (r >= 0) {
+              const uint32_t base = smem_u32(stage + (c32 >> 1) * BK * 128) + rl * 128;
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const int cj = (c32 & 1) * 4 + q;
+                st_shared_v4(base + ((cj ^ (rl & 7)) << 4),
+                             pack_bf16x2(__uint_as_float(v[8 * q]), __uint_as_float(v[8 * q + 1])),
+                             pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3])),
+                             pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5])),
+                             pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7])));
+              }
+            }
+          }
+          tc_fence_before();
+          mbar_arrive(&b.o_empty[buf]);
+          fence_proxy_async();
+          __syncwarp();
+          const int64_t y = t0 + static_cast<int64_t>(i) * BK + 16 * w4;
+          // A chunk ends on a block boundary or at N, so the tensor map's
+          // bound at N is the only clip needed.
+          if (lane == 0 && y < t1) {
+#pragma unroll
+            for (int p = 0; p < DV / 64; ++p)
+              tma_store_3d(&tm_o, stage + p * BK * 128, 64 * p, static_cast<int>(y),
+                           static_cast<int>(bh));
+            bulk_commit_group();
+          }
+          continue;
+        }
         const int64_t row = t0 + static_cast<int64_t>(i) * BK + r;
         const bool valid = r >= 0 && row < t1;
         uint4* dst = reinterpret_cast<uint4*>(ob + (valid ? row : 0) * DV);
@@ -756,6 +819,7 @@ la2_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         tc_fence_before();
         mbar_arrive(&b.o_empty[buf]);
       }
+      if (CF::TMA_STORE && lane == 0) bulk_wait_group<0>();  // stores done before exit
     }
   }
 
@@ -827,13 +891,13 @@ inline bool make_tmap_3d(CUtensorMap* m, const void* base, int64_t BH, int64_t N
 
 template <int BK, int D, int DV, int MODE, bool DQ = false>
 inline la2_status launch_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk,
-                                   const CUtensorMap& tv, const sm100::Params& p, int64_t units,
-                                   cudaStream_t st) {
+                                   const CUtensorMap& tv, const CUtensorMap& to,
+                                   const sm100::Params& p, int64_t units, cudaStream_t st) {
   using CF = sm100::Cfg<BK, D, DV>;
   auto kern = sm100::la2_fwd_sm100_kernel<BK, D, DV, MODE, DQ>;
   static bool attr_done[128];  // one per template instantiation
   if (!smem_attribute_set(kern, CF::SMEM, attr_done)) return LA2_ERR_CUDA;
-  kern<<<static_cast<unsigned>(units), sm100::kThreads, CF::SMEM, st>>>(tq, tk, tv, p);
+  kern<<<static_cast<unsigned>(units), sm100::kThreads, CF::SMEM, st>>>(tq, tk, tv, to, p);
   return cudaGetLastError() == cudaSuccess ? LA2_OK : LA2_ERR_CUDA;
 }
 

@@ -34,7 +34,11 @@ struct BCfg {
   static constexpr int OFF_PT = OFF_ST + NS * STAGE;
   static constexpr int OFF_PDT = OFF_PT + PTILE;
   static constexpr int OFF_SNAP = OFF_PDT + PTILE;
-  static constexpr int OFF_BAR = OFF_SNAP + SNAP;
+  // Bk=64: dV and dK leave through one swizzled staging tile each and
+  // per-warp TMA stores.
+  static constexpr bool TMA_STORE = BK == 64;
+  static constexpr int OFF_OST = OFF_SNAP + SNAP;
+  static constexpr int OFF_BAR = OFF_OST + (TMA_STORE ? 2 * TILE : 0);
   static constexpr int NBAR = 2 * NS + 12;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
   // TMEM columns: U, dV, dK (A^T aliases dK), S^T
@@ -49,7 +53,7 @@ struct BCfg {
 struct BwdParams {
   __nv_bfloat16* dk;       // [BH][N][D]
   __nv_bfloat16* dv;       // [BH][N][DV]
-  const float* init_u;     // [BH][C][D][DV]: suffix (causal) or total in slot 0 (non-causal)
+  const float* init_u;     // [BH][C][D*DV] (state_f4 layout): suffix (causal) or total in slot 0
   int64_t N, L, C;
   int64_t spin_limit;
   int causal;
@@ -60,7 +64,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 la2_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v,
-                          const __grid_constant__ CUtensorMap tm_do, const BwdParams prm) {
+                          const __grid_constant__ CUtensorMap tm_do,
+                          const __grid_constant__ CUtensorMap tm_dk,
+                          const __grid_constant__ CUtensorMap tm_dv, const BwdParams prm) {
   using CF = BCfg<BK, D, DV>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -113,6 +119,10 @@ la2_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     tma_prefetch(&tm_k);
     tma_prefetch(&tm_v);
     tma_prefetch(&tm_do);
+    if (CF::TMA_STORE) {
+      tma_prefetch(&tm_dk);
+      tma_prefetch(&tm_dv);
+    }
   }
   if (warp == kWarpMma) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -153,7 +163,12 @@ la2_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         for (int j = max(0, issued - CF::NS); j < issued; ++j) drain_wait(&st_full[j % CF::NS], (j / CF::NS) & 1);
     }
   } else if (warp == kWarpMma) {
-    if (lane == 0) {
+    // The whole warp runs the issue loop; one elected lane issues each
+    // tcgen05 instruction.
+    {
+      auto wait_w = [&](uint64_t* b, uint32_t par, int where) -> bool {
+        return __all_sync(0xffffffffu, wait_bar(b, par, lim, abort_flag, where));
+      };
       const uint64_t dKm = make_desc(0, 16, 1024);
       const uint64_t dMN = make_desc(0, BK * 128, 1024);
       const uint64_t dSnapMN = make_desc(0, D * 128, 1024);
@@ -166,26 +181,26 @@ la2_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         const int slot = s % CF::NS;
         const uint32_t aq = smem_u32(tile(slot, 0)), ak = smem_u32(tile(slot, 1));
         const uint32_t av = smem_u32(tile(slot, 2)), ado = smem_u32(tile(slot, 3));
-        if (!wait_bar(&st_full[slot], (s / CF::NS) & 1, lim, abort_flag, 210)) { ok = false; break; }
+        if (!wait_w(&st_full[slot], (s / CF::NS) & 1, 210)) { ok = false; break; }
         // the dK/dV accumulators (and the A^T scratch inside dK) must be free
-        if (!wait_bar(g_empty, (s & 1) ^ 1, lim, abort_flag, 211)) { ok = false; break; }
+        if (!wait_w(g_empty, (s & 1) ^ 1, 211)) { ok = false; break; }
         const bool have_u = s > 0 || has_init;
         if (causal) {
-          if (!wait_bar(s_read, (s & 1) ^ 1, lim, abort_flag, 212)) { ok = false; break; }
+          if (!wait_w(s_read, (s & 1) ^ 1, 212)) { ok = false; break; }
           tc_fence_after();
           // S^T = K Q^T and A^T = V dO^T (both K-major operands, K = 128)
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t off = ((kk >> 2) * BK * 128 + (kk & 3) * 32) >> 4;
-            mma_bf16_ss(tST, dKm + (ak >> 4) + off, dKm + (aq >> 4) + off, CF::ID_ST, kk > 0);
+            mma_bf16_ss_warp(tST, dKm + (ak >> 4) + off, dKm + (aq >> 4) + off, CF::ID_ST, kk > 0);
           }
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t off = ((kk >> 2) * BK * 128 + (kk & 3) * 32) >> 4;
-            mma_bf16_ss(tDK, dKm + (av >> 4) + off, dKm + (ado >> 4) + off, CF::ID_ST, kk > 0);
+            mma_bf16_ss_warp(tDK, dKm + (av >> 4) + off, dKm + (ado >> 4) + off, CF::ID_ST, kk > 0);
           }
-          mma_commit(s_full);
+          mma_commit_warp(s_full);
         }
         if (have_u && (causal || s == 0)) {
-          if (!wait_bar(snap_full, snap_ph, lim, abort_flag, 213)) { ok = false; break; }
+          if (!wait_w(snap_full, snap_ph, 213)) { ok = false; break; }
           snap_ph ^= 1;
         }
         tc_fence_after();
@@ -193,17 +208,17 @@ la2_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           // dV = K U: A = K (K-major, K = d), B[n=e][k=c] = U[c][e] (snapshot, MN-major)
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t off = ((kk >> 2) * BK * 128 + (kk & 3) * 32) >> 4;
-            mma_bf16_ss(tDV, dKm + (ak >> 4) + off, dSnapMN + (snap0 >> 4) + kk * (2048 >> 4), CF::ID_MN,
+            mma_bf16_ss_warp(tDV, dKm + (ak >> 4) + off, dSnapMN + (snap0 >> 4) + kk * (2048 >> 4), CF::ID_MN,
                         kk > 0);
           }
         }
         if (causal) {
           // U += Q^T dO (after the snapshot of the old U was taken)
           for (int kk = 0; kk < BK / 16; ++kk)
-            mma_bf16_ss(tU, dMN + (aq >> 4) + kk * (2048 >> 4), dMN + (ado >> 4) + kk * (2048 >> 4),
+            mma_bf16_ss_warp(tU, dMN + (aq >> 4) + kk * (2048 >> 4), dMN + (ado >> 4) + kk * (2048 >> 4),
                         CF::ID_UPD, (have_u || kk > 0) ? 1u : 0u);
           // dK region: A^T must have been read by the mask warpgroup
-          if (!wait_bar(s_read, s & 1, lim, abort_flag, 214)) { ok = false; break; }
+          if (!wait_w(s_read, s & 1, 214)) { ok = false; break; }
           tc_fence_after();
         }
         if (have_u) {
@@ -211,32 +226,32 @@ la2_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t off = ((kk >> 2) * BK * 128 + (kk & 3) * 32) >> 4;
             const uint32_t soff = ((kk >> 2) * D * 128 + (kk & 3) * 32) >> 4;
-            mma_bf16_ss(tDK, dKm + (av >> 4) + off, dKm + (snap0 >> 4) + soff, CF::ID_KM, kk > 0);
+            mma_bf16_ss_warp(tDK, dKm + (av >> 4) + off, dKm + (snap0 >> 4) + soff, CF::ID_KM, kk > 0);
           }
         }
         // U is updated and no issued MMA reads the snapshot any more: the
         // state warpgroup may take the next one
-        if (causal) mma_commit(u_updated);
+        if (causal) mma_commit_warp(u_updated);
         if (causal) {
-          if (!wait_bar(p_full, s & 1, lim, abort_flag, 215)) { ok = false; break; }
+          if (!wait_w(p_full, s & 1, 215)) { ok = false; break; }
           tc_fence_after();
           // dV += P^T dO ; dK += Pd^T Q  (A = masked tiles, K-major, K = BK; B MN-major)
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint32_t off = ((kk >> 2) * BK * 128 + (kk & 3) * 32) >> 4;
-            mma_bf16_ss(tDV, dKm + (pt0 >> 4) + off, dMN + (ado >> 4) + kk * (2048 >> 4), CF::ID_MN,
+            mma_bf16_ss_warp(tDV, dKm + (pt0 >> 4) + off, dMN + (ado >> 4) + kk * (2048 >> 4), CF::ID_MN,
                         (have_u || kk > 0) ? 1u : 0u);
           }
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint32_t off = ((kk >> 2) * BK * 128 + (kk & 3) * 32) >> 4;
-            mma_bf16_ss(tDK, dKm + (pdt0 >> 4) + off, dMN + (aq >> 4) + kk * (2048 >> 4), CF::ID_MN,
+            mma_bf16_ss_warp(tDK, dKm + (pdt0 >> 4) + off, dMN + (aq >> 4) + kk * (2048 >> 4), CF::ID_MN,
                         (have_u || kk > 0) ? 1u : 0u);
           }
-          mma_commit(p_empty);
+          mma_commit_warp(p_empty);
         }
-        mma_commit(g_full);
-        mma_commit(&st_empty[slot]);
+        mma_commit_warp(g_full);
+        mma_commit_warp(&st_empty[slot]);
       }
-      mma_commit(drain);
+      mma_commit_warp(drain);
       drain_wait(drain, 0);
     }
   } else if (wg == kWgMask) {
@@ -303,10 +318,10 @@ la2_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll 1
       for (int c32 = 0; c32 < DV / 32; ++c32) {
         uint32_t u[32];
-        const float4* src = reinterpret_cast<const float4*>(init + static_cast<int64_t>(r) * DV + c32 * 32);
+        const float4* src = reinterpret_cast<const float4*>(init);
 #pragma unroll
         for (int q4 = 0; q4 < 8; ++q4) {
-          const float4 x = src[q4];
+          const float4 x = src[state_f4<D>(r, c32 * 8 + q4)];
           u[4 * q4] = __float_as_uint(x.x);
           u[4 * q4 + 1] = __float_as_uint(x.y);
           u[4 * q4 + 2] = __float_as_uint(x.z);
@@ -346,6 +361,53 @@ la2_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       const int i = nblk - 1 - s;
       if (!__all_sync(0xffffffffu, wait_bar(g_full, s & 1, lim, abort_flag, 240))) break;
       tc_fence_after();
+      if constexpr (CF::TMA_STORE) {
+        // Warp w4 stages its 16 rows of dV and dK (128B-swizzled 64-column
+        // panels) and stores them with TMA.
+        if (lane == 0) bulk_wait_group_read<0>();  // this warp's stores of the last block have read
+        __syncwarp();
+        const int rl = lane & 15;
+        for (int which = 0; which < 2; ++which) {
+          uint8_t* stage = smem + CF::OFF_OST + which * CF::TILE + w4 * 16 * 128;
+          const uint32_t src = tmem + (which == 0 ? CF::COL_DV : CF::COL_DK) + lane_off;
+#pragma unroll
+          for (int c32 = 0; c32 < 128 / 32; ++c32) {
+            uint32_t v[32];
+            tmem_ld32(src + c32 * 32, v);
+            tmem_ld_wait();
+            if (r >= 0) {
+              const uint32_t base = smem_u32(stage + (c32 >> 1) * BK * 128) + rl * 128;
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const int cj = (c32 & 1) * 4 + q;
+                st_shared_v4(base + ((cj ^ (rl & 7)) << 4),
+                             pack_bf16x2(__uint_as_float(v[8 * q]), __uint_as_float(v[8 * q + 1])),
+                             pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3])),
+                             pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5])),
+                             pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7])));
+              }
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(g_empty);
+        fence_proxy_async();
+        __syncwarp();
+        // chunks end on block boundaries or at N (the tensor maps clip at N)
+        const int64_t y = t0 + static_cast<int64_t>(i) * BK + 16 * w4;
+        if (lane == 0 && y < t1) {
+          for (int which = 0; which < 2; ++which) {
+            uint8_t* stage = smem + CF::OFF_OST + which * CF::TILE + w4 * 16 * 128;
+            const CUtensorMap* map = which == 0 ? &tm_dv : &tm_dk;
+#pragma unroll
+            for (int p = 0; p < 2; ++p)
+              tma_store_3d(map, stage + p * BK * 128, 64 * p, static_cast<int>(y),
+                           static_cast<int>(bh));
+          }
+          bulk_commit_group();
+        }
+        continue;
+      }
       const int64_t row = t0 + static_cast<int64_t>(i) * BK + r;
       const bool valid = r >= 0 && row < t1;
       for (int which = 0; which < 2; ++which) {
@@ -372,6 +434,7 @@ la2_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       tc_fence_before();
       mbar_arrive(g_empty);
     }
+    if (CF::TMA_STORE && lane == 0) bulk_wait_group<0>();  // stores done before exit
   }
 
   tc_fence_before();
@@ -387,12 +450,14 @@ la2_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
 template <int BK>
 inline la2_status launch_bwd_dkdv_sm100(const CUtensorMap& tq, const CUtensorMap& tk,
                                         const CUtensorMap& tv, const CUtensorMap& tdo,
+                                        const CUtensorMap& tdk, const CUtensorMap& tdv,
                                         const sm100::BwdParams& p, int64_t units, cudaStream_t st) {
   using CF = sm100::BCfg<BK, 128, 128>;
   auto kern = sm100::la2_bwd_dkdv_sm100_kernel<BK, 128, 128>;
   static bool attr_done[128];
   if (!smem_attribute_set(kern, CF::SMEM, attr_done)) return LA2_ERR_CUDA;
-  kern<<<static_cast<unsigned>(units), sm100::kThreads, CF::SMEM, st>>>(tq, tk, tv, tdo, p);
+  kern<<<static_cast<unsigned>(units), sm100::kThreads, CF::SMEM, st>>>(tq, tk, tv, tdo, tdk, tdv,
+                                                                         p);
   return cudaGetLastError() == cudaSuccess ? LA2_OK : LA2_ERR_CUDA;
 }
 

@@ -190,10 +190,13 @@ struct StepIter {
   }
 };
 
-template <int BK, int D, int DV>
+template <int BK, int D, int DV, int KIND = KIND_MAIN>
 struct CCfg {
+  // The state-only pass (KIND_AGG) holds no Q, P, snapshot or O tiles and
+  // spends that space on a deeper K/V ring: its loads are latency-bound.
+  static constexpr bool AGG = KIND == KIND_AGG;
   static constexpr int QS = BK == 64 ? 3 : 1;
-  static constexpr int KS = BK == 64 ? 3 : 2;
+  static constexpr int KS = AGG ? (BK == 64 ? 6 : 3) : (BK == 64 ? 3 : 2);
   static constexpr int NSB = BK == 64 ? 2 : 1;    // S buffers (TMEM)
   static constexpr int NPB = BK == 64 ? 2 : 1;    // P buffers (SMEM)
   // One snapshot buffer suffices: the state role writes snapshot m+1 only after
@@ -202,7 +205,7 @@ struct CCfg {
   // Bk=64: O leaves through a swizzled staging tile and per-warp TMA stores
   // (plain row stores from the epilogue crowd the SM's memory-instruction
   // queue that the MMA warp's barrier and tcgen05 instructions also use).
-  static constexpr bool TMA_STORE = BK == 64;
+  static constexpr bool TMA_STORE = BK == 64 && !AGG;
   static constexpr int OSTAGE = TMA_STORE ? 2 : 0;
   // Q rides in the K/V ring (one barrier per step) when the rings are as deep.
   static constexpr bool QWITHKV = QS == KS;
@@ -217,11 +220,11 @@ struct CCfg {
   static constexpr int SNAP = D * DV * 2;
   static constexpr int OTILE = BK * DV * 2;
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + QS * QTILE;
+  static constexpr int OFF_K = OFF_Q + (AGG ? 0 : QS * QTILE);
   static constexpr int OFF_V = OFF_K + KS * KTILE;
   static constexpr int OFF_P = OFF_V + KS * VTILE;
-  static constexpr int OFF_SNAP = OFF_P + NPB * PTILE;
-  static constexpr int OFF_OST = OFF_SNAP + NSNAP * SNAP;
+  static constexpr int OFF_SNAP = OFF_P + (AGG ? 0 : NPB * PTILE);
+  static constexpr int OFF_OST = OFF_SNAP + (AGG ? 0 : NSNAP * SNAP);
   static constexpr int OFF_BAR = OFF_OST + OSTAGE * OTILE;
   static constexpr int NBAR = 2 * QS + 2 * KS + 15;  // rings + 6 pairs + 3 singles
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
@@ -356,7 +359,7 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_v,
                         const __grid_constant__ CUtensorMap tm_o,
                         const __grid_constant__ RangeTable rt, const CausalParams prm) {
-  using CF = CCfg<BK, D, DV>;
+  using CF = CCfg<BK, D, DV, KIND>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -956,7 +959,7 @@ inline la2_status launch_causal_sm100(const CUtensorMap& tq, const CUtensorMap& 
                                       const CUtensorMap& tv, const CUtensorMap& to,
                                       const sm100::RangeTable& rt,
                                       const sm100::CausalParams& p, int grid, cudaStream_t st) {
-  using CF = sm100::CCfg<BK, D, DV>;
+  using CF = sm100::CCfg<BK, D, DV, KIND>;
   auto kern = sm100::la2_causal_sm100_kernel<BK, D, DV, KIND>;
   static bool attr_done[128];  // one per template instantiation
   if (!smem_attribute_set(kern, CF::SMEM, attr_done)) return LA2_ERR_CUDA;
