@@ -48,6 +48,8 @@ def parse():
                     help="also print one line per sequence-length sweep point and the 512K case")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true",
+                    help="skip nvidia-smi clock sampling (and its extra steps), e.g. under a profiler")
     return ap.parse_args()
 
 
@@ -115,9 +117,10 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.monotonic(), line.strip()))
 
-    def stop(self):
+    def stop(self, t0=None, t1=None):
+        """Stop sampling; summarise the samples taken between host times t0 and t1."""
         if not self.proc:
             return None
         self.proc.terminate()
@@ -129,7 +132,9 @@ class ClockSampler:
             self.t.join(timeout=2)
         sm, smax, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        for t, ln in self.lines:
+            if (t0 is not None and t < t0) or (t1 is not None and t > t1):
+                continue
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 9:
                 continue
@@ -359,7 +364,7 @@ def bench_workload(args, w, dev, la2, world, rank, local, hbm, peak_kind, main):
         step(i)
     la2.check(stream)
 
-    sampler = ClockSampler(local) if main else None
+    sampler = ClockSampler(local) if main and not args.no_clocks else None
     la2.la2_profile_enable(1)
     _barrier(world)
     torch.cuda.synchronize(dev)
@@ -368,14 +373,36 @@ def bench_workload(args, w, dev, la2, world, rank, local, hbm, peak_kind, main):
         time.sleep(0.3)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
+    th0 = time.monotonic()
     e0.record(stream)
     for i in range(args.steps):
         step(i)
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    clocks = sampler.stop() if sampler else None
-    _barrier(world)
+    th1 = time.monotonic()
     la2.la2_profile_enable(0)
+    clocks = None
+    if sampler:
+        if th1 - th0 >= 1.0:
+            clocks = sampler.stop(th0, th1)
+            if clocks:
+                clocks["window"] = "timed region"
+        else:
+            # nvidia-smi samples every 100 ms: keep the same workload running
+            # (unprofiled, untimed) for about a second and sample there.
+            tw0 = time.monotonic()
+            n = 0
+            while time.monotonic() - tw0 < 1.2:
+                step(args.steps + n)
+                n += 1
+            torch.cuda.synchronize(dev)
+            tw1 = time.monotonic()
+            clocks = sampler.stop(tw0 + 0.1, tw1)
+            if clocks:
+                clocks["window"] = (f"{n} further steps of the same workload right after the timed "
+                                    f"region ({tw1 - tw0:.1f} s; the timed region lasted "
+                                    f"{1e3 * (th1 - th0):.1f} ms)")
+    _barrier(world)
     la2.check(stream)
     ms = e0.elapsed_time(e1)
     ms_max = _max_over_ranks(ms, world, dev)
