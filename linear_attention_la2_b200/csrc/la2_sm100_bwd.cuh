@@ -41,8 +41,13 @@ struct BCfg {
   static constexpr int OFF_BAR = OFF_OST + (TMA_STORE ? 2 * TILE : 0);
   static constexpr int NBAR = 2 * NS + 12;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
-  // TMEM columns: U, dV, dK (A^T aliases dK), S^T
+  // TMEM columns: U, dV, dK, S^T, A^T
   static constexpr uint32_t COL_U = 0, COL_DV = 128, COL_DK = 256, COL_ST = 384;
+  // Bk=64: A^T gets the last 64 columns, so the next block's S^T and A^T need
+  // not wait for the epilogue to read dK; Bk=128: A^T aliases dK.
+  static constexpr bool AT_OWN = BK == 64;
+  static constexpr uint32_t COL_AT = AT_OWN ? COL_ST + BK : COL_DK;
+  static_assert(COL_ST + BK + (AT_OWN ? BK : 0) <= 512, "TMEM columns");
   static constexpr uint32_t ID_ST = make_idesc(BK, BK, false, false);   // K Q^T, V dO^T
   static constexpr uint32_t ID_MN = make_idesc(BK, 128, false, true);   // X[K-major] * Y[MN-major]
   static constexpr uint32_t ID_KM = make_idesc(BK, 128, false, false);  // X[K-major] * Y[K-major]
@@ -173,7 +178,7 @@ la2_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       const uint64_t dMN = make_desc(0, BK * 128, 1024);
       const uint64_t dSnapMN = make_desc(0, D * 128, 1024);
       const uint32_t tU = tmem + CF::COL_U, tDV = tmem + CF::COL_DV, tDK = tmem + CF::COL_DK;
-      const uint32_t tST = tmem + CF::COL_ST;
+      const uint32_t tST = tmem + CF::COL_ST, tAT = tmem + CF::COL_AT;
       const uint32_t snap0 = smem_u32(sSnap), pt0 = smem_u32(sPT), pdt0 = smem_u32(sPdT);
       int snap_ph = 0;
       bool ok = true;
@@ -182,8 +187,8 @@ la2_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         const uint32_t aq = smem_u32(tile(slot, 0)), ak = smem_u32(tile(slot, 1));
         const uint32_t av = smem_u32(tile(slot, 2)), ado = smem_u32(tile(slot, 3));
         if (!wait_w(&st_full[slot], (s / CF::NS) & 1, 210)) { ok = false; break; }
-        // the dK/dV accumulators (and the A^T scratch inside dK) must be free
-        if (!wait_w(g_empty, (s & 1) ^ 1, 211)) { ok = false; break; }
+        // A^T aliasing dK: the epilogue must have read the last block's dK
+        if (!CF::AT_OWN && !wait_w(g_empty, (s & 1) ^ 1, 211)) { ok = false; break; }
         const bool have_u = s > 0 || has_init;
         if (causal) {
           if (!wait_w(s_read, (s & 1) ^ 1, 212)) { ok = false; break; }
@@ -195,10 +200,12 @@ la2_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           }
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t off = ((kk >> 2) * BK * 128 + (kk & 3) * 32) >> 4;
-            mma_bf16_ss_warp(tDK, dKm + (av >> 4) + off, dKm + (ado >> 4) + off, CF::ID_ST, kk > 0);
+            mma_bf16_ss_warp(tAT, dKm + (av >> 4) + off, dKm + (ado >> 4) + off, CF::ID_ST, kk > 0);
           }
           mma_commit_warp(s_full);
         }
+        // the dK/dV accumulators must be free (the epilogue read the last block's)
+        if (CF::AT_OWN && !wait_w(g_empty, (s & 1) ^ 1, 216)) { ok = false; break; }
         if (have_u && (causal || s == 0)) {
           if (!wait_w(snap_full, snap_ph, 213)) { ok = false; break; }
           snap_ph ^= 1;
@@ -217,9 +224,11 @@ la2_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           for (int kk = 0; kk < BK / 16; ++kk)
             mma_bf16_ss_warp(tU, dMN + (aq >> 4) + kk * (2048 >> 4), dMN + (ado >> 4) + kk * (2048 >> 4),
                         CF::ID_UPD, (have_u || kk > 0) ? 1u : 0u);
-          // dK region: A^T must have been read by the mask warpgroup
-          if (!wait_w(s_read, s & 1, 214)) { ok = false; break; }
-          tc_fence_after();
+          // A^T aliasing dK: the mask warpgroup must have read it
+          if (!CF::AT_OWN) {
+            if (!wait_w(s_read, s & 1, 214)) { ok = false; break; }
+            tc_fence_after();
+          }
         }
         if (have_u) {
           // dK = V U^T: A = V (K-major, K = dv), B[n=c][k=e] = U[c][e] (snapshot, K-major)
@@ -260,7 +269,7 @@ la2_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       const int r = acc_row<BK>(w4, lane);
       const uint32_t lane_off = static_cast<uint32_t>(32 * w4) << 16;
       const uint32_t bases[2] = {smem_u32(sPT), smem_u32(sPdT)};
-      const uint32_t srcs[2] = {tmem + CF::COL_ST + lane_off, tmem + CF::COL_DK + lane_off};
+      const uint32_t srcs[2] = {tmem + CF::COL_ST + lane_off, tmem + CF::COL_AT + lane_off};
       for (int s = 0; s < nblk; ++s) {
         if (!__all_sync(0xffffffffu, wait_bar(s_full, s & 1, lim, abort_flag, 220))) break;
         if (!__all_sync(0xffffffffu, wait_bar(p_empty, (s & 1) ^ 1, lim, abort_flag, 221))) break;

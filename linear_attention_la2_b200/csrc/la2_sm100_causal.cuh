@@ -872,7 +872,7 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
 // block moves half the bytes and its loads stay latency-bound).
 constexpr double kPrepassCost = 0.5;
 constexpr double kRangeStateCost = 0.5;  // separate state launch, per block
-constexpr double kLaunchCost = 3.0;      // extra launch + initial-state sum, in main blocks
+constexpr double kLaunchCost = 8.0;      // extra launch + initial-state sum, in main blocks
 
 struct RangePlan {
   int R = 0;
