@@ -4,8 +4,10 @@ from .la2_oracle import (  # noqa: F401
     backward,
     backward_rows,
     blocked_forward,
+    decode_step,
     forward,
     forward_rows,
+    kv_state,
     recurrent_forward,
     relative_frobenius,
 )

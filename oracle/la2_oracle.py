@@ -30,7 +30,9 @@ All arithmetic is float64 on the exact (already rounded) input values.
 ``forward`` / ``backward`` / ``*_rows`` are the plain definition. ``recurrent_*``
 is the RNN form and ``blocked_forward`` the block algorithm of point 2; those two
 exist to pin the definition (and to check very long sequences where the O(N^2)
-definition is too slow on a CPU), never the other way round.
+definition is too slow on a CPU), never the other way round. ``kv_state`` (the
+state after a prefill) and ``decode_step`` (one RNN-mode step) are the oracle of
+the inference form.
 
 Parity status: every function here is pinned by ``tests/test_oracle.py``
 (brute force on tiny integer inputs, closed forms, RNN-form equality, block-size
@@ -200,6 +202,43 @@ def recurrent_forward(q, k, v) -> np.ndarray:
                 kv += np.outer(k[b, h, t], v[b, h, t])
                 out[b, h, t] = q[b, h, t] @ kv
     return out
+
+
+def kv_state(k, v, state=None) -> np.ndarray:
+    """The KV state a causal pass leaves behind: ``state + sum_t k_t^T v_t``.
+
+    Shapes ``k [B,H,N,d]``, ``v [B,H,N,dv]``, ``state [B,H,d,dv]`` (zero when
+    omitted). This is the state the block algorithm of point 2 carries past a
+    sequence's last block, and the state an RNN-mode step (speed section)
+    continues from. Defined as a plain sum of outer products.
+    """
+    k, v = _f64(k), _f64(v)
+    if k.ndim != 4 or v.ndim != 4 or k.shape[:3] != v.shape[:3]:
+        raise ValueError("k [B,H,N,d] and v [B,H,N,dv] expected")
+    out = np.zeros(k.shape[:2] + (k.shape[3], v.shape[3])) if state is None else _f64(state).copy()
+    for b in range(k.shape[0]):
+        for h in range(k.shape[1]):
+            for t in range(k.shape[2]):
+                out[b, h] += np.outer(k[b, h, t], v[b, h, t])
+    return out
+
+
+def decode_step(q, k, v, state):
+    """One RNN-mode step for one new token per (b, h) (article, speed section).
+
+    ``q, k [B,H,d]``, ``v [B,H,dv]``, ``state [B,H,d,dv]``. Returns
+    ``(o, new_state)`` with ``new_state = state + k^T v`` and
+    ``o = q new_state``: the token's own pair is included, as the diagonal of
+    the causal mask is in the left product.
+    """
+    q, k, v, s = _f64(q), _f64(k), _f64(v), _f64(state)
+    if q.ndim != 3 or k.shape != q.shape or v.shape[:2] != q.shape[:2]:
+        raise ValueError("q, k [B,H,d] and v [B,H,dv] expected")
+    if s.shape != q.shape[:2] + (q.shape[2], v.shape[2]):
+        raise ValueError("state [B,H,d,dv] expected")
+    new = s + k[..., :, None] * v[..., None, :]
+    o = np.einsum("bhd,bhde->bhe", q, new)
+    return o, new
 
 
 def blocked_forward(q, k, v, block: int, causal: bool = True) -> np.ndarray:
