@@ -45,7 +45,10 @@ def parse():
     ap.add_argument("--N", type=int, default=0, help="override the sequence length")
     ap.add_argument("--impl", default="la2", choices=["la2", "reference"])
     ap.add_argument("--sweep", action="store_true",
-                    help="also print one line per sequence-length sweep point and the 512K case")
+                    help="also print one line per sequence-length sweep point, the 512K case and "
+                         "the decode step")
+    ap.add_argument("--decode", action="store_true",
+                    help="also print the decode-step line (one RNN-mode token per sequence)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true",
@@ -287,6 +290,10 @@ def run_gpu(args):
         ln = bench_workload(args, lw, dev, la2, world, rank, local, hbm, peak_kind, main=False)
         if rank == 0:
             print(json.dumps(ln), flush=True)
+    if args.sweep or args.decode:
+        ln = bench_decode(args, dev, la2, world, hbm, peak_kind)
+        if rank == 0:
+            print(json.dumps(ln), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -452,6 +459,73 @@ def bench_workload(args, w, dev, la2, world, rank, local, hbm, peak_kind, main):
         line["cpu_baseline"] = {"value": r, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                                 "sample": sample}
     return line
+
+
+DECODE = dict(name="bf16_decode_b64h32", B=64, H=32, d=128, dv=128, seed=5)
+
+
+def bench_decode(args, dev, la2, world, hbm, peak_kind):
+    """One step = one new token for each of the B*H sequences through
+    la2_decode_step (state += k^T v, o = q state) on a [B,H,d,dv] fp32 state that
+    is larger than L2; q, k, v rotate over 8 sets."""
+    import torch
+
+    c = DECODE
+    B, H, d, dv = c["B"], c["H"], c["d"], c["dv"]
+    g = torch.Generator().manual_seed(c["seed"])
+    sets = [tuple((torch.randn((B, H, n), generator=g) / math.sqrt(d)).to(torch.bfloat16).to(dev)
+                  for n in (d, d, dv)) for _ in range(8)]
+    state = (torch.randn((B, H, d, dv), generator=g) * 0.01).to(dev)
+    o = torch.empty((B, H, dv), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    st = la2._stream_handle(stream)
+
+    def step(i):
+        q, k, v = sets[i % len(sets)]
+        rc = la2.la2_decode_step(la2._ptr(q), la2._ptr(k), la2._ptr(v), la2._ptr(o),
+                                 la2._ptr(state), B, H, d, dv, la2.LA2_BF16, st)
+        if rc != 0:
+            raise la2.La2Error(rc)
+
+    for i in range(args.warmup):
+        step(i)
+    la2.check(stream)
+    la2.la2_profile_enable(1)
+    _barrier(world)
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    la2.la2_profile_enable(0)
+    _barrier(world)
+    la2.check(stream)
+    ms_max = _max_over_ranks(e0.elapsed_time(e1), world, dev)
+    per_kernel = {}
+    for kid in range(la2.la2_profile_num_kernels()):
+        n, kms = la2.la2_profile_collect(kid)
+        if n:
+            per_kernel[la2.la2_profile_kernel_name(kid)] = {"launches": n, "ms": kms}
+    k_ms = per_kernel["la2_decode_step"]["ms"] / per_kernel["la2_decode_step"]["launches"]
+    bytes_step = B * H * (2 * d * dv * 4 + (2 * d + 2 * dv) * 2)
+    achieved = bytes_step / (k_ms / 1e3) / 1e9
+    return {
+        "metric": "decode tokens/s (one RNN-mode token per (b,h) sequence), 1 B200",
+        "value": whole_job_rate(B * H, args.steps, world, ms_max), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{c['name']}: decode step B={B} H={H} d={d} dv={dv} bf16 q/k/v/o, "
+                               "fp32 state", "B": B, "H": H, "d": d, "dv": dv,
+                   "l2": f"state {B * H * d * dv * 4 / 1e6:.0f} MB > L2"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": None, "kernel": "la2_decode_step",
+                     "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)"},
+        "gpu_launches": sum(v["launches"] for v in per_kernel.values()), "kernels": per_kernel,
+    }
 
 
 def e2e_measure(args, w, dev, la2, world, base, ws, ws_bytes, dt):

@@ -139,6 +139,40 @@ LA2_API int64_t la2_plan_ranges(int64_t B, int64_t H, int64_t N, int64_t d, int6
                                 int64_t *starts, int64_t cap);
 
 /*
+ * Inference form (article, section "Lightning Attention-2速度对比": linear
+ * attention converts losslessly to an RNN; section "Lightning Attention-2简介",
+ * point 2: the KV state carried from block to block). A per-sequence state
+ * S is d x dv fp32, row-major; `state` is [B, H, d, dv] fp32 device memory
+ * owned by the caller, 16-byte aligned, updated in place.
+ *
+ * la2_kv_state: the state a prefill leaves, S += sum_t k_t^T v_t over the N
+ * tokens of each sequence (pass a zeroed state for a fresh sequence; a later
+ * call continues it). k [B,H,N,d], v [B,H,N,dv] in `dt`; shapes as for
+ * la2_forward with block 64. Scratch: la2_kv_state_workspace_size() bytes of
+ * `workspace` (256-byte aligned; (size_t)-1 for an invalid shape). The per-chunk
+ * states are summed in a fixed order, so repeated calls give identical bits.
+ * Errors as for la2_forward; `state` must not overlap k, v or the workspace.
+ */
+LA2_API size_t la2_kv_state_workspace_size(int64_t B, int64_t H, int64_t N, int64_t d, int64_t dv,
+                                           la2_dtype dt);
+LA2_API la2_status la2_kv_state(const void *k, const void *v, float *state, int64_t B, int64_t H,
+                                int64_t N, int64_t d, int64_t dv, la2_dtype dt, void *workspace,
+                                size_t workspace_bytes, la2_stream_t stream);
+
+/*
+ * la2_decode_step: one new token per sequence in RNN form,
+ *     S += k^T v,   o = q S
+ * (the token's own pair counts, as the diagonal of the causal mask does).
+ * q, k [B,H,d], v, o [B,H,dv] in `dt` (aligned to their element size), state
+ * as above. Any d, dv >= 1 and both dtypes; fp32 arithmetic. Continuing from
+ * la2_kv_state over tokens 0..N-1, step t gives row t of la2_forward's causal
+ * output. o must not overlap any input or the state; B or H = 0 is empty.
+ */
+LA2_API la2_status la2_decode_step(const void *q, const void *k, const void *v, void *o,
+                                   float *state, int64_t B, int64_t H, int64_t d, int64_t dv,
+                                   la2_dtype dt, la2_stream_t stream);
+
+/*
  * Upper bound, in spin iterations, of every device-side wait (mbarrier or
  * flag). When a wait exceeds it the kernel records LA2_ERR_TIMEOUT in the
  * device error word, stops its work and returns; la2_check() reports it.

@@ -15,6 +15,7 @@
 
 #include "la2.h"
 #include "la2_common.cuh"
+#include "la2_decode.cuh"
 #include "la2_simt.cuh"
 #include "la2_sm100.cuh"
 #include "la2_sm100_causal.cuh"
@@ -34,13 +35,16 @@ enum KernelId : int {
   K_STATE_TC,
   K_BWD_DQ_TC,
   K_BWD_DKDV_TC,
+  K_DECODE,
+  K_STATE_ACC,
   K_COUNT
 };
 
 static const char* kKernelNames[K_COUNT] = {
     "la2_chunk_state_simt", "la2_chunk_scan",      "la2_fwd_simt",
     "la2_bwd_dq_simt",      "la2_bwd_dkdv_simt",   "la2_fwd_sm100",
-    "la2_chunk_state_sm100", "la2_bwd_dq_sm100",   "la2_bwd_dkdv_sm100"};
+    "la2_chunk_state_sm100", "la2_bwd_dq_sm100",   "la2_bwd_dkdv_sm100",
+    "la2_decode_step",      "la2_state_accumulate"};
 
 struct EventRecord {
   int kernel;
@@ -506,6 +510,111 @@ la2_status la2_set_spin_limit(int64_t iterations) {
   if (iterations < 0) return LA2_ERR_INVALID_ARG;
   g_spin_limit = iterations;
   return LA2_OK;
+}
+
+size_t la2_kv_state_workspace_size(int64_t B, int64_t H, int64_t N, int64_t d, int64_t dv,
+                                   la2_dtype dt) {
+  if (check_shape(B, H, N, d, dv, 0, 64, dt, false) != LA2_OK) return (size_t)-1;
+  if (B == 0 || H == 0 || N == 0) return 0;
+  const int sms = device_sm_count();
+  if (sms <= 0) return (size_t)-1;
+  return make_plan(B, H, N, d, dv, 0, 64, dt, false, sms).ws_bytes;
+}
+
+la2_status la2_kv_state(const void* k, const void* v, float* state, int64_t B, int64_t H, int64_t N,
+                        int64_t d, int64_t dv, la2_dtype dt, void* workspace,
+                        size_t workspace_bytes, la2_stream_t stream) {
+  la2_status s = check_shape(B, H, N, d, dv, 0, 64, dt, false);
+  if (s != LA2_OK) return s;
+  if (B == 0 || H == 0 || N == 0) return LA2_OK;
+  if (!k || !v || !state) return LA2_ERR_INVALID_ARG;
+  if (!is_aligned(k, 16) || !is_aligned(v, 16) || !is_aligned(state, 16)) return LA2_ERR_INVALID_ARG;
+  const size_t es = dt == LA2_BF16 ? 2 : 4;
+  const int64_t BH = B * H;
+  const size_t nk = (size_t)BH * N * d * es, nv = (size_t)BH * N * dv * es;
+  const size_t ns = (size_t)BH * d * dv * sizeof(float);
+  if (overlaps(state, ns, k, nk) || overlaps(state, ns, v, nv)) return LA2_ERR_INVALID_ARG;
+  const int sms = device_sm_count();
+  if (sms <= 0) return LA2_ERR_CUDA;
+  // The non-causal plan: per-chunk states K_c^T V_c, then their sum per sequence.
+  const Plan p = make_plan(B, H, N, d, dv, 0, 64, dt, false, sms);
+  if (!workspace || workspace_bytes < p.ws_bytes) return LA2_ERR_WORKSPACE;
+  if (!is_aligned(workspace, 256)) return LA2_ERR_INVALID_ARG;
+  if (overlaps(workspace, p.ws_bytes, state, ns)) return LA2_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  float* chunks = static_cast<float*>(workspace);
+  if (p.tc) {
+    CUtensorMap tk, tv;
+    if (!make_tmap_3d(&tk, k, BH, N, 128, 64) || !make_tmap_3d(&tv, v, BH, N, 128, 64))
+      return LA2_ERR_CUDA;
+    sm100::Params ps{};
+    ps.N = N;
+    ps.L = p.L;
+    ps.C = p.C;
+    ps.units_per_seq = p.C;
+    ps.out_states = chunks;
+    ps.spin_limit = spin_limit();
+    LaunchTimer t(K_STATE_TC, st);
+    s = launch_fwd_sm100<64, 128, 128, sm100::MODE_STATE>(tk, tk, tv, tk, ps, BH * p.C, st);
+  } else {
+    s = dt == LA2_BF16 ? run_chunk_states<__nv_bfloat16>(k, v, chunks, BH, N, (int)d, (int)dv, p, st)
+                       : run_chunk_states<float>(k, v, chunks, BH, N, (int)d, (int)dv, p, st);
+  }
+  if (s != LA2_OK) return s;
+  const int nel = (int)(d * dv);
+  LaunchTimer t(K_STATE_ACC, st);
+  state_accumulate_kernel<<<dim3((unsigned)((nel + 255) / 256), (unsigned)BH), 256, 0, st>>>(
+      chunks, state, p.C, (int)d, (int)dv, p.tc ? 1 : 0);
+  return launch_status();
+}
+
+la2_status la2_decode_step(const void* q, const void* k, const void* v, void* o, float* state,
+                           int64_t B, int64_t H, int64_t d, int64_t dv, la2_dtype dt,
+                           la2_stream_t stream) {
+  if (B < 0 || H < 0 || d < 1 || dv < 1) return LA2_ERR_INVALID_ARG;
+  if (dt != LA2_F32 && dt != LA2_BF16) return LA2_ERR_INVALID_ARG;
+  if (double(B) * double(H) * double(d) * double(dv) > 9.0e18) return LA2_ERR_INVALID_ARG;
+  if (B == 0 || H == 0) return LA2_OK;
+  if (!q || !k || !v || !o || !state) return LA2_ERR_INVALID_ARG;
+  const size_t es = dt == LA2_BF16 ? 2 : 4;
+  if (!is_aligned(q, es) || !is_aligned(k, es) || !is_aligned(v, es) || !is_aligned(o, es) ||
+      !is_aligned(state, 4))
+    return LA2_ERR_INVALID_ARG;
+  const int64_t BH = B * H;
+  if (BH > 0x7fffffff || (dv + 31) / 32 > 65535) return LA2_ERR_UNSUPPORTED;
+  const size_t nq = (size_t)BH * d * es, nv = (size_t)BH * dv * es;
+  const size_t ns = (size_t)BH * d * dv * sizeof(float);
+  if (overlaps(o, nv, q, nq) || overlaps(o, nv, k, nq) || overlaps(o, nv, v, nv) ||
+      overlaps(o, nv, state, ns) || overlaps(state, ns, q, nq) || overlaps(state, ns, k, nq) ||
+      overlaps(state, ns, v, nv))
+    return LA2_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  LaunchTimer t(K_DECODE, st);
+  // Four columns per lane when rows of the state, v and o allow 16-, 8- or
+  // 16-byte vector accesses.
+  if (dv % 4 == 0 && is_aligned(state, 16) && is_aligned(v, 4 * es) && is_aligned(o, es)) {
+    const dim3 grid4((unsigned)BH, (unsigned)((dv + 127) / 128));
+    if (dt == LA2_BF16)
+      decode_step_v4_kernel<__nv_bfloat16><<<grid4, 32 * kDecodeWarps, 0, st>>>(
+          static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+          static_cast<const __nv_bfloat16*>(v), static_cast<__nv_bfloat16*>(o), state, (int)d,
+          (int)dv);
+    else
+      decode_step_v4_kernel<float><<<grid4, 32 * kDecodeWarps, 0, st>>>(
+          static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
+          static_cast<float*>(o), state, (int)d, (int)dv);
+    return launch_status();
+  }
+  const dim3 grid((unsigned)BH, (unsigned)((dv + 31) / 32));
+  if (dt == LA2_BF16)
+    decode_step_kernel<__nv_bfloat16><<<grid, 32 * kDecodeWarps, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+        static_cast<const __nv_bfloat16*>(v), static_cast<__nv_bfloat16*>(o), state, (int)d, (int)dv);
+  else
+    decode_step_kernel<float><<<grid, 32 * kDecodeWarps, 0, st>>>(
+        static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
+        static_cast<float*>(o), state, (int)d, (int)dv);
+  return launch_status();
 }
 
 la2_status la2_forward(const void* q, const void* k, const void* v, void* o, int64_t B, int64_t H,

@@ -56,6 +56,9 @@ _SIGS = {
     "la2_version": (_int, []),
     "la2_forward_noalloc": (_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _int, _int,
                                    _int, _vp]),
+    "la2_kv_state_workspace_size": (_sz, [_i64, _i64, _i64, _i64, _i64, _int]),
+    "la2_kv_state": (_int, [_vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _int, _vp, _sz, _vp]),
+    "la2_decode_step": (_int, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _int, _vp]),
 }
 
 EXPORTED = tuple(_SIGS)
@@ -77,6 +80,9 @@ la2_profile_enable = _lib.la2_profile_enable
 la2_profile_num_kernels = _lib.la2_profile_num_kernels
 la2_version = _lib.la2_version
 la2_forward_noalloc = _lib.la2_forward_noalloc
+la2_kv_state_workspace_size = _lib.la2_kv_state_workspace_size
+la2_kv_state = _lib.la2_kv_state
+la2_decode_step = _lib.la2_decode_step
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -202,6 +208,46 @@ def backward(q, k, v, do, causal: bool = True, block: int = 64, outs=None, works
                         d, dv, int(causal), block, dt, _ptr(ws), ws.numel() if ws is not None else 0,
                         _stream_handle(stream)))
     return dq, dk, dvv
+
+
+def kv_state(k, v, state=None, workspace=None, stream=None):
+    """state += sum_t k_t^T v_t per sequence; k [B,H,N,d], v [B,H,N,dv] CUDA
+    tensors, state [B,H,d,dv] float32 (zeros if omitted). Returns the state."""
+    import torch
+
+    _check_inputs(k, v)
+    B, H, N, d = k.shape
+    dv = v.shape[-1]
+    dt = _dtype_code(k)
+    if state is None:
+        state = torch.zeros((B, H, d, dv), dtype=torch.float32, device=k.device)
+    _check_inputs(state)
+    if state.dtype != torch.float32:
+        raise La2Error(LA2_ERR_INVALID_ARG)
+    need = la2_kv_state_workspace_size(B, H, N, d, dv, dt)
+    if need == ctypes.c_size_t(-1).value:
+        raise La2Error(LA2_ERR_INVALID_ARG)
+    ws = workspace if workspace is not None else _workspace(need, k.device)
+    _raise(la2_kv_state(_ptr(k), _ptr(v), _ptr(state), B, H, N, d, dv, dt, _ptr(ws),
+                        ws.numel() if ws is not None else 0, _stream_handle(stream)))
+    return state
+
+
+def decode_step(q, k, v, state, out=None, stream=None):
+    """One RNN-mode token per sequence: state += k^T v, o = q state. q, k [B,H,d],
+    v [B,H,dv] CUDA tensors, state [B,H,d,dv] float32 (updated in place). Returns o."""
+    import torch
+
+    _check_inputs(q, k, v, state)
+    if state.dtype != torch.float32:
+        raise La2Error(LA2_ERR_INVALID_ARG)
+    B, H, d = q.shape
+    dv = v.shape[-1]
+    if out is None:
+        out = torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
+    _raise(la2_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(state), B, H, d, dv,
+                           _dtype_code(q), _stream_handle(stream)))
+    return out
 
 
 def check(stream=None):

@@ -119,3 +119,40 @@ def test_profiler_names():
     assert all(names) and len(set(names)) == n
     assert la2.la2_profile_kernel_name(n) == ""
     assert la2.la2_version() > 0
+
+
+def _dec(**kw):
+    a = dict(q=NULL, k=NULL, v=NULL, o=NULL, s=NULL, B=1, H=2, d=64, dv=32, dt=la2.LA2_BF16)
+    a.update(kw)
+    return la2.la2_decode_step(a["q"], a["k"], a["v"], a["o"], a["s"], a["B"], a["H"], a["d"],
+                               a["dv"], a["dt"], NULL)
+
+
+def test_decode_step_rejects_bad_arguments():
+    P = [ctypes.c_void_p(0x100000 * (i + 1)) for i in range(5)]
+    ok = dict(q=P[0], k=P[1], v=P[2], o=P[3], s=P[4])
+    assert _dec() == la2.LA2_ERR_INVALID_ARG                     # NULL pointers
+    assert _dec(B=0) == la2.LA2_OK                               # empty problem
+    assert _dec(d=0, **ok) == la2.LA2_ERR_INVALID_ARG
+    assert _dec(dv=-1, **ok) == la2.LA2_ERR_INVALID_ARG
+    assert _dec(dt=9, **ok) == la2.LA2_ERR_INVALID_ARG
+    assert _dec(**dict(ok, q=ctypes.c_void_p(0x100001))) == la2.LA2_ERR_INVALID_ARG  # misaligned
+    assert _dec(**dict(ok, s=ctypes.c_void_p(0x100002))) == la2.LA2_ERR_INVALID_ARG  # state misaligned
+    assert _dec(**dict(ok, o=ctypes.c_void_p(0x100000 + 64))) == la2.LA2_ERR_INVALID_ARG  # o overlaps q
+    # the state (2*64*32*4 = 16 KiB) overlaps v when placed just before it
+    assert _dec(**dict(ok, s=ctypes.c_void_p(0x300000 - 4096))) == la2.LA2_ERR_INVALID_ARG
+
+
+def test_kv_state_rejects_bad_arguments():
+    ks = la2.la2_kv_state
+    bad = ctypes.c_size_t(-1).value
+    assert la2.la2_kv_state_workspace_size(1, 1, 16, 64, 64, 7) == bad
+    assert la2.la2_kv_state_workspace_size(1, 1, 16, 96, 64, la2.LA2_BF16) == bad
+    assert la2.la2_kv_state_workspace_size(0, 1, 16, 64, 64, la2.LA2_F32) == 0
+    assert ks(NULL, NULL, NULL, 1, 1, 16, 64, 64, la2.LA2_F32, NULL, 0, NULL) == la2.LA2_ERR_INVALID_ARG
+    assert ks(NULL, NULL, NULL, 1, 0, 16, 64, 64, la2.LA2_F32, NULL, 0, NULL) == la2.LA2_OK
+    assert ks(NULL, NULL, NULL, 1, 1, -2, 64, 64, la2.LA2_F32, NULL, 0, NULL) == la2.LA2_ERR_INVALID_ARG
+    P = [ctypes.c_void_p(0x1000000 * (i + 1)) for i in range(3)]
+    # state overlapping k
+    assert ks(P[0], P[1], ctypes.c_void_p(0x1000000 + 256), 1, 1, 16, 64, 64, la2.LA2_F32, NULL, 0,
+              NULL) == la2.LA2_ERR_INVALID_ARG
