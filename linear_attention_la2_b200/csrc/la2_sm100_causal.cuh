@@ -86,14 +86,15 @@ struct Step {
 template <int KIND>
 struct StepIter {
   const RangeTable* rt;
+  // Task indices fit in 32 bits (the host rejects larger task lists).
   int32_t r;
-  int64_t f, fend;      // KIND_MAIN: next task / end of the current range
-  int64_t seg_end;      // end of the open segment (0 when none is open)
-  int64_t seg_lo;
-  int64_t bh;           // sequence of task f
-  int64_t blk;          // block of task f inside its sequence
+  int32_t f, fend;      // KIND_MAIN: next task / end of the current range
+  int32_t seg_end;      // end of the open segment (0 when none is open)
+  int32_t seg_lo;
+  int32_t bh;           // sequence of task f
+  int32_t blk;          // block of task f inside its sequence
   uint8_t seg_init;
-  int64_t pre_bh;
+  int32_t pre_bh;
   int32_t pre_blk, pre_end, pre_lo;
 
   __device__ __forceinline__ void begin(const RangeTable* t) {
@@ -111,7 +112,7 @@ struct StepIter {
   // Next step of this CTA; false when its ranges are exhausted. No recursion
   // and one division per range, so every role can call it each step.
   __device__ __forceinline__ bool next(Step& s) {
-    const int64_t T = rt->T;
+    const int32_t T = static_cast<int32_t>(rt->T);
     if (pre_blk >= pre_end) {
       if (KIND == KIND_AGG) {
         // One state pass per range whose end falls inside a sequence.
@@ -119,14 +120,14 @@ struct StepIter {
         while (!found) {
           r += static_cast<int32_t>(gridDim.x);
           if (r >= rt->R - 1) return false;  // the last range's state is never needed
-          const int64_t e = rt->starts[r + 1];
-          const int64_t hb = (e - 1) / T;
+          const int32_t e = static_cast<int32_t>(rt->starts[r + 1]);
+          const int32_t hb = (e - 1) / T;
           if (e - hb * T == T) continue;  // ends on a sequence boundary
-          const int64_t lo = max(rt->starts[r], hb * T);
+          const int32_t lo = max(static_cast<int32_t>(rt->starts[r]), hb * T);
           pre_bh = hb;
-          pre_lo = static_cast<int32_t>(lo - hb * T);
+          pre_lo = lo - hb * T;
           pre_blk = pre_lo;
-          pre_end = static_cast<int32_t>(e - hb * T);
+          pre_end = e - hb * T;
           found = true;
         }
       } else {
@@ -134,8 +135,8 @@ struct StepIter {
           do {
             r += static_cast<int32_t>(gridDim.x);
             if (r >= rt->R) return false;
-            f = rt->starts[r];
-            fend = rt->starts[r + 1];
+            f = static_cast<int32_t>(rt->starts[r]);
+            fend = static_cast<int32_t>(rt->starts[r + 1]);
           } while (f >= fend);
           seg_end = 0;
           bh = f / T;
@@ -947,6 +948,7 @@ inline RangePlan plan_ranges(int64_t BH, int64_t N, int block, int sms, int64_t 
 
 inline bool fill_range_table(const RangePlan& p, sm100::RangeTable* t) {
   if (p.R < 1 || p.R > sm100::kMaxRanges) return false;
+  if (p.starts.back() > 0x7fffffff) return false;  // task indices are 32-bit on the device
   t->R = p.R;
   t->prefix_mode = p.prefix_mode;
   t->T = p.T;
