@@ -51,6 +51,9 @@ def parse():
                     help="also print the decode-step line (one RNN-mode token per sequence)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-every", type=int, default=4,
+                    help="bracket the launches of every n-th timed step with per-kernel CUDA "
+                         "events (1 = every step); the step time is measured over all steps")
     ap.add_argument("--no-clocks", action="store_true",
                     help="skip nvidia-smi clock sampling (and its extra steps), e.g. under a profiler")
     return ap.parse_args()
@@ -372,7 +375,7 @@ def bench_workload(args, w, dev, la2, world, rank, local, hbm, peak_kind, main):
     la2.check(stream)
 
     sampler = ClockSampler(local) if main and not args.no_clocks else None
-    la2.la2_profile_enable(1)
+    every = max(1, args.profile_every)
     _barrier(world)
     torch.cuda.synchronize(dev)
     if sampler:
@@ -381,9 +384,20 @@ def bench_workload(args, w, dev, la2, world, rank, local, hbm, peak_kind, main):
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     th0 = time.monotonic()
+    la2.la2_profile_enable(1)  # clear the records ...
+    la2.la2_profile_enable(0)  # ... and record only the sampled steps
     e0.record(stream)
+    profiled_steps = 0
     for i in range(args.steps):
+        # per-kernel events around the launches of every `every`-th step only:
+        # an event pair per launch also costs device time between kernels
+        prof = i % every == 0
+        if prof:
+            la2.la2_profile_enable(2)
+            profiled_steps += 1
         step(i)
+        if prof:
+            la2.la2_profile_enable(0)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     th1 = time.monotonic()
@@ -421,6 +435,8 @@ def bench_workload(args, w, dev, la2, world, rank, local, hbm, peak_kind, main):
         if n:
             per_kernel[la2.la2_profile_kernel_name(kid)] = {"launches": n, "ms": kms}
             launches += n
+    # every step launches the same kernels: scale the timed sample to all steps
+    launches = launches * args.steps // max(1, profiled_steps)
     dom = max(per_kernel, key=lambda k: per_kernel[k]["ms"]) if per_kernel else None
 
     value = whole_job_rate(w.tokens, args.steps, world, ms_max)
@@ -446,6 +462,8 @@ def bench_workload(args, w, dev, la2, world, rank, local, hbm, peak_kind, main):
             "(b,h) sequences per rank)"),
         "tflops": tflops, "step_roofline_frac": step_frac, "roofline": roofline,
         "gpu_launches": launches, "kernels": per_kernel,
+        "kernel_timing": (f"CUDA events around each launch of {profiled_steps} of the "
+                          f"{args.steps} timed steps (every {every}th step)"),
     }
     if clocks:
         line["clocks"] = clocks
@@ -490,14 +508,23 @@ def bench_decode(args, dev, la2, world, hbm, peak_kind):
     for i in range(args.warmup):
         step(i)
     la2.check(stream)
-    la2.la2_profile_enable(1)
+    every = max(1, args.profile_every)
     _barrier(world)
     torch.cuda.synchronize(dev)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
+    la2.la2_profile_enable(1)
+    la2.la2_profile_enable(0)
     e0.record(stream)
+    profiled_steps = 0
     for i in range(args.steps):
+        prof = i % every == 0
+        if prof:
+            la2.la2_profile_enable(2)
+            profiled_steps += 1
         step(i)
+        if prof:
+            la2.la2_profile_enable(0)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     la2.la2_profile_enable(0)
@@ -524,7 +551,10 @@ def bench_decode(args, dev, la2, world, hbm, peak_kind):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm, "traffic": None, "kernel": "la2_decode_step",
                      "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)"},
-        "gpu_launches": sum(v["launches"] for v in per_kernel.values()), "kernels": per_kernel,
+        "gpu_launches": sum(v["launches"] for v in per_kernel.values()) * args.steps
+        // max(1, profiled_steps), "kernels": per_kernel,
+        "kernel_timing": (f"CUDA events around each launch of {profiled_steps} of the "
+                          f"{args.steps} timed steps (every {every}th step)"),
     }
 
 

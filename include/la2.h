@@ -183,10 +183,13 @@ LA2_API la2_status la2_set_spin_limit(int64_t iterations);
 /*
  * Per-kernel launch timing, for benchmarks. While enabled, every kernel the
  * library launches is bracketed by a pair of CUDA events on its stream.
- * la2_profile_collect() synchronises those events and returns, for kernel id
- * `kernel`, the number of launches and their summed device time in ms since
- * the last la2_profile_enable(1). Ids run from 0 to la2_profile_num_kernels()-1
- * and la2_profile_kernel_name() names them. Not thread-safe.
+ * la2_profile_enable(1) clears the records and starts recording, (0) pauses,
+ * (2) resumes without clearing (so a benchmark can time a sample of its
+ * steps); other values give LA2_ERR_INVALID_ARG. la2_profile_collect()
+ * synchronises the events and returns, for kernel id `kernel`, the number of
+ * recorded launches and their summed device time in ms since the last
+ * la2_profile_enable(1). Ids run from 0 to la2_profile_num_kernels()-1 and
+ * la2_profile_kernel_name() names them. Not thread-safe.
  */
 LA2_API la2_status la2_profile_enable(int on);
 LA2_API int la2_profile_num_kernels(void);

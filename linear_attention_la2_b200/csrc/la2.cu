@@ -753,8 +753,9 @@ const char* la2_status_string(la2_status s) {
 }
 
 la2_status la2_profile_enable(int on) {
+  if (on < 0 || on > 2) return LA2_ERR_INVALID_ARG;
   g_prof.on = on != 0;
-  if (g_prof.on) g_prof.used = 0;
+  if (on == 1) g_prof.used = 0;
   return LA2_OK;
 }
 

@@ -82,7 +82,7 @@ decode_step_v4_kernel(const T* __restrict__ q, const T* __restrict__ k, const T*
   if (j < dv) {
     const float4 vj = load4<T>(v + bh * dv + j);
     float* col = state + bh * static_cast<int64_t>(d) * dv + j;
-#pragma unroll 8
+#pragma unroll 16  // every row of a thread in flight at d = 128
     for (int i = w; i < d; i += kDecodeWarps) {
       float4* p = reinterpret_cast<float4*>(col + static_cast<int64_t>(i) * dv);
       const float ki = to_f32(kb[i]), qi = to_f32(qb[i]);

@@ -119,6 +119,9 @@ def test_profiler_names():
     assert all(names) and len(set(names)) == n
     assert la2.la2_profile_kernel_name(n) == ""
     assert la2.la2_version() > 0
+    assert la2.la2_profile_enable(3) == la2.LA2_ERR_INVALID_ARG
+    for on in (1, 0, 2, 0):
+        assert la2.la2_profile_enable(on) == la2.LA2_OK
 
 
 def _dec(**kw):
