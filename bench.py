@@ -176,7 +176,9 @@ def workload_from_args(args):
     return w
 
 
-def flops_per_token(w):
+def flops_per_token(w, causal=True):
+    if not causal:  # O = Q (K^T V): the state pass and the map pass
+        return 4 * w.d * w.dv
     return 2 * w.block * (w.d + w.dv) + 4 * w.d * w.dv
 
 
@@ -249,10 +251,11 @@ def run_reference(args):
     return 0
 
 
-def config_of(w):
-    return {"workload": f"{w.name}: causal forward B={w.B} H={w.H} N={w.N} d={w.d} dv={w.dv} "
+def config_of(w, causal=True):
+    kind = "causal" if causal else "non-causal"
+    return {"workload": f"{w.name}: {kind} forward B={w.B} H={w.H} N={w.N} d={w.d} dv={w.dv} "
                         f"block={w.block} {w.dtype}", "B": w.B, "H": w.H, "N": w.N, "d": w.d,
-            "dv": w.dv, "block": w.block, "causal": True}
+            "dv": w.dv, "block": w.block, "causal": causal}
 
 
 # ------------------------------------------------------------------- GPU
@@ -293,6 +296,11 @@ def run_gpu(args):
         ln = bench_workload(args, lw, dev, la2, world, rank, local, hbm, peak_kind, main=False)
         if rank == 0:
             print(json.dumps(ln), flush=True)
+    if args.sweep:
+        ln = bench_workload(args, w, dev, la2, world, rank, local, hbm, peak_kind, main=False,
+                            causal=False)
+        if rank == 0:
+            print(json.dumps(ln), flush=True)
     if args.sweep or args.decode:
         ln = bench_decode(args, dev, la2, world, hbm, peak_kind)
         if rank == 0:
@@ -326,7 +334,7 @@ def _barrier(world):
         dist.barrier()
 
 
-def bench_workload(args, w, dev, la2, world, rank, local, hbm, peak_kind, main):
+def bench_workload(args, w, dev, la2, world, rank, local, hbm, peak_kind, main, causal=True):
     import torch
 
     from linear_attention_la2_b200 import inputs as I
@@ -347,7 +355,7 @@ def bench_workload(args, w, dev, la2, world, rank, local, hbm, peak_kind, main):
         o = torch.empty((w.B, w.H, w.N, w.dv), dtype=w.torch_dtype, device=dev)
         sets.append((q, k, v, o))
     dt = la2.LA2_BF16 if w.dtype == "bf16" else la2.LA2_F32
-    ws_bytes = la2.workspace_bytes(w.B, w.H, w.N, w.d, w.dv, True, w.block, dt, False)
+    ws_bytes = la2.workspace_bytes(w.B, w.H, w.N, w.d, w.dv, causal, w.block, dt, False)
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
     st = la2._stream_handle(stream)
 
@@ -360,7 +368,7 @@ def bench_workload(args, w, dev, la2, world, rank, local, hbm, peak_kind, main):
     def step(i):
         q, k, v, o = sets[i % nsets]
         rc = la2.la2_forward(la2._ptr(q), la2._ptr(k), la2._ptr(v), la2._ptr(o), w.B, w.H, w.N, w.d,
-                             w.dv, 1, w.block, dt, la2._ptr(ws), ws_bytes, st)
+                             w.dv, int(causal), w.block, dt, la2._ptr(ws), ws_bytes, st)
         if rc != 0:
             raise la2.La2Error(rc)
         if w.backward:
@@ -440,7 +448,7 @@ def bench_workload(args, w, dev, la2, world, rank, local, hbm, peak_kind, main):
     dom = max(per_kernel, key=lambda k: per_kernel[k]["ms"]) if per_kernel else None
 
     value = whole_job_rate(w.tokens, args.steps, world, ms_max)
-    tflops = flops_per_token(w) * value / 1e12
+    tflops = flops_per_token(w, causal) * value / 1e12
     roofline = None
     if dom:
         avg_ms = per_kernel[dom]["ms"] / per_kernel[dom]["launches"]
@@ -453,10 +461,11 @@ def bench_workload(args, w, dev, la2, world, rank, local, hbm, peak_kind, main):
     step_frac = (w.tokens * bytes_per_token(w) * args.steps * world / (ms_max / 1e3) / 1e9) / (hbm * world)
 
     line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "metric": METRIC if causal else METRIC.replace("causal", "non-causal", 1), "value": value,
+        "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
-        "data": "synthetic", "config": dict(config_of(w), l2=(
+        "data": "synthetic", "config": dict(config_of(w, causal), l2=(
             f"{nsets} rotating input sets of {set_bytes / 1e6:.0f} MB (> L2 126 MB)" if nsets > 1
             else f"inputs {set_bytes / 1e6:.0f} MB > L2"), parallelism=f"dp{world} (independent "
             "(b,h) sequences per rank)"),
