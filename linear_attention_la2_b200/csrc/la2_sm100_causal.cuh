@@ -420,6 +420,10 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int64_t lim = prm.spin_limit;
+  // Everything above touches only this CTA's shared memory, TMEM and kernel
+  // parameters; from here on global memory is read and written.
+  pdl_launch_dependents();
+  pdl_wait();
 
   // Range-state mode: a CTA's range (at most one per CTA) that starts inside
   // a sequence gets its initial state from the consumer warpgroups before
@@ -965,7 +969,20 @@ inline la2_status launch_causal_sm100(const CUtensorMap& tq, const CUtensorMap& 
   auto kern = sm100::la2_causal_sm100_kernel<BK, D, DV, KIND>;
   static bool attr_done[128];  // one per template instantiation
   if (!smem_attribute_set(kern, CF::SMEM, attr_done)) return LA2_ERR_CUDA;
-  kern<<<static_cast<unsigned>(grid), sm100::kThreads, CF::SMEM, st>>>(tq, tk, tv, to, rt, p);
+  // Programmatic stream serialization: this grid may begin launching while
+  // the previous kernel of the stream finishes; the kernel waits for it
+  // (griddepcontrol.wait) before it touches global memory.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(sm100::kThreads);
+  cfg.dynamicSmemBytes = CF::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, to, rt, p) != cudaSuccess) return LA2_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? LA2_OK : LA2_ERR_CUDA;
 }
 
