@@ -241,7 +241,8 @@ static la2_status run_chunk_states(const void* a, const void* b, float* out, int
 static la2_status run_scan(float* s, int64_t BH, int nel, const Plan& p, int mode, cudaStream_t st) {
   dim3 grid((nel + kSimtThreads - 1) / kSimtThreads, (unsigned)BH);
   LaunchTimer t(K_CHUNK_SCAN, st);
-  chunk_scan_kernel<<<grid, kSimtThreads, 0, st>>>(s, p.C, nel, mode);
+  if (launch_pdl(chunk_scan_kernel, grid, dim3(kSimtThreads), 0, st, s, p.C, nel, mode) != cudaSuccess)
+    return LA2_ERR_CUDA;
   return launch_status();
 }
 
@@ -563,8 +564,10 @@ la2_status la2_kv_state(const void* k, const void* v, float* state, int64_t B, i
   if (s != LA2_OK) return s;
   const int nel = (int)(d * dv);
   LaunchTimer t(K_STATE_ACC, st);
-  state_accumulate_kernel<<<dim3((unsigned)((nel + 255) / 256), (unsigned)BH), 256, 0, st>>>(
-      chunks, state, p.C, (int)d, (int)dv, p.tc ? 1 : 0);
+  if (launch_pdl(state_accumulate_kernel, dim3((unsigned)((nel + 255) / 256), (unsigned)BH),
+                 dim3(256), 0, st, static_cast<const float*>(chunks), state, p.C, (int)d, (int)dv,
+                 p.tc ? 1 : 0) != cudaSuccess)
+    return LA2_ERR_CUDA;
   return launch_status();
 }
 
@@ -592,28 +595,32 @@ la2_status la2_decode_step(const void* q, const void* k, const void* v, void* o,
   LaunchTimer t(K_DECODE, st);
   // Four columns per lane when rows of the state, v and o allow 16-, 8- or
   // 16-byte vector accesses.
+  const dim3 block(32 * kDecodeWarps);
+  cudaError_t e;
   if (dv % 4 == 0 && is_aligned(state, 16) && is_aligned(v, 4 * es) && is_aligned(o, es)) {
     const dim3 grid4((unsigned)BH, (unsigned)((dv + 127) / 128));
     if (dt == LA2_BF16)
-      decode_step_v4_kernel<__nv_bfloat16><<<grid4, 32 * kDecodeWarps, 0, st>>>(
-          static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-          static_cast<const __nv_bfloat16*>(v), static_cast<__nv_bfloat16*>(o), state, (int)d,
-          (int)dv);
+      e = launch_pdl(decode_step_v4_kernel<__nv_bfloat16>, grid4, block, 0, st,
+                     static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+                     static_cast<const __nv_bfloat16*>(v), static_cast<__nv_bfloat16*>(o), state,
+                     (int)d, (int)dv);
     else
-      decode_step_v4_kernel<float><<<grid4, 32 * kDecodeWarps, 0, st>>>(
-          static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
-          static_cast<float*>(o), state, (int)d, (int)dv);
-    return launch_status();
+      e = launch_pdl(decode_step_v4_kernel<float>, grid4, block, 0, st,
+                     static_cast<const float*>(q), static_cast<const float*>(k),
+                     static_cast<const float*>(v), static_cast<float*>(o), state, (int)d, (int)dv);
+  } else {
+    const dim3 grid((unsigned)BH, (unsigned)((dv + 31) / 32));
+    if (dt == LA2_BF16)
+      e = launch_pdl(decode_step_kernel<__nv_bfloat16>, grid, block, 0, st,
+                     static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+                     static_cast<const __nv_bfloat16*>(v), static_cast<__nv_bfloat16*>(o), state,
+                     (int)d, (int)dv);
+    else
+      e = launch_pdl(decode_step_kernel<float>, grid, block, 0, st, static_cast<const float*>(q),
+                     static_cast<const float*>(k), static_cast<const float*>(v),
+                     static_cast<float*>(o), state, (int)d, (int)dv);
   }
-  const dim3 grid((unsigned)BH, (unsigned)((dv + 31) / 32));
-  if (dt == LA2_BF16)
-    decode_step_kernel<__nv_bfloat16><<<grid, 32 * kDecodeWarps, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-        static_cast<const __nv_bfloat16*>(v), static_cast<__nv_bfloat16*>(o), state, (int)d, (int)dv);
-  else
-    decode_step_kernel<float><<<grid, 32 * kDecodeWarps, 0, st>>>(
-        static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
-        static_cast<float*>(o), state, (int)d, (int)dv);
+  if (e != cudaSuccess) return LA2_ERR_CUDA;
   return launch_status();
 }
 

@@ -24,6 +24,8 @@ template <typename T>
 __global__ void __launch_bounds__(32 * kDecodeWarps)
 decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                    T* __restrict__ o, float* __restrict__ state, int d, int dv) {
+  pdl_launch_dependents();
+  pdl_wait();
   __shared__ float part[kDecodeWarps][32];
   const int64_t bh = blockIdx.x;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
@@ -72,6 +74,8 @@ template <typename T>
 __global__ void __launch_bounds__(32 * kDecodeWarps)
 decode_step_v4_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                       T* __restrict__ o, float* __restrict__ state, int d, int dv) {
+  pdl_launch_dependents();
+  pdl_wait();
   __shared__ float4 part[kDecodeWarps][32];
   const int64_t bh = blockIdx.x;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
@@ -124,6 +128,8 @@ decode_step_v4_kernel(const T* __restrict__ q, const T* __restrict__ k, const T*
 __global__ void __launch_bounds__(256)
 state_accumulate_kernel(const float* __restrict__ chunks, float* __restrict__ state, int64_t C,
                         int d, int dv, int chunk_major) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int nel = d * dv;
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
   if (e >= nel) return;

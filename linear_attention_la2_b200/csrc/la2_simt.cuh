@@ -84,6 +84,8 @@ chunk_state_kernel(const T* __restrict__ a, const T* __restrict__ b, float* __re
 // ----------------------------------------------------------------------------
 __global__ void __launch_bounds__(kSimtThreads)
 chunk_scan_kernel(float* __restrict__ s, int64_t C, int nel, int mode) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
   if (e >= nel) return;
   float* p = s + (int64_t)blockIdx.y * C * nel + e;

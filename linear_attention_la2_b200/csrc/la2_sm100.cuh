@@ -70,14 +70,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Programmatic dependent launch: let the next kernel of the stream start its
-// launch now (its CTAs still wait in pdl_wait for this grid), and wait until
-// the previous kernel of the stream has completed and its memory is visible.
-// Both are no-ops for kernels launched without the attribute.
-__device__ __forceinline__ void pdl_launch_dependents() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 
 __device__ __forceinline__ void fence_barrier_init() {
@@ -488,6 +480,8 @@ la2_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   tc_fence_after();
   const uint32_t tmem = *b.tmem_base;
   const int64_t lim = prm.spin_limit;
+  pdl_launch_dependents();  // global memory is touched only after this point
+  pdl_wait();
 
   uint8_t* sQ = smem + CF::OFF_Q;
   uint8_t* sK = smem + CF::OFF_K;
@@ -907,7 +901,9 @@ inline la2_status launch_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk,
   auto kern = sm100::la2_fwd_sm100_kernel<BK, D, DV, MODE, DQ>;
   static bool attr_done[128];  // one per template instantiation
   if (!smem_attribute_set(kern, CF::SMEM, attr_done)) return LA2_ERR_CUDA;
-  kern<<<static_cast<unsigned>(units), sm100::kThreads, CF::SMEM, st>>>(tq, tk, tv, to, p);
+  if (launch_pdl(kern, dim3(static_cast<unsigned>(units)), dim3(sm100::kThreads), CF::SMEM, st, tq,
+                 tk, tv, to, p) != cudaSuccess)
+    return LA2_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? LA2_OK : LA2_ERR_CUDA;
 }
 

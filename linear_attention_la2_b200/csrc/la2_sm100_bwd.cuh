@@ -138,6 +138,8 @@ la2_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int64_t lim = prm.spin_limit;
+  pdl_launch_dependents();  // global memory is touched only after this point
+  pdl_wait();
   uint8_t* sStage = smem + CF::OFF_ST;
   uint8_t* sPT = smem + CF::OFF_PT;
   uint8_t* sPdT = smem + CF::OFF_PDT;
@@ -465,8 +467,9 @@ inline la2_status launch_bwd_dkdv_sm100(const CUtensorMap& tq, const CUtensorMap
   auto kern = sm100::la2_bwd_dkdv_sm100_kernel<BK, 128, 128>;
   static bool attr_done[128];
   if (!smem_attribute_set(kern, CF::SMEM, attr_done)) return LA2_ERR_CUDA;
-  kern<<<static_cast<unsigned>(units), sm100::kThreads, CF::SMEM, st>>>(tq, tk, tv, tdo, tdk, tdv,
-                                                                         p);
+  if (launch_pdl(kern, dim3(static_cast<unsigned>(units)), dim3(sm100::kThreads), CF::SMEM, st, tq,
+                 tk, tv, tdo, tdk, tdv, p) != cudaSuccess)
+    return LA2_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? LA2_OK : LA2_ERR_CUDA;
 }
 
