@@ -155,8 +155,12 @@ static Plan make_plan_uncached(int64_t B, int64_t H, int64_t N, int64_t d, int64
   } else {
     // Enough (b, h, chunk) units for about two per SM, chunks no shorter than
     // four blocks so the chunk-state pass stays a small fraction of the work.
-    const int64_t target = 2 * (int64_t)std::max(sms, 1);
-    int64_t C = std::max<int64_t>(1, (target + BH - 1) / std::max<int64_t>(BH, 1));
+    // Tensor-core non-causal forward: about one wave, since the map pass sums
+    // a sequence's chunk states itself.
+    const bool one_wave = p.tc && !causal && !is_bwd;
+    const int64_t target = (one_wave ? 1 : 2) * (int64_t)std::max(sms, 1);
+    int64_t C = one_wave ? std::max<int64_t>(1, target / std::max<int64_t>(BH, 1))
+                         : std::max<int64_t>(1, (target + BH - 1) / std::max<int64_t>(BH, 1));
     C = std::min<int64_t>(C, std::max<int64_t>(1, T / 4));
     L = ((T + C - 1) / C) * block;
   }
@@ -328,6 +332,10 @@ static la2_status causal_range_split(const void* q, const void* k, const void* v
   return launch_causal_sm100<BK, D, DV, sm100::KIND_MAIN>(tq, tk, tv, to, rt, cp, grid, st);
 }
 
+// Non-causal: up to this many chunk states per sequence are added up inside
+// the map pass (no scan launch); more are scanned into slot 0 first.
+constexpr int64_t kSumInKernel = 8;
+
 // Tensor-core forward. Causal: the range split above. Non-causal: chunk
 // states, their total, then every block against the total state.
 template <int BK>
@@ -357,8 +365,12 @@ static la2_status forward_sm100_bk(const void* q, const void* k, const void* v, 
     s = launch_fwd_sm100<BK, D, DV, sm100::MODE_STATE>(tq, tk, tv, tq, ps, BH * p.C, st);
   }
   if (s != LA2_OK) return s;
-  s = run_scan(states, BH, nel, p, 2, st);
-  if (s != LA2_OK) return s;
+  // A few chunk states: the map pass adds them up itself; many: scan first.
+  prm.init_count = p.C <= kSumInKernel ? p.C : 1;
+  if (p.C > kSumInKernel) {
+    s = run_scan(states, BH, nel, p, 2, st);
+    if (s != LA2_OK) return s;
+  }
   prm.init_states = states;
   prm.units_per_seq = p.C;
   CUtensorMap to_nc = tq;
@@ -408,7 +420,7 @@ static la2_status backward_sm100_bk(const void* q, const void* k, const void* v,
       s = launch_fwd_sm100<BK, D, DV, sm100::MODE_STATE>(tq, tq, tdo, tq, ps, BH * p.C, st);
     }
     if (s != LA2_OK) return s;
-    if (!dq_split) {
+    if (!dq_split && (causal || p.C > kSumInKernel)) {
       s = run_scan(s_kv, BH, nel, p, causal ? 0 : 2, st);
       if (s != LA2_OK) return s;
     }
@@ -425,6 +437,7 @@ static la2_status backward_sm100_bk(const void* q, const void* k, const void* v,
     pq.L = p.L;
     pq.C = p.C;
     pq.units_per_seq = p.C;
+    pq.init_count = p.C <= kSumInKernel ? p.C : 1;  // non-causal dQ: summed here or scanned
     pq.spin_limit = spin;
     CUtensorMap tdq = tq;
     if (sm100::Cfg<BK, D, DV>::TMA_STORE && !make_tmap_3d(&tdq, dq, BH, N, D, 16)) return LA2_ERR_CUDA;

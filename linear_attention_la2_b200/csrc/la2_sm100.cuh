@@ -307,7 +307,9 @@ struct Cfg {
 
 struct Params {
   __nv_bfloat16* o;           // [BH][N][DV] (forward modes)
-  const float* init_states;   // [BH][C][D][DV]: prefix (causal) or total in slot 0 (non-causal)
+  const float* init_states;   // [BH][C][D*DV] (state_f4): scanned prefix (causal); non-causal:
+                              // slots 0..init_count-1 of the sequence, summed by the kernel
+  int64_t init_count;         // non-causal: chunk states to add up (1 after a total scan)
   float* out_states;          // MODE_STATE output [BH][C][D][DV]
   int64_t N;
   int64_t L;                  // chunk length (multiple of BK)
@@ -708,11 +710,19 @@ la2_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           float vals[32];
           uint32_t u[32];
           if (r >= 0) {
-            const float4* src = reinterpret_cast<const float4*>(init);
+            // Non-causal: the total is the sum of the sequence's first
+            // init_count chunk states, added here in chunk order (a few chunk
+            // states: no separate scan launch; many: scanned into slot 0).
+            const int64_t nsum = MODE == MODE_NONCAUSAL ? prm.init_count : 1;
 #pragma unroll
-            for (int q4 = 0; q4 < 8; ++q4) {
-              const float4 x = src[state_f4<D>(r, c32 * 8 + q4)];
-              vals[4 * q4] = x.x; vals[4 * q4 + 1] = x.y; vals[4 * q4 + 2] = x.z; vals[4 * q4 + 3] = x.w;
+            for (int j = 0; j < 32; ++j) vals[j] = 0.f;
+            for (int64_t cc = 0; cc < nsum; ++cc) {
+              const float4* src = reinterpret_cast<const float4*>(init + cc * (int64_t)(D * DV));
+#pragma unroll
+              for (int q4 = 0; q4 < 8; ++q4) {
+                const float4 x = src[state_f4<D>(r, c32 * 8 + q4)];
+                vals[4 * q4] += x.x; vals[4 * q4 + 1] += x.y; vals[4 * q4 + 2] += x.z; vals[4 * q4 + 3] += x.w;
+              }
             }
           } else {
 #pragma unroll
