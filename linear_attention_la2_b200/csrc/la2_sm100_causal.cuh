@@ -877,7 +877,7 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
 // block moves half the bytes and its loads stay latency-bound).
 constexpr double kPrepassCost = 0.5;
 constexpr double kRangeStateCost = 0.5;  // separate state launch, per block
-constexpr double kLaunchCost = 8.0;      // extra launch + initial-state sum, in main blocks
+constexpr double kLaunchCost = 8.0;      // extra launch + initial-state sum, in Bk=64 main blocks
 
 struct RangePlan {
   int R = 0;
@@ -934,7 +934,9 @@ inline RangePlan plan_ranges(int64_t BH, int64_t N, int block, int sms, int64_t 
   const double tau_pre = hi;
   // (b) range-state plan: equal split; a separate launch computes range states
   const int n_eq = static_cast<int>(std::min<int64_t>(G, total));
-  const double tau_eq = static_cast<double>(total) / n_eq * (1.0 + kRangeStateCost) + kLaunchCost;
+  // the launch cost is a time: in units of this block size's main block
+  const double launch = kLaunchCost * 64.0 / static_cast<double>(block);
+  const double tau_eq = static_cast<double>(total) / n_eq * (1.0 + kRangeStateCost) + launch;
   if (tau_pre <= tau_eq && n_pre <= sm100::kMaxRanges) {
     p.prefix_mode = 0;
     p.starts = pre_starts;
