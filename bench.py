@@ -30,6 +30,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 L2_BYTES = 126 * 1024 * 1024
+CLOCK_RAMP_S = 0.2
 METRIC = "causal linear-attn fwd tokens/s (B·H·N/s), TFLOP/s, % of roofline, 1 B200"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
@@ -384,11 +385,18 @@ def bench_workload(args, w, dev, la2, world, rank, local, hbm, peak_kind, main, 
 
     sampler = ClockSampler(local) if main and not args.no_clocks else None
     every = max(1, args.profile_every)
-    _barrier(world)
-    torch.cuda.synchronize(dev)
     if sampler:
         sampler.start()
-        time.sleep(0.3)
+    # Clock ramp: after the requested warm-up, keep the same workload running
+    # (untimed) for CLOCK_RAMP_S so the timed region does not start at the
+    # clocks of an idle GPU (input preparation leaves it idle for seconds).
+    ramp_steps = 0
+    tr0 = time.monotonic()
+    while time.monotonic() - tr0 < CLOCK_RAMP_S:
+        step(args.warmup + ramp_steps)
+        ramp_steps += 1
+    _barrier(world)
+    torch.cuda.synchronize(dev)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     th0 = time.monotonic()
@@ -473,6 +481,8 @@ def bench_workload(args, w, dev, la2, world, rank, local, hbm, peak_kind, main, 
         "gpu_launches": launches, "kernels": per_kernel,
         "kernel_timing": (f"CUDA events around each launch of {profiled_steps} of the "
                           f"{args.steps} timed steps (every {every}th step)"),
+        "clock_ramp": f"{ramp_steps} untimed steps ({CLOCK_RAMP_S} s) after the {args.warmup} "
+                      "warm-up steps",
     }
     if clocks:
         line["clocks"] = clocks
