@@ -19,8 +19,10 @@
 // The state never leaves the SM: it is accumulated in TMEM, and a bf16 copy
 // (the "snapshot") is written to SMEM each block as the B operand of Q_i*KV.
 //
-// Warp roles (16 warps): 0 TMA producer, 1 MMA issuer (+ TMEM allocation),
-// 4-7 mask/convert S -> P, 8-11 KV snapshot, 12-15 epilogue O -> HBM.
+// Warp roles (16 warps): 0 TMA producer, 1 MMA issuer (the whole warp runs the
+// loop, one elected lane issues; + TMEM allocation), 4-7 mask/convert S -> P,
+// 8-11 KV snapshot, 12-15 epilogue O -> HBM (Bk=64: swizzled staging tile and
+// TMA stores).
 //
 // Every wait is bounded (iteration count and a wall-clock deadline); on
 // expiry the waiting role records LA2_ERR_TIMEOUT in the device error word,

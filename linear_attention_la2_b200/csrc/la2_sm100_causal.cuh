@@ -15,8 +15,10 @@
 // sequence; its initial state is either
 //   * rebuilt by a pre-pass over the sequence's earlier blocks (K and V only,
 //     KV += K^T V, no output) - one launch, no workspace; or
-//   * the sum of the per-range states that la2_range_state (the same kernel,
-//     KIND_AGG) wrote for the earlier ranges of that sequence.
+//   * the sum of the per-range states that a state-only launch of the same
+//     kernel (KIND_AGG) wrote for the earlier ranges of that sequence; the
+//     three consumer warpgroups add them up at CTA start.
+// The host picks the cheaper of the two from a cost model (plan_ranges).
 //
 // Per main block (one CTA, warp-specialised):
 //   S   = Q K^T           tcgen05 M=Bk N=Bk K=d          TMEM
@@ -24,9 +26,11 @@
 //   KV += K^T V           tcgen05 M=d N=dv K=Bk          TMEM (fp32 state)
 //   O   = Q bf16(KV_old)  tcgen05 M=Bk N=dv K=d          TMEM (snapshot taken before the update)
 //   O  += P V             tcgen05 M=Bk N=dv K=Bk
-// The KV update is issued as soon as the snapshot of the old state is in SMEM,
-// so the next block's snapshot can start while this block's products run, and
-// S of the next block is issued before P V of this one.
+// One warp issues the MMAs (one elected lane per instruction) in the order
+// S; Q bf16(KV_old) once the snapshot of the old state is in SMEM; the KV
+// update; P V once the mask warpgroup has written P. The state warpgroup turns
+// the updated state into the next snapshot while P V and the next block's S
+// run. At Bk=64 O leaves through a swizzled staging tile and TMA stores.
 #pragma once
 
 #include "la2_sm100.cuh"
@@ -48,9 +52,6 @@ __device__ unsigned long long g_trace[kTraceEvents][kTraceSteps];
   do {                           \
   } while (0)
 #endif
-
-// Issue S of the next block before P V of this one (needs a Q ring deeper than 1).
-constexpr bool kPrefetchS = false;
 
 constexpr int kMaxRanges = 160;  // the range table travels as a kernel parameter (< 4 KB)
 
