@@ -32,7 +32,8 @@ is the RNN form and ``blocked_forward`` the block algorithm of point 2; those tw
 exist to pin the definition (and to check very long sequences where the O(N^2)
 definition is too slow on a CPU), never the other way round. ``kv_state`` (the
 state after a prefill) and ``decode_step`` (one RNN-mode step) are the oracle of
-the inference form.
+the inference form; ``forward_gqa`` / ``backward_gqa`` the oracle of grouped K/V
+heads (a layout of the same op: each query head reads the K/V head of its group).
 
 Parity status: every function here is pinned by ``tests/test_oracle.py``
 (brute force on tiny integer inputs, closed forms, RNN-form equality, block-size
@@ -202,6 +203,54 @@ def recurrent_forward(q, k, v) -> np.ndarray:
                 kv += np.outer(k[b, h, t], v[b, h, t])
                 out[b, h, t] = q[b, h, t] @ kv
     return out
+
+
+def _group(H: int, Hkv: int) -> int:
+    if Hkv < 1 or H % Hkv:
+        raise ValueError("H must be a multiple of the number of K/V heads")
+    return H // Hkv
+
+
+def forward_gqa(q, k, v, causal: bool = True) -> np.ndarray:
+    """Grouped K/V heads (GQA; MQA when there is one K/V head): ``q [B,H,N,d]``,
+    ``k [B,Hkv,N,d]``, ``v [B,Hkv,N,dv]``; query head h attends through K/V head
+    ``h // (H // Hkv)`` with the left product of point 1, one (b, h) at a time.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    if q.ndim != 4 or k.shape[:3] != (q.shape[0], k.shape[1], q.shape[2]) or v.shape[:3] != k.shape[:3]:
+        raise ValueError("q [B,H,N,d], k [B,Hkv,N,d], v [B,Hkv,N,dv] expected")
+    B, H, N, _ = q.shape
+    g = _group(H, k.shape[1])
+    out = np.empty((B, H, N, v.shape[3]))
+    keep = np.tri(N, dtype=bool) if causal else np.ones((N, N), dtype=bool)
+    for b in range(B):
+        for h in range(H):
+            S = q[b, h] @ k[b, h // g].T
+            out[b, h] = np.where(keep, S, 0.0) @ v[b, h // g]
+    return out
+
+
+def backward_gqa(q, k, v, do, causal: bool = True):
+    """Gradients of ``L = <dO, O>`` for ``forward_gqa``: per query head the closed
+    forms of ``backward``; a K/V head's dK and dV add up over the query heads of
+    its group (each of them reads that K/V head).
+    """
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    B, H, N, _ = q.shape
+    g = _group(H, k.shape[1])
+    keep = np.tri(N, dtype=bool) if causal else np.ones((N, N), dtype=bool)
+    dq = np.empty_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for b in range(B):
+        for h in range(H):
+            kv = h // g
+            dP = np.where(keep, do[b, h] @ v[b, kv].T, 0.0)
+            P = np.where(keep, q[b, h] @ k[b, kv].T, 0.0)
+            dq[b, h] = dP @ k[b, kv]
+            dk[b, kv] += dP.T @ q[b, h]
+            dv[b, kv] += P.T @ do[b, h]
+    return dq, dk, dv
 
 
 def kv_state(k, v, state=None) -> np.ndarray:
