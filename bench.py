@@ -2,11 +2,15 @@
 """Causal linear-attention forward throughput on B200 (Lightning Attention-2).
 
 One step = one causal forward pass O = ((Q K^T) ⊙ M) V over one batch of the
-workload (default: B=4, H=16, N=2048, d=dv=128, block 64, bf16 in/out, fp32
-accumulation and state), through libla2's C ABI. Prints one JSON line.
+workload (default: the long-context case B=1, H=8, N=524288, d=dv=128,
+block 128, bf16 in/out, fp32 accumulation and state), through libla2's C ABI.
+Prints one JSON line.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                   [--impl reference] [--sweep]
+
+--sweep adds one line per other workload: B=4 H=16 N=2048, the sequence-length
+sweep, the non-causal form, forward + backward and the decode step.
 
 N > 1 is launched with torch.distributed.run: every rank runs the same
 workload on its own GPU (independent (b, h) sequences, no data-path
@@ -32,6 +36,7 @@ sys.path.insert(0, ROOT)
 L2_BYTES = 126 * 1024 * 1024
 CLOCK_RAMP_S = 0.2
 METRIC = "causal linear-attn fwd tokens/s (B·H·N/s), TFLOP/s, % of roofline, 1 B200"
+FWDBWD_METRIC = "causal linear-attn fwd+bwd tokens/s (B·H·N/s), TFLOP/s, % of roofline, 1 B200"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
@@ -41,7 +46,7 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="bf16_b4h16_n2k")
+    ap.add_argument("--workload", default="bf16_long_512k")
     ap.add_argument("--block", type=int, default=0, help="override the workload's block size")
     ap.add_argument("--N", type=int, default=0, help="override the sequence length")
     ap.add_argument("--impl", default="la2", choices=["la2", "reference"])
@@ -178,76 +183,149 @@ def workload_from_args(args):
 
 
 def flops_per_token(w, causal=True):
-    if not causal:  # O = Q (K^T V): the state pass and the map pass
-        return 4 * w.d * w.dv
-    return 2 * w.block * (w.d + w.dv) + 4 * w.d * w.dv
+    """Dense-tile flops per token·head of one step (the N^2 work LA2 avoids is
+    not counted). Forward: S = Q K^T and P V inside a block (2 Bk d + 2 Bk dv),
+    Q KV and the state update (2 d dv each); non-causal: K^T V and Q KV only.
+    A forward + backward step adds the backward's 2 Bk (3d + 2dv) + 10 d dv
+    (dP and S inside a block, the dQ, dK, dV products, two state updates)."""
+    if not causal:
+        f = 4 * w.d * w.dv
+    else:
+        f = 2 * w.block * (w.d + w.dv) + 4 * w.d * w.dv
+    if w.backward:
+        f += 2 * w.block * (3 * w.d + 2 * w.dv) + 10 * w.d * w.dv
+    return f
 
 
 def bytes_per_token(w):
+    """HBM bytes per token·head each step must move at least: the forward reads
+    Q, K, V and writes O; the backward reads Q, K, V, dO and writes dQ, dK, dV."""
     es = 2 if w.dtype == "bf16" else 4
-    return (2 * w.d + 2 * w.dv) * es
+    b = (2 * w.d + 2 * w.dv) * es
+    if w.backward:
+        b += (4 * w.d + 3 * w.dv) * es
+    return b
 
 
 # -------------------------------------------------------------- CPU oracle
 
 
-def cpu_oracle_rate(w, budget_s=10.0, max_heads=None):
-    """Time the float64 oracle (as it stands) on whole (b, h) sequences of the
-    workload until ~budget_s of CPU work; returns (tokens/s, sample text, cores)."""
-    import torch
+# Sequences longer than this are timed in the oracle's RNN form over a prefix
+# of one sequence (its left product is O(N^2) per sequence), plus the left
+# product at sampled rows.
+LEFT_PRODUCT_MAX_N = 16384
+RNN_SAMPLE_TOKENS = 16384
+ROW_SAMPLE = 64
 
-    import oracle
-    from linear_attention_la2_b200 import inputs as I
 
+def _oracle_cores():
     try:
         from threadpoolctl import threadpool_info
 
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
     except Exception:  # pragma: no cover
-        cores = os.cpu_count() or 1
-    g = torch.Generator().manual_seed(w.seed)
-    scale = 1.0 / math.sqrt(w.d)
-    heads, tokens, elapsed = 0, 0, 0.0
-    limit = max_heads or w.B * w.H
-    while heads == 0 or (elapsed < budget_s and heads < limit):
-        q = (torch.randn((1, 1, w.N, w.d), generator=g) * scale).to(w.torch_dtype)
-        k = (torch.randn((1, 1, w.N, w.d), generator=g) * scale).to(w.torch_dtype)
-        v = (torch.randn((1, 1, w.N, w.dv), generator=g) * scale).to(w.torch_dtype)
-        t0 = time.perf_counter()
-        oracle.forward(q, k, v, True)
-        elapsed += time.perf_counter() - t0
-        heads += 1
-        tokens += w.N
-    sample = (f"{heads} whole (b,h) sequences of N={w.N} (of {w.B * w.H}), float64 left product "
-              f"O=((QK^T)⊙M)V, {elapsed:.1f} s")
-    return tokens / elapsed, sample, cores
+        return os.cpu_count() or 1
+
+
+def oracle_sample_plan(w, causal=True):
+    """What one bounded oracle sample of workload ``w`` computes: (form, tokens
+    per sample, text). Whole (b, h) sequences with the float64 left product
+    (and the closed-form backward for a forward + backward step) when one
+    sequence costs about a second or less; else the float64 RNN form over the
+    first RNN_SAMPLE_TOKENS tokens of a sequence."""
+    if w.N <= LEFT_PRODUCT_MAX_N or not causal:
+        what = "left product O=((QK^T)⊙M)V" if causal else "left product O=(QK^T)V"
+        if w.backward:
+            what += " + closed-form dQ, dK, dV"
+        return "left", w.N, f"one whole (b,h) sequence of N={w.N}, float64 {what}"
+    n = min(w.N, RNN_SAMPLE_TOKENS)
+    return "rnn", n, (f"the first {n} tokens of one (b,h) sequence of N={w.N}, float64 RNN form "
+                      "KV_t = KV_(t-1) + k_t^T v_t, o_t = q_t KV_t (the left product is "
+                      "O(N^2) per sequence at this length)")
+
+
+def oracle_sample(w, i, causal=True):
+    """Run one bounded oracle sample (the ``i``-th; inputs drawn with the
+    workload's recipe and seed ``w.seed + i``, outside the timing). Returns
+    (tokens, seconds)."""
+    import oracle
+    from linear_attention_la2_b200 import inputs as I
+
+    form, n, _ = oracle_sample_plan(w, causal)
+    ins = I.make_custom(1, 1, n, w.d, w.dv, w.dtype, seed=w.seed + i, with_grad_out=w.backward)
+    t0 = time.perf_counter()
+    if form == "left":
+        oracle.forward(ins["q"], ins["k"], ins["v"], causal)
+        if w.backward:
+            oracle.backward(ins["q"], ins["k"], ins["v"], ins["do"], causal)
+    else:
+        oracle.recurrent_forward(ins["q"], ins["k"], ins["v"])
+    return n, time.perf_counter() - t0
+
+
+def oracle_rows_rate(w, rows=ROW_SAMPLE):
+    """Left product at ``rows`` sampled rows of one sequence of full length N
+    (float64): output rows per second. The O(N^2) definition itself, where a
+    whole sequence is out of reach."""
+    import oracle
+    from linear_attention_la2_b200 import inputs as I
+
+    ins = I.make_custom(1, 1, w.N, w.d, w.dv, w.dtype, seed=w.seed)
+    rr = I.sample_rows(w.N, w.block, w.seed, count=rows, max_blocks=2)[-rows:]
+    t0 = time.perf_counter()
+    oracle.forward_rows(ins["q"], ins["k"], ins["v"], rr, True)
+    return len(rr) / (time.perf_counter() - t0), len(rr)
+
+
+def cpu_oracle_rate(w, budget_s=10.0, causal=True):
+    """The oracle as it stands, timed on the host cores: one untimed warm-up
+    sample, then samples (oracle_sample) until about ``budget_s`` seconds.
+    The reference arm times the same samples, one per step."""
+    _, _, text = oracle_sample_plan(w, causal)
+    oracle_sample(w, 0, causal)
+    tokens, elapsed, k = 0, 0.0, 0
+    while k == 0 or (elapsed < budget_s and k < 64):
+        n, t = oracle_sample(w, k + 1, causal)
+        tokens += n
+        elapsed += t
+        k += 1
+    rec = {"value": tokens / elapsed, "unit": "tokens/s", "cores": _oracle_cores(), "kind": "oracle",
+           "sample": f"{k} samples, each {text}; {elapsed:.1f} s"}
+    if oracle_sample_plan(w, causal)[0] == "rnn":
+        rate, nrows = oracle_rows_rate(w)
+        rec["left_product_rows_per_s"] = rate
+        rec["left_product_sample"] = (f"{nrows} sampled rows of one sequence of N={w.N}, float64 "
+                                      "left product (output rows/s; a full sequence needs N rows)")
+    return rec
 
 
 def run_reference(args):
-    """--impl reference: the oracle on the host cores, same metric and config."""
+    """--impl reference: the oracle on the host cores, same metric and config;
+    each step is one bounded sample of the workload (oracle_sample)."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
     w = workload_from_args(args)
-    # one step = one whole (b, h) sequence of the workload
-    rate_steps = []
+    _, _, text = oracle_sample_plan(w)
+    total, tokens = 0.0, 0
     for i in range(args.warmup + args.steps):
-        r, sample, cores = cpu_oracle_rate(w, budget_s=0.0, max_heads=1)
+        n, t = oracle_sample(w, i)
         if i >= args.warmup:
-            rate_steps.append(w.N / r)
-    total = sum(rate_steps)
-    value = args.steps * w.N / total
+            total += t
+            tokens += n
+    value = tokens / total
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": config_of(w),
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                         "sample": f"each step: one (b,h) sequence of N={w.N} of the workload, "
-                                   "float64 left product on host cores"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": _oracle_cores(),
+                         "kind": "oracle", "sample": f"each step: {text}, on host cores"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
+    if w.backward:
+        line["metric"] = FWDBWD_METRIC
     print(json.dumps(line))
     return 0
 
@@ -287,18 +365,17 @@ def run_gpu(args):
     if rank == 0:
         print(json.dumps(line), flush=True)
     if args.sweep:
-        for N in I.SWEEP_N:
-            for b in I.SWEEP_BLOCKS:
-                sw = I.sweep_workload(N, b)
-                ln = bench_workload(args, sw, dev, la2, world, rank, local, hbm, peak_kind, main=False)
-                if rank == 0:
-                    print(json.dumps(ln), flush=True)
-        lw = I.WORKLOADS["bf16_long_512k"]
-        ln = bench_workload(args, lw, dev, la2, world, rank, local, hbm, peak_kind, main=False)
-        if rank == 0:
-            print(json.dumps(ln), flush=True)
-    if args.sweep:
-        ln = bench_workload(args, w, dev, la2, world, rank, local, hbm, peak_kind, main=False,
+        others = [I.WORKLOADS["bf16_b4h16_n2k"]]
+        others += [I.sweep_workload(N, b) for N in I.SWEEP_N for b in I.SWEEP_BLOCKS]
+        others += [I.WORKLOADS["bf16_long_512k"], I.WORKLOADS["bf16_fwdbwd_b2h32_n8k"]]
+        for sw in others:
+            if sw.name == w.name:
+                continue
+            ln = bench_workload(args, sw, dev, la2, world, rank, local, hbm, peak_kind, main=False)
+            if rank == 0:
+                print(json.dumps(ln), flush=True)
+        nc = I.WORKLOADS["bf16_b4h16_n2k"]
+        ln = bench_workload(args, nc, dev, la2, world, rank, local, hbm, peak_kind, main=False,
                             causal=False)
         if rank == 0:
             print(json.dumps(ln), flush=True)
@@ -453,19 +530,9 @@ def bench_workload(args, w, dev, la2, world, rank, local, hbm, peak_kind, main, 
             launches += n
     # every step launches the same kernels: scale the timed sample to all steps
     launches = launches * args.steps // max(1, profiled_steps)
-    dom = max(per_kernel, key=lambda k: per_kernel[k]["ms"]) if per_kernel else None
-
     value = whole_job_rate(w.tokens, args.steps, world, ms_max)
     tflops = flops_per_token(w, causal) * value / 1e12
-    roofline = None
-    if dom:
-        avg_ms = per_kernel[dom]["ms"] / per_kernel[dom]["launches"]
-        alg_bytes = w.tokens * bytes_per_token(w)
-        achieved = alg_bytes / (avg_ms / 1e3) / 1e9
-        roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                    "frac": achieved / hbm, "traffic": recorded_traffic(dom, w.name),
-                    "kernel": dom, "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)"
-                    if peak_kind == "measured" else "fallback 6.65 TB/s"}
+    roofline = op_roofline(w, per_kernel, profiled_steps, hbm, peak_kind, causal)
     step_frac = (w.tokens * bytes_per_token(w) * args.steps * world / (ms_max / 1e3) / 1e9) / (hbm * world)
 
     line = {
@@ -487,15 +554,41 @@ def bench_workload(args, w, dev, la2, world, rank, local, hbm, peak_kind, main, 
     if clocks:
         line["clocks"] = clocks
     if w.backward:
-        line["metric"] = "causal linear-attn fwd+bwd tokens/s (B·H·N/s), 1 B200"
+        line["metric"] = FWDBWD_METRIC
         line["config"]["workload"] += " (+ backward)"
     if main and not args.no_e2e and not w.backward:
         line["e2e"] = e2e_measure(args, w, dev, la2, world, base, ws, ws_bytes, dt)
     if main and rank == 0 and world == 1 and not args.no_cpu_baseline:
-        r, sample, cores = cpu_oracle_rate(w, budget_s=10.0)
-        line["cpu_baseline"] = {"value": r, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                                "sample": sample}
+        line["cpu_baseline"] = cpu_oracle_rate(w, budget_s=10.0, causal=causal)
     return line
+
+
+def op_roofline(w, per_kernel, profiled_steps, hbm, peak_kind, causal=True):
+    """Roofline of the whole op: the algorithmic bytes of one step over the
+    summed device time of every launch of that step (CUDA events around each
+    launch on the launching stream). Per kernel: launches and time per step,
+    and its share of the step's kernel time. ``traffic`` is the summed DRAM
+    bytes (ncu) of one step's launches when every kernel of the step has a
+    capture taken on the current sources, else None."""
+    if not per_kernel or profiled_steps < 1:
+        return None
+    step_ms = sum(v["ms"] for v in per_kernel.values()) / profiled_steps
+    alg_bytes = w.tokens * bytes_per_token(w)
+    achieved = alg_bytes / (step_ms / 1e3) / 1e9
+    kernels, traffic = {}, 0
+    tag = w.name if causal else w.name + "_noncausal"
+    for name, v in per_kernel.items():
+        launches = v["launches"] / profiled_steps
+        kernels[name] = {"launches_per_step": launches, "ms_per_step": v["ms"] / profiled_steps,
+                         "share": v["ms"] / profiled_steps / step_ms}
+        rec = recorded_traffic(name, tag)
+        traffic = None if (traffic is None or rec is None) else traffic + rec * launches
+    dom = max(kernels, key=lambda k: kernels[k]["ms_per_step"])
+    return {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+            "traffic": traffic, "alg_bytes_per_step": alg_bytes, "scope": "op",
+            "kernel": dom, "kernels": kernels,
+            "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)" if peak_kind == "measured"
+            else "fallback 6.65 TB/s"}
 
 
 DECODE = dict(name="bf16_decode_b64h32", B=64, H=32, d=128, dv=128, seed=5)

@@ -31,11 +31,19 @@
  *    pointers may then be NULL. Negative sizes, d or dv < 1, causal not in
  *    {0, 1}, an unknown dtype, a NULL or misaligned pointer, or outputs
  *    overlapping inputs give LA2_ERR_INVALID_ARG.
- *  - Supported shapes. LA2_BF16: d, dv in {64, 128}, block in {64, 128}
- *    (tensor-core path, fp32 accumulation and fp32 state). LA2_F32: any
+ *  - Supported shapes. LA2_BF16: d, dv in {64, 128}, block in {64, 128};
+ *    d = dv = 128 runs on the tensor cores (tcgen05, fp32 accumulation in
+ *    tensor memory, fp32 state), every other bf16 shape on the CUDA-core
+ *    kernels (fp32 accumulation and state as well). LA2_F32: any
  *    1 <= d, dv <= 128 and block in {16, 32, 64, 128} whose tiles fit in
  *    shared memory (fp32 CUDA-core path). Anything else gives
  *    LA2_ERR_UNSUPPORTED.
+ *  - Thread safety. The compute entry points keep no state between calls
+ *    apart from a small cache of work plans (mutex-protected). Three
+ *    process-wide settings are test and benchmark hooks, NOT thread-safe:
+ *    la2_set_chunk_len, la2_set_spin_limit and the la2_profile_* calls. Set
+ *    them before other threads call the library, and leave them at their
+ *    defaults (0) in production.
  *  - `block` is the algorithm's block size Bk. N need not be a multiple of
  *    it: the ragged last block is zero-padded on load and not stored.
  *  - Gradients are those of L = <dO, O>; backward needs no saved forward
@@ -114,15 +122,17 @@ LA2_API la2_status la2_check(la2_stream_t stream);
 LA2_API const char *la2_status_string(la2_status s);
 
 /*
- * Work split override. 0 (the default) lets the library split the work
- * from B*H, N and the SM count (see la2_plan_ranges). A positive value cuts
- * every sequence into chunks of `chunk_len` rows (rounded up to a multiple of
- * `block`) that run in parallel from the sum of the earlier chunks' KV states
- * (a sum, so any split gives the same result up to fp32 rounding order).
- * Process-wide; it changes la2_workspace_size for later calls. A forced split
- * of the tensor-core causal forward into more than 160 chunks in total gives
- * LA2_ERR_UNSUPPORTED at the call. Returns LA2_ERR_INVALID_ARG for a negative
- * value.
+ * Work split override, a test hook. 0 (the default) lets the library split
+ * the work from B*H, N and the SM count (see la2_plan_ranges). A positive
+ * value cuts every sequence into chunks of `chunk_len` rows (rounded up to a
+ * multiple of `block`) that run in parallel from the sum of the earlier
+ * chunks' KV states (a sum, so any split gives the same result up to fp32
+ * rounding order). Process-wide and not thread-safe: it changes the plan and
+ * la2_workspace_size of every later call from any thread. A forced split of the
+ * tensor-core causal path into more than 160 chunks in total runs on the
+ * chunk kernels instead of the persistent range split (same results; the
+ * workspace size accounts for it). Returns LA2_ERR_INVALID_ARG for a
+ * negative value.
  */
 LA2_API la2_status la2_set_chunk_len(int64_t chunk_len);
 
@@ -177,6 +187,7 @@ LA2_API la2_status la2_decode_step(const void *q, const void *k, const void *v, 
  * flag). When a wait exceeds it the kernel records LA2_ERR_TIMEOUT in the
  * device error word, stops its work and returns; la2_check() reports it.
  * 0 restores the default (large enough to be reached only by a fault).
+ * Process-wide test hook, not thread-safe.
  */
 LA2_API la2_status la2_set_spin_limit(int64_t iterations);
 
@@ -189,7 +200,8 @@ LA2_API la2_status la2_set_spin_limit(int64_t iterations);
  * synchronises the events and returns, for kernel id `kernel`, the number of
  * recorded launches and their summed device time in ms since the last
  * la2_profile_enable(1). Ids run from 0 to la2_profile_num_kernels()-1 and
- * la2_profile_kernel_name() names them. Not thread-safe.
+ * la2_profile_kernel_name() names them. Process-wide benchmark hook, not
+ * thread-safe: while enabled, the launches of every thread are recorded.
  */
 LA2_API la2_status la2_profile_enable(int on);
 LA2_API int la2_profile_num_kernels(void);

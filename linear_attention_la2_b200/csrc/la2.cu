@@ -166,10 +166,16 @@ static Plan make_plan_uncached(int64_t B, int64_t H, int64_t N, int64_t d, int64
   }
   L = std::max<int64_t>(L, block);
   const size_t state_bytes = (size_t)d * (size_t)dv * sizeof(float);
+  // The range split runs when its table holds the ranges (always for the
+  // automatic plan; a forced split of many sequences can exceed it) and its
+  // task indices fit in 32 bits. Otherwise the chunk path below runs, for the
+  // forward as for the backward's dQ pass.
+  bool range_fits = false;
   if (p.tc && causal) {
-    p.ranges = true;
     p.rp = plan_ranges(BH, N, block, sms, g_chunk_len);
-    if (!is_bwd) {
+    range_fits = p.rp.R >= 1 && p.rp.R <= sm100::kMaxRanges && BH * T <= 0x7fffffff;
+    p.ranges = range_fits;
+    if (!is_bwd && range_fits) {
       p.need_states = p.rp.prefix_mode == 1;
       p.ws_bytes = p.need_states ? (size_t)p.rp.R * state_bytes : 0;
       return p;
@@ -184,7 +190,7 @@ static Plan make_plan_uncached(int64_t B, int64_t H, int64_t N, int64_t d, int64
     // Workspace: [U chunk states | K^T V chunk states or the dQ pass's range
     // states, whichever is larger]. The dQ pass takes the range split when
     // its table can hold the ranges, else the chunk path.
-    p.dq_ranges = p.rp.R >= 1 && p.rp.R <= sm100::kMaxRanges;
+    p.dq_ranges = range_fits;
     const size_t agg = p.dq_ranges && p.rp.prefix_mode == 1 ? (size_t)p.rp.R * state_bytes : 0;
     const size_t kv = p.need_states ? one : 0;
     p.ws_bytes = (p.need_states ? one : 0) + std::max(agg, kv);
@@ -342,7 +348,7 @@ template <int BK>
 static la2_status forward_sm100_bk(const void* q, const void* k, const void* v, void* o,
                                    int64_t BH, int64_t N, int causal, float* states,
                                    const Plan& p, int64_t spin, cudaStream_t st) {
-  if (causal)
+  if (causal && p.ranges)
     return causal_range_split<BK>(q, k, v, o, BH, N, states, p.rp, spin, st, K_STATE_TC, K_FWD_TC);
   constexpr int D = 128, DV = 128;
   CUtensorMap tq, tk, tv;
@@ -357,6 +363,28 @@ static la2_status forward_sm100_bk(const void* q, const void* k, const void* v, 
   prm.spin_limit = spin;
   la2_status s = LA2_OK;
   const int nel = D * DV;
+  CUtensorMap to_c = tq;
+  if (sm100::Cfg<BK, D, DV>::TMA_STORE && !make_tmap_3d(&to_c, o, BH, N, DV, 16)) return LA2_ERR_CUDA;
+  if (causal) {
+    // A split the range table cannot hold: chunk states, their exclusive
+    // prefix per sequence, then every chunk's block loop from its prefix.
+    if (p.need_states) {
+      sm100::Params ps = prm;
+      ps.out_states = states;
+      ps.units_per_seq = p.C;
+      {
+        LaunchTimer t(K_STATE_TC, st);
+        s = launch_fwd_sm100<BK, D, DV, sm100::MODE_STATE>(tq, tk, tv, tq, ps, BH * p.C, st);
+      }
+      if (s != LA2_OK) return s;
+      s = run_scan(states, BH, nel, p, 0, st);
+      if (s != LA2_OK) return s;
+    }
+    prm.init_states = p.need_states ? states : nullptr;
+    prm.units_per_seq = p.C;
+    LaunchTimer t(K_FWD_TC, st);
+    return launch_fwd_sm100<BK, D, DV, sm100::MODE_CAUSAL>(tq, tk, tv, to_c, prm, BH * p.C, st);
+  }
   sm100::Params ps = prm;
   ps.out_states = states;
   ps.units_per_seq = p.C;
@@ -373,10 +401,8 @@ static la2_status forward_sm100_bk(const void* q, const void* k, const void* v, 
   }
   prm.init_states = states;
   prm.units_per_seq = p.C;
-  CUtensorMap to_nc = tq;
-  if (sm100::Cfg<BK, D, DV>::TMA_STORE && !make_tmap_3d(&to_nc, o, BH, N, DV, 16)) return LA2_ERR_CUDA;
   LaunchTimer t(K_FWD_TC, st);
-  return launch_fwd_sm100<BK, D, DV, sm100::MODE_NONCAUSAL>(tq, tk, tv, to_nc, prm, BH * p.C, st);
+  return launch_fwd_sm100<BK, D, DV, sm100::MODE_NONCAUSAL>(tq, tk, tv, to_c, prm, BH * p.C, st);
 }
 
 // Tensor-core backward: chunk states K^T V (prefix for dQ) and Q^T dO

@@ -806,12 +806,14 @@ la2_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           const int64_t y = t0 + static_cast<int64_t>(i) * BK + 16 * w4;
           // A chunk ends on a block boundary or at N, so the tensor map's
           // bound at N is the only clip needed.
-          if (lane == 0 && y < t1) {
+          if (lane == 0) {
+            if (y < t1) {
 #pragma unroll
-            for (int p = 0; p < DV / 64; ++p)
-              tma_store_3d(&tm_o, stage + p * BK * 128, 64 * p, static_cast<int>(y),
-                           static_cast<int>(bh));
-            bulk_commit_group();
+              for (int p = 0; p < DV / 64; ++p)
+                tma_store_3d(&tm_o, stage + p * BK * 128, 64 * p, static_cast<int>(y),
+                             static_cast<int>(bh));
+            }
+            bulk_commit_group();  // one group per block (empty past the end): see the wait above
           }
           continue;
         }

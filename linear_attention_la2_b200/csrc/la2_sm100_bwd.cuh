@@ -406,16 +406,18 @@ la2_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         __syncwarp();
         // chunks end on block boundaries or at N (the tensor maps clip at N)
         const int64_t y = t0 + static_cast<int64_t>(i) * BK + 16 * w4;
-        if (lane == 0 && y < t1) {
-          for (int which = 0; which < 2; ++which) {
-            uint8_t* stage = smem + CF::OFF_OST + which * CF::TILE + w4 * 16 * 128;
-            const CUtensorMap* map = which == 0 ? &tm_dv : &tm_dk;
+        if (lane == 0) {
+          if (y < t1) {
+            for (int which = 0; which < 2; ++which) {
+              uint8_t* stage = smem + CF::OFF_OST + which * CF::TILE + w4 * 16 * 128;
+              const CUtensorMap* map = which == 0 ? &tm_dv : &tm_dk;
 #pragma unroll
-            for (int p = 0; p < 2; ++p)
-              tma_store_3d(map, stage + p * BK * 128, 64 * p, static_cast<int>(y),
-                           static_cast<int>(bh));
+              for (int p = 0; p < 2; ++p)
+                tma_store_3d(map, stage + p * BK * 128, 64 * p, static_cast<int>(y),
+                             static_cast<int>(bh));
+            }
           }
-          bulk_commit_group();
+          bulk_commit_group();  // one group per block, empty past the end
         }
         continue;
       }

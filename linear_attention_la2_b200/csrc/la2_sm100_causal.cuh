@@ -823,11 +823,17 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           fence_proxy_async();
           __syncwarp();
           const int64_t y = static_cast<int64_t>(st.blk) * BK + 16 * w4;
-          if (lane == 0 && y < prm.N) {  // rows past N are clipped by the tensor map
+          if (lane == 0) {
+            if (y < prm.N) {  // rows past N are clipped by the tensor map
 #pragma unroll
-            for (int p = 0; p < DV / 64; ++p)
-              tma_store_3d(&tm_o, stage + p * BK * 128, 64 * p, static_cast<int>(y),
-                           static_cast<int>(st.bh));
+              for (int p = 0; p < DV / 64; ++p)
+                tma_store_3d(&tm_o, stage + p * BK * 128, 64 * p, static_cast<int>(y),
+                             static_cast<int>(st.bh));
+            }
+            // One bulk group per block, empty when every row of this warp lies
+            // past N: the wait above counts groups, and a skipped group would
+            // let block m reuse the staging tile that block m-2's store may
+            // still be reading (a range can run on into the next sequence).
             bulk_commit_group();
           }
           if (threadIdx.x % 128 == 0) LA2_TRACE_POINT(12, m);

@@ -157,12 +157,17 @@ def workspace_bytes(B, H, N, d, dv, causal, block, dtype_code, is_backward) -> i
     return int(n)
 
 
-def _workspace(nbytes, device):
+def _workspace(nbytes, device, stream):
+    """Scratch for one call, allocated on the stream the kernels run on, so the
+    caching allocator cannot hand it to other work while they still use it."""
     import torch
 
     if nbytes == 0:
         return None
-    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+    if stream is None:
+        return torch.empty(nbytes, dtype=torch.uint8, device=device)
+    with torch.cuda.stream(stream):
+        return torch.empty(nbytes, dtype=torch.uint8, device=device)
 
 
 def _check_inputs(*ts):
@@ -173,18 +178,45 @@ def _check_inputs(*ts):
             raise La2Error(LA2_ERR_INVALID_ARG)
 
 
+def _check_like(ref, shape, dtype, *ts):
+    """Every tensor in ``ts`` must have ``shape``, ``dtype`` and ref's device:
+    the library sizes every tensor map and loop from q's shape, so a shorter
+    k, v, dO or output would be read or written past its end."""
+    for t in ts:
+        if tuple(t.shape) != tuple(shape) or t.dtype != dtype or t.device != ref.device:
+            raise La2Error(LA2_ERR_INVALID_ARG)
+
+
+def _check_workspace(ws, need, device):
+    import torch
+
+    if ws is None:
+        if need:
+            raise La2Error(LA2_ERR_WORKSPACE)
+        return
+    if not ws.is_cuda or ws.device != device or not ws.is_contiguous() or ws.dtype != torch.uint8:
+        raise La2Error(LA2_ERR_INVALID_ARG)
+
+
 def forward(q, k, v, causal: bool = True, block: int = 64, out=None, workspace=None, stream=None):
     """O = ((Q K^T) ⊙ M) V for [B,H,N,d] CUDA tensors; returns O."""
     import torch
 
     _check_inputs(q, k, v)
+    if q.dim() != 4 or v.dim() != 4:
+        raise La2Error(LA2_ERR_INVALID_ARG)
     B, H, N, d = q.shape
     dv = v.shape[-1]
     dt = _dtype_code(q)
+    _check_like(q, q.shape, q.dtype, k)
+    _check_like(q, (B, H, N, dv), q.dtype, v)
     if out is None:
         out = torch.empty((B, H, N, dv), dtype=q.dtype, device=q.device)
+    _check_inputs(out)
+    _check_like(q, (B, H, N, dv), q.dtype, out)
     need = workspace_bytes(B, H, N, d, dv, causal, block, dt, False)
-    ws = workspace if workspace is not None else _workspace(need, q.device)
+    ws = workspace if workspace is not None else _workspace(need, q.device, stream)
+    _check_workspace(ws, need, q.device)
     _raise(la2_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, N, d, dv, int(causal), block, dt,
                        _ptr(ws), ws.numel() if ws is not None else 0, _stream_handle(stream)))
     return out
@@ -196,14 +228,22 @@ def backward(q, k, v, do, causal: bool = True, block: int = 64, outs=None, works
     import torch
 
     _check_inputs(q, k, v, do)
+    if q.dim() != 4 or v.dim() != 4:
+        raise La2Error(LA2_ERR_INVALID_ARG)
     B, H, N, d = q.shape
     dv = v.shape[-1]
     dt = _dtype_code(q)
+    _check_like(q, q.shape, q.dtype, k)
+    _check_like(q, (B, H, N, dv), q.dtype, v, do)
     if outs is None:
         outs = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
     dq, dk, dvv = outs
+    _check_inputs(dq, dk, dvv)
+    _check_like(q, q.shape, q.dtype, dq, dk)
+    _check_like(q, (B, H, N, dv), q.dtype, dvv)
     need = workspace_bytes(B, H, N, d, dv, causal, block, dt, True)
-    ws = workspace if workspace is not None else _workspace(need, q.device)
+    ws = workspace if workspace is not None else _workspace(need, q.device, stream)
+    _check_workspace(ws, need, q.device)
     _raise(la2_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dvv), B, H, N,
                         d, dv, int(causal), block, dt, _ptr(ws), ws.numel() if ws is not None else 0,
                         _stream_handle(stream)))
@@ -216,18 +256,21 @@ def kv_state(k, v, state=None, workspace=None, stream=None):
     import torch
 
     _check_inputs(k, v)
+    if k.dim() != 4 or v.dim() != 4:
+        raise La2Error(LA2_ERR_INVALID_ARG)
     B, H, N, d = k.shape
     dv = v.shape[-1]
     dt = _dtype_code(k)
+    _check_like(k, (B, H, N, dv), k.dtype, v)
     if state is None:
         state = torch.zeros((B, H, d, dv), dtype=torch.float32, device=k.device)
     _check_inputs(state)
-    if state.dtype != torch.float32:
-        raise La2Error(LA2_ERR_INVALID_ARG)
+    _check_like(k, (B, H, d, dv), torch.float32, state)
     need = la2_kv_state_workspace_size(B, H, N, d, dv, dt)
     if need == ctypes.c_size_t(-1).value:
         raise La2Error(LA2_ERR_INVALID_ARG)
-    ws = workspace if workspace is not None else _workspace(need, k.device)
+    ws = workspace if workspace is not None else _workspace(need, k.device, stream)
+    _check_workspace(ws, need, k.device)
     _raise(la2_kv_state(_ptr(k), _ptr(v), _ptr(state), B, H, N, d, dv, dt, _ptr(ws),
                         ws.numel() if ws is not None else 0, _stream_handle(stream)))
     return state
@@ -239,12 +282,18 @@ def decode_step(q, k, v, state, out=None, stream=None):
     import torch
 
     _check_inputs(q, k, v, state)
-    if state.dtype != torch.float32:
+    if q.dim() != 3 or v.dim() != 3:
         raise La2Error(LA2_ERR_INVALID_ARG)
     B, H, d = q.shape
     dv = v.shape[-1]
+    _dtype_code(q)
+    _check_like(q, q.shape, q.dtype, k)
+    _check_like(q, (B, H, dv), q.dtype, v)
+    _check_like(q, (B, H, d, dv), torch.float32, state)
     if out is None:
         out = torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
+    _check_inputs(out)
+    _check_like(q, (B, H, dv), q.dtype, out)
     _raise(la2_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(state), B, H, d, dv,
                            _dtype_code(q), _stream_handle(stream)))
     return out

@@ -25,6 +25,41 @@ def test_work_per_token_matches_the_block_algorithm():
     assert bench.bytes_per_token(I.WORKLOADS["fp32_small"]) == (2 * 64 + 2 * 64) * 4
 
 
+def test_work_per_token_of_a_forward_backward_step():
+    w = I.WORKLOADS["bf16_fwdbwd_b2h32_n8k"]
+    # forward 1024 B; backward reads Q, K, V, dO and writes dQ, dK, dV: 1792 B
+    assert bench.bytes_per_token(w) == 1024 + 1792 == 2816
+    assert bench.flops_per_token(w) == 98304 + 2 * 64 * (3 * 128 + 2 * 128) + 10 * 128 * 128
+    assert bench.flops_per_token(w) == 98304 + 245760
+
+
+def test_op_roofline_counts_every_launch_of_the_step():
+    w = I.WORKLOADS["bf16_long_512k"]
+    per_kernel = {"main": {"launches": 2, "ms": 1.5}, "state": {"launches": 2, "ms": 0.5}}
+    r = bench.op_roofline(w, per_kernel, 2, 6545.0, "measured")
+    step_s = (1.5 + 0.5) / 2 / 1e3
+    assert r["scope"] == "op" and r["kernel"] == "main"
+    assert abs(r["achieved"] - w.tokens * 1024 / step_s / 1e9) < 1e-6
+    assert abs(r["frac"] - r["achieved"] / 6545.0) < 1e-12
+    assert abs(r["kernels"]["state"]["share"] - 0.25) < 1e-12
+    assert r["kernels"]["main"]["launches_per_step"] == 1
+    assert r["traffic"] is None  # no capture of these kernels on the current sources
+    assert bench.op_roofline(w, {}, 0, 6545.0, "measured") is None
+
+
+def test_oracle_samples_are_bounded():
+    long = I.WORKLOADS["bf16_long_512k"]
+    form, n, text = bench.oracle_sample_plan(long)
+    assert form == "rnn" and n == bench.RNN_SAMPLE_TOKENS and "RNN form" in text
+    form, n, _ = bench.oracle_sample_plan(I.WORKLOADS["bf16_b4h16_n2k"])
+    assert (form, n) == ("left", 2048)
+    form, n, text = bench.oracle_sample_plan(I.WORKLOADS["bf16_fwdbwd_b2h32_n8k"])
+    assert (form, n) == ("left", 8192) and "dQ, dK, dV" in text
+    small = I.WORKLOADS["fp32_small"]
+    n, t = bench.oracle_sample(small, 0)
+    assert n == 256 and t > 0
+
+
 def test_config_names_the_form():
     w = I.WORKLOADS["bf16_b4h16_n2k"]
     assert bench.config_of(w)["workload"].startswith("bf16_b4h16_n2k: causal forward")

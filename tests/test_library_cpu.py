@@ -159,3 +159,38 @@ def test_kv_state_rejects_bad_arguments():
     # state overlapping k
     assert ks(P[0], P[1], ctypes.c_void_p(0x1000000 + 256), 1, 1, 16, 64, 64, la2.LA2_F32, NULL, 0,
               NULL) == la2.LA2_ERR_INVALID_ARG
+
+
+def test_binding_rejects_mismatched_tensors():
+    """The binding checks every tensor against q before the library sizes its
+    tensor maps from q's shape (a shorter k, v or output would be read or
+    written past its end)."""
+    import torch
+
+    q = torch.zeros(1, 2, 16, 64)
+    la2._check_like(q, q.shape, q.dtype, torch.zeros(1, 2, 16, 64))
+    for bad in (torch.zeros(1, 2, 15, 64), torch.zeros(2, 2, 16, 64), torch.zeros(1, 2, 16, 32),
+                torch.zeros(1, 2, 16, 64, dtype=torch.bfloat16)):
+        with pytest.raises(la2.La2Error) as e:
+            la2._check_like(q, q.shape, q.dtype, bad)
+        assert e.value.code == la2.LA2_ERR_INVALID_ARG
+    # host tensors are rejected before anything reaches the library
+    for fn, args in ((la2.forward, (q, q, q)), (la2.backward, (q, q, q, q)),
+                     (la2.kv_state, (q, q)), (la2.decode_step, (q[0], q[0], q[0], q))):
+        with pytest.raises(la2.La2Error):
+            fn(*args)
+    with pytest.raises(la2.La2Error) as e:
+        la2._check_workspace(None, 256, None)
+    assert e.value.code == la2.LA2_ERR_WORKSPACE
+
+
+def test_header_states_the_tensor_core_shapes():
+    """The header's supported-shape text matches the dispatch: bf16 runs on the
+    tensor cores only at d = dv = 128."""
+    text = open(os.path.join(ROOT, "include", "la2.h")).read()
+    assert "d = dv = 128 runs on the tensor cores" in text
+    src = open(os.path.join(ROOT, "linear_attention_la2_b200", "csrc", "la2_sm100.cuh")).read()
+    assert "return d == 128 && dv == 128 && (block == 64 || block == 128);" in src
+    # bf16 shapes off the tensor-core path are accepted (pointer check fails first)
+    assert _fwd(dt=la2.LA2_BF16, d=64, dv=128) == la2.LA2_ERR_INVALID_ARG
+    assert _fwd(dt=la2.LA2_BF16, d=128, dv=64, block=128) == la2.LA2_ERR_INVALID_ARG
