@@ -112,6 +112,32 @@ LA2_API la2_status la2_backward(const void *q, const void *k, const void *v, con
                         void *workspace, size_t workspace_bytes, la2_stream_t stream);
 
 /*
+ * Grouped K/V heads: GQA, and MQA when Hkv = 1 (cccbook long-context chapter,
+ * section on MQA/GQA; mhpn.cn blog, section 3: several query heads share one
+ * key/value head). The same op per query head, with query head h of batch b
+ * reading K/V head h / (H / Hkv) of batch b:
+ *   o[b,h] = ((q[b,h] k[b,h/G]^T) ⊙ M) v[b,h/G],  G = H / Hkv.
+ * q, o: [B,H,N,d] / [B,H,N,dv]; k: [B,Hkv,N,d]; v: [B,Hkv,N,dv]; H must be a
+ * multiple of Hkv >= 1 (else LA2_ERR_INVALID_ARG). Every other convention as
+ * for la2_forward / la2_backward / la2_workspace_size; Hkv = H is exactly those
+ * calls. In the backward a K/V head's gradients add up over the query heads
+ * that read it: dk [B,Hkv,N,d] and dvv [B,Hkv,N,dv] receive those sums (fp32
+ * accumulation, one rounding to the element type); dq is [B,H,N,d].
+ */
+LA2_API size_t la2_workspace_size_gqa(int64_t B, int64_t H, int64_t Hkv, int64_t N, int64_t d,
+                                      int64_t dv, int causal, int block, la2_dtype dt,
+                                      int is_backward);
+LA2_API la2_status la2_forward_gqa(const void *q, const void *k, const void *v, void *o,
+                                   int64_t B, int64_t H, int64_t Hkv, int64_t N, int64_t d,
+                                   int64_t dv, int causal, int block, la2_dtype dt,
+                                   void *workspace, size_t workspace_bytes, la2_stream_t stream);
+LA2_API la2_status la2_backward_gqa(const void *q, const void *k, const void *v, const void *dout,
+                                    void *dq, void *dk, void *dvv, int64_t B, int64_t H,
+                                    int64_t Hkv, int64_t N, int64_t d, int64_t dv, int causal,
+                                    int block, la2_dtype dt, void *workspace,
+                                    size_t workspace_bytes, la2_stream_t stream);
+
+/*
  * Synchronises `stream`, then reports and clears the device-side error word
  * that kernels set when a bounded wait gives up (LA2_ERR_TIMEOUT), or
  * LA2_ERR_CUDA if the stream holds a CUDA error. LA2_OK otherwise.

@@ -119,8 +119,12 @@ static bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
 
 // Shape checks shared by every entry point. Returns LA2_OK or an error.
 static la2_status check_shape(int64_t B, int64_t H, int64_t N, int64_t d, int64_t dv, int causal,
-                              int block, la2_dtype dt, bool is_bwd) {
+                              int block, la2_dtype dt, bool is_bwd, int64_t Hkv = -1) {
+  if (Hkv < 0) Hkv = H;  // plain layout: one K/V head per query head
   if (B < 0 || H < 0 || N < 0 || d < 1 || dv < 1) return LA2_ERR_INVALID_ARG;
+  // grouped heads: Hkv >= 1 divides H (an empty H takes any Hkv >= 0)
+  if (H > 0 && (Hkv < 1 || H % Hkv != 0)) return LA2_ERR_INVALID_ARG;
+  if (H > 0x7fffffff) return LA2_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return LA2_ERR_INVALID_ARG;
   if (dt != LA2_F32 && dt != LA2_BF16) return LA2_ERR_INVALID_ARG;
   if (block < 1) return LA2_ERR_INVALID_ARG;
@@ -140,14 +144,18 @@ static la2_status check_shape(int64_t B, int64_t H, int64_t N, int64_t d, int64_
                              : fwd_simt_smem((int)d, (int)dv, block, es);
   const bool tc = (dt == LA2_BF16) && sm100_supports(d, dv, block, is_bwd);
   if (!tc && smem > 227 * 1024) return LA2_ERR_UNSUPPORTED;
+  if (!tc && is_bwd && !bwd_dkdv_simt_fits((int)d, (int)dv, block)) return LA2_ERR_UNSUPPORTED;
   return LA2_OK;
 }
 
-static Plan make_plan_uncached(int64_t B, int64_t H, int64_t N, int64_t d, int64_t dv, int causal,
-                               int block, la2_dtype dt, bool is_bwd, int sms) {
+static Plan make_plan_uncached(int64_t B, int64_t H, int64_t Hkv, int64_t N, int64_t d, int64_t dv,
+                               int causal, int block, la2_dtype dt, bool is_bwd, int sms) {
   Plan p;
   const int64_t BH = B * H;
+  const int64_t BHkv = B * Hkv;
   const int64_t T = (N + block - 1) / block;
+  // The backward's heaviest pass (dK, dV) runs one unit per K/V sequence and chunk.
+  const int64_t BHu = is_bwd ? BHkv : BH;
   p.tc = (dt == LA2_BF16) && sm100_supports(d, dv, block, is_bwd);
   int64_t L;
   if (g_chunk_len > 0) {
@@ -159,8 +167,8 @@ static Plan make_plan_uncached(int64_t B, int64_t H, int64_t N, int64_t d, int64
     // a sequence's chunk states itself.
     const bool one_wave = p.tc && !causal && !is_bwd;
     const int64_t target = (one_wave ? 1 : 2) * (int64_t)std::max(sms, 1);
-    int64_t C = one_wave ? std::max<int64_t>(1, target / std::max<int64_t>(BH, 1))
-                         : std::max<int64_t>(1, (target + BH - 1) / std::max<int64_t>(BH, 1));
+    int64_t C = one_wave ? std::max<int64_t>(1, target / std::max<int64_t>(BHu, 1))
+                         : std::max<int64_t>(1, (target + BHu - 1) / std::max<int64_t>(BHu, 1));
     C = std::min<int64_t>(C, std::max<int64_t>(1, T / 4));
     L = ((T + C - 1) / C) * block;
   }
@@ -184,7 +192,8 @@ static Plan make_plan_uncached(int64_t B, int64_t H, int64_t N, int64_t d, int64
   p.L = L;
   p.C = std::max<int64_t>(1, (N + L - 1) / L);
   p.need_states = (p.C > 1) || !causal;
-  const size_t one = (size_t)BH * (size_t)p.C * state_bytes;
+  // chunk states belong to K/V sequences (shared by a group's query heads)
+  const size_t one = (size_t)BHkv * (size_t)p.C * state_bytes;
   p.ws_bytes = p.need_states ? one * (is_bwd ? 2 : 1) : 0;
   if (p.tc && causal && is_bwd) {
     // Workspace: [U chunk states | K^T V chunk states or the dQ pass's range
@@ -201,28 +210,30 @@ static Plan make_plan_uncached(int64_t B, int64_t H, int64_t N, int64_t d, int64
 // Plans are pure functions of the arguments, the split override and the SM
 // count; the range split is a small search, so recent plans are kept.
 struct PlanKey {
-  int64_t B, H, N, d, dv, chunk_len;
+  int64_t B, H, Hkv, N, d, dv, chunk_len;
   int causal, block, dt, is_bwd, sms;
   bool operator==(const PlanKey& o) const {
-    return B == o.B && H == o.H && N == o.N && d == o.d && dv == o.dv && chunk_len == o.chunk_len &&
-           causal == o.causal && block == o.block && dt == o.dt && is_bwd == o.is_bwd && sms == o.sms;
+    return B == o.B && H == o.H && Hkv == o.Hkv && N == o.N && d == o.d && dv == o.dv &&
+           chunk_len == o.chunk_len && causal == o.causal && block == o.block && dt == o.dt &&
+           is_bwd == o.is_bwd && sms == o.sms;
   }
 };
 
 static Plan make_plan(int64_t B, int64_t H, int64_t N, int64_t d, int64_t dv, int causal, int block,
-                      la2_dtype dt, bool is_bwd, int sms) {
+                      la2_dtype dt, bool is_bwd, int sms, int64_t Hkv = -1) {
+  if (Hkv < 0) Hkv = H;
   constexpr int kSlots = 16;
   static PlanKey keys[kSlots];
   static Plan plans[kSlots];
   static int used = 0, next_slot = 0;
   static std::mutex mu;
-  const PlanKey k{B, H, N, d, dv, g_chunk_len, causal, block, static_cast<int>(dt), is_bwd ? 1 : 0, sms};
+  const PlanKey k{B, H, Hkv, N, d, dv, g_chunk_len, causal, block, static_cast<int>(dt), is_bwd ? 1 : 0, sms};
   {
     std::lock_guard<std::mutex> lock(mu);
     for (int i = 0; i < used; ++i)
       if (keys[i] == k) return plans[i];
   }
-  Plan p = make_plan_uncached(B, H, N, d, dv, causal, block, dt, is_bwd, sms);
+  Plan p = make_plan_uncached(B, H, Hkv, N, d, dv, causal, block, dt, is_bwd, sms);
   std::lock_guard<std::mutex> lock(mu);
   keys[next_slot] = k;
   plans[next_slot] = p;
@@ -238,18 +249,27 @@ static la2_status launch_status() {
   return e == cudaSuccess ? LA2_OK : LA2_ERR_CUDA;
 }
 
+// Query and K/V head counts of a call: H query heads per batch entry, G query
+// heads per K/V head (G = 1 for the plain layout).
+struct Heads {
+  int64_t BH;    // query sequences
+  int64_t BHkv;  // K/V sequences
+  int32_t H, G;
+};
+
 template <typename T>
-static la2_status run_chunk_states(const void* a, const void* b, float* out, int64_t BH, int64_t N,
-                                   int da, int db, const Plan& p, cudaStream_t st) {
+static la2_status run_chunk_states(const void* a, const void* b, float* out, int64_t nseq, int64_t N,
+                                   int da, int db, const Plan& p, cudaStream_t st, int32_t H = 1,
+                                   int32_t G = 1, int group = 1) {
   const size_t smem = chunk_state_smem(da, db);
   LaunchTimer t(K_CHUNK_STATE, st);
-  chunk_state_kernel<T><<<(unsigned)(BH * p.C), kSimtThreads, smem, st>>>(
-      static_cast<const T*>(a), static_cast<const T*>(b), out, N, da, db, p.L, p.C);
+  chunk_state_kernel<T><<<(unsigned)(nseq * p.C), kSimtThreads, smem, st>>>(
+      static_cast<const T*>(a), static_cast<const T*>(b), out, N, da, db, p.L, p.C, H, G, group);
   return launch_status();
 }
 
-static la2_status run_scan(float* s, int64_t BH, int nel, const Plan& p, int mode, cudaStream_t st) {
-  dim3 grid((nel + kSimtThreads - 1) / kSimtThreads, (unsigned)BH);
+static la2_status run_scan(float* s, int64_t nseq, int nel, const Plan& p, int mode, cudaStream_t st) {
+  dim3 grid((nel + kSimtThreads - 1) / kSimtThreads, (unsigned)nseq);
   LaunchTimer t(K_CHUNK_SCAN, st);
   if (launch_pdl(chunk_scan_kernel, grid, dim3(kSimtThreads), 0, st, s, p.C, nel, mode) != cudaSuccess)
     return LA2_ERR_CUDA;
@@ -257,7 +277,7 @@ static la2_status run_scan(float* s, int64_t BH, int nel, const Plan& p, int mod
 }
 
 template <typename T>
-static la2_status forward_simt(const void* q, const void* k, const void* v, void* o, int64_t BH,
+static la2_status forward_simt(const void* q, const void* k, const void* v, void* o, const Heads& hd,
                                int64_t N, int d, int dv, int causal, int block, float* states,
                                const Plan& p, cudaStream_t st) {
   const size_t smem = fwd_simt_smem(d, dv, block, sizeof(T));
@@ -265,15 +285,15 @@ static la2_status forward_simt(const void* q, const void* k, const void* v, void
                            (int)smem) != cudaSuccess)
     return LA2_ERR_CUDA;
   LaunchTimer t(K_FWD_SIMT, st);
-  fwd_simt_kernel<T><<<(unsigned)(BH * p.C), kSimtThreads, smem, st>>>(
+  fwd_simt_kernel<T><<<(unsigned)(hd.BH * p.C), kSimtThreads, smem, st>>>(
       static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v),
-      static_cast<T*>(o), states, N, d, dv, block, p.L, p.C, causal);
+      static_cast<T*>(o), states, N, d, dv, block, p.L, p.C, causal, hd.H, hd.G);
   return launch_status();
 }
 
 template <typename T>
 static la2_status backward_simt(const void* q, const void* k, const void* v, const void* dout,
-                                void* dq, void* dk, void* dvv, int64_t BH, int64_t N, int d,
+                                void* dq, void* dk, void* dvv, const Heads& hd, int64_t N, int d,
                                 int dv, int causal, int block, float* s_kv, float* s_u,
                                 const Plan& p, cudaStream_t st) {
   const size_t smem_q = bwd_dq_simt_smem(d, dv, block, sizeof(T));
@@ -285,18 +305,18 @@ static la2_status backward_simt(const void* q, const void* k, const void* v, con
     return LA2_ERR_CUDA;
   {
     LaunchTimer t(K_BWD_DQ_SIMT, st);
-    bwd_dq_simt_kernel<T><<<(unsigned)(BH * p.C), kSimtThreads, smem_q, st>>>(
+    bwd_dq_simt_kernel<T><<<(unsigned)(hd.BH * p.C), kSimtThreads, smem_q, st>>>(
         static_cast<const T*>(k), static_cast<const T*>(v), static_cast<const T*>(dout),
-        static_cast<T*>(dq), s_kv, N, d, dv, block, p.L, p.C, causal);
+        static_cast<T*>(dq), s_kv, N, d, dv, block, p.L, p.C, causal, hd.H, hd.G);
   }
   la2_status s = launch_status();
   if (s != LA2_OK) return s;
   {
     LaunchTimer t(K_BWD_DKDV_SIMT, st);
-    bwd_dkdv_simt_kernel<T><<<(unsigned)(BH * p.C), kSimtThreads, smem_kv, st>>>(
+    bwd_dkdv_simt_kernel<T><<<(unsigned)(hd.BHkv * p.C), kSimtThreads, smem_kv, st>>>(
         static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v),
         static_cast<const T*>(dout), static_cast<T*>(dk), static_cast<T*>(dvv), s_u, N, d, dv,
-        block, p.L, p.C, causal);
+        block, p.L, p.C, causal, hd.H, hd.G);
   }
   return launch_status();
 }
@@ -306,27 +326,30 @@ static la2_status backward_simt(const void* q, const void* k, const void* v, con
 // starts inside a sequence gets its initial state from a pre-pass over the
 // sequence's earlier blocks or from the range states of a separate pass.
 // Also the dQ pass of the backward, with (dO, V, K) in the (Q, K, V) slots.
+// The K and V slots hold hd.BHkv sequences, read through the head map.
 template <int BK>
 static la2_status causal_range_split(const void* q, const void* k, const void* v, void* o,
-                                     int64_t BH, int64_t N, float* range_states,
+                                     const Heads& hd, int64_t N, float* range_states,
                                      const RangePlan& rp, int64_t spin, cudaStream_t st,
                                      int kid_states, int kid_main) {
   constexpr int D = 128, DV = 128;
   CUtensorMap tq, tk, tv;
-  if (!make_tmap_3d(&tq, q, BH, N, D, BK) || !make_tmap_3d(&tk, k, BH, N, D, BK) ||
-      !make_tmap_3d(&tv, v, BH, N, DV, BK))
+  if (!make_tmap_3d(&tq, q, hd.BH, N, D, BK) || !make_tmap_3d(&tk, k, hd.BHkv, N, D, BK) ||
+      !make_tmap_3d(&tv, v, hd.BHkv, N, DV, BK))
     return LA2_ERR_CUDA;
   sm100::RangeTable rt;
   if (!fill_range_table(rp, &rt)) return LA2_ERR_UNSUPPORTED;
   // O tiles leave through per-warp TMA stores of 16 rows at Bk=64.
   CUtensorMap to = tq;
-  if (sm100::CCfg<BK, D, DV>::TMA_STORE && !make_tmap_3d(&to, o, BH, N, DV, 16))
+  if (sm100::CCfg<BK, D, DV>::TMA_STORE && !make_tmap_3d(&to, o, hd.BH, N, DV, 16))
     return LA2_ERR_CUDA;
   sm100::CausalParams cp{};
   cp.o = static_cast<__nv_bfloat16*>(o);
   cp.agg = range_states;
   cp.N = N;
   cp.spin_limit = spin;
+  cp.H = hd.H;
+  cp.G = hd.G;
   const int sms = device_sm_count();
   const int grid = std::max(1, std::min(rp.R, sms));
   if (rp.prefix_mode == 1) {
@@ -342,18 +365,39 @@ static la2_status causal_range_split(const void* q, const void* k, const void* v
 // the map pass (no scan launch); more are scanned into slot 0 first.
 constexpr int64_t kSumInKernel = 8;
 
-// Tensor-core forward. Causal: the range split above. Non-causal: chunk
-// states, their total, then every block against the total state.
+// K^T V chunk states of every K/V sequence (MODE_STATE, one unit per K/V
+// sequence and chunk; tk and tv hold hd.BHkv sequences).
+template <int BK>
+static la2_status kv_chunk_states(const CUtensorMap& tk, const CUtensorMap& tv, float* states,
+                                  const Heads& hd, int64_t N, const Plan& p, int64_t spin,
+                                  cudaStream_t st) {
+  sm100::Params ps{};
+  ps.N = N;
+  ps.L = p.L;
+  ps.C = p.C;
+  ps.units_per_seq = p.C;
+  ps.out_states = states;
+  ps.spin_limit = spin;
+  ps.H = hd.H;
+  ps.G = hd.G;
+  ps.state_group = 1;
+  LaunchTimer t(K_STATE_TC, st);
+  return launch_fwd_sm100<BK, 128, 128, sm100::MODE_STATE>(tk, tk, tv, tk, ps, hd.BHkv * p.C, st);
+}
+
+// Tensor-core forward. Causal: the range split above (or, for splits the
+// range table cannot hold, chunk states, their prefix, and the chunk loops).
+// Non-causal: chunk states, their total, then every block against the total.
 template <int BK>
 static la2_status forward_sm100_bk(const void* q, const void* k, const void* v, void* o,
-                                   int64_t BH, int64_t N, int causal, float* states,
+                                   const Heads& hd, int64_t N, int causal, float* states,
                                    const Plan& p, int64_t spin, cudaStream_t st) {
   if (causal && p.ranges)
-    return causal_range_split<BK>(q, k, v, o, BH, N, states, p.rp, spin, st, K_STATE_TC, K_FWD_TC);
+    return causal_range_split<BK>(q, k, v, o, hd, N, states, p.rp, spin, st, K_STATE_TC, K_FWD_TC);
   constexpr int D = 128, DV = 128;
   CUtensorMap tq, tk, tv;
-  if (!make_tmap_3d(&tq, q, BH, N, D, BK) || !make_tmap_3d(&tk, k, BH, N, D, BK) ||
-      !make_tmap_3d(&tv, v, BH, N, DV, BK))
+  if (!make_tmap_3d(&tq, q, hd.BH, N, D, BK) || !make_tmap_3d(&tk, k, hd.BHkv, N, D, BK) ||
+      !make_tmap_3d(&tv, v, hd.BHkv, N, DV, BK))
     return LA2_ERR_CUDA;
   sm100::Params prm{};
   prm.o = static_cast<__nv_bfloat16*>(o);
@@ -361,62 +405,84 @@ static la2_status forward_sm100_bk(const void* q, const void* k, const void* v, 
   prm.L = p.L;
   prm.C = p.C;
   prm.spin_limit = spin;
+  prm.H = hd.H;
+  prm.G = hd.G;
+  prm.state_group = 1;
   la2_status s = LA2_OK;
   const int nel = D * DV;
   CUtensorMap to_c = tq;
-  if (sm100::Cfg<BK, D, DV>::TMA_STORE && !make_tmap_3d(&to_c, o, BH, N, DV, 16)) return LA2_ERR_CUDA;
+  if (sm100::Cfg<BK, D, DV>::TMA_STORE && !make_tmap_3d(&to_c, o, hd.BH, N, DV, 16)) return LA2_ERR_CUDA;
   if (causal) {
     // A split the range table cannot hold: chunk states, their exclusive
     // prefix per sequence, then every chunk's block loop from its prefix.
     if (p.need_states) {
-      sm100::Params ps = prm;
-      ps.out_states = states;
-      ps.units_per_seq = p.C;
-      {
-        LaunchTimer t(K_STATE_TC, st);
-        s = launch_fwd_sm100<BK, D, DV, sm100::MODE_STATE>(tq, tk, tv, tq, ps, BH * p.C, st);
-      }
+      s = kv_chunk_states<BK>(tk, tv, states, hd, N, p, spin, st);
       if (s != LA2_OK) return s;
-      s = run_scan(states, BH, nel, p, 0, st);
+      s = run_scan(states, hd.BHkv, nel, p, 0, st);
       if (s != LA2_OK) return s;
     }
     prm.init_states = p.need_states ? states : nullptr;
     prm.units_per_seq = p.C;
     LaunchTimer t(K_FWD_TC, st);
-    return launch_fwd_sm100<BK, D, DV, sm100::MODE_CAUSAL>(tq, tk, tv, to_c, prm, BH * p.C, st);
+    return launch_fwd_sm100<BK, D, DV, sm100::MODE_CAUSAL>(tq, tk, tv, to_c, prm, hd.BH * p.C, st);
   }
-  sm100::Params ps = prm;
-  ps.out_states = states;
-  ps.units_per_seq = p.C;
-  {
-    LaunchTimer t(K_STATE_TC, st);
-    s = launch_fwd_sm100<BK, D, DV, sm100::MODE_STATE>(tq, tk, tv, tq, ps, BH * p.C, st);
-  }
+  s = kv_chunk_states<BK>(tk, tv, states, hd, N, p, spin, st);
   if (s != LA2_OK) return s;
   // A few chunk states: the map pass adds them up itself; many: scan first.
   prm.init_count = p.C <= kSumInKernel ? p.C : 1;
   if (p.C > kSumInKernel) {
-    s = run_scan(states, BH, nel, p, 2, st);
+    s = run_scan(states, hd.BHkv, nel, p, 2, st);
     if (s != LA2_OK) return s;
   }
   prm.init_states = states;
   prm.units_per_seq = p.C;
   LaunchTimer t(K_FWD_TC, st);
-  return launch_fwd_sm100<BK, D, DV, sm100::MODE_NONCAUSAL>(tq, tk, tv, to_c, prm, BH * p.C, st);
+  return launch_fwd_sm100<BK, D, DV, sm100::MODE_NONCAUSAL>(tq, tk, tv, to_c, prm, hd.BH * p.C, st);
+}
+
+// The dK/dV pass: one unit per K/V sequence and chunk, reverse block order,
+// the group's query heads walked per block (tiles of TB rows).
+template <int TB>
+static la2_status dkdv_sm100(const void* q, const void* k, const void* v, const void* dout, void* dk,
+                             void* dvv, const Heads& hd, int64_t N, int causal, const float* s_u,
+                             const Plan& p, int64_t spin, cudaStream_t st) {
+  constexpr int D = 128, DV = 128;
+  CUtensorMap tq, tk, tv, tdo;
+  if (!make_tmap_3d(&tq, q, hd.BH, N, D, TB) || !make_tmap_3d(&tk, k, hd.BHkv, N, D, TB) ||
+      !make_tmap_3d(&tv, v, hd.BHkv, N, DV, TB) || !make_tmap_3d(&tdo, dout, hd.BH, N, DV, TB))
+    return LA2_ERR_CUDA;
+  sm100::BwdParams pb{};
+  pb.dk = static_cast<__nv_bfloat16*>(dk);
+  pb.dv = static_cast<__nv_bfloat16*>(dvv);
+  pb.init_u = s_u;
+  pb.N = N;
+  pb.L = p.L;
+  pb.C = p.C;
+  pb.spin_limit = spin;
+  pb.causal = causal;
+  pb.H = hd.H;
+  pb.G = hd.G;
+  CUtensorMap tdk = tq, tdv = tq;
+  if (sm100::BCfg<TB, D, DV>::TMA_STORE &&
+      (!make_tmap_3d(&tdk, dk, hd.BHkv, N, D, 16) || !make_tmap_3d(&tdv, dvv, hd.BHkv, N, DV, 16)))
+    return LA2_ERR_CUDA;
+  LaunchTimer t(K_BWD_DKDV_TC, st);
+  return launch_bwd_dkdv_sm100<TB>(tq, tk, tv, tdo, tdk, tdv, pb, hd.BHkv * p.C, st);
 }
 
 // Tensor-core backward: chunk states K^T V (prefix for dQ) and Q^T dO
-// (suffix for dK, dV), their scans, then the dQ pass (the block loop with
-// dO, V, K in the Q, K, V slots) and the reverse dK/dV pass.
+// (suffix for dK, dV; summed over a group's query heads), their scans, then
+// the dQ pass (the block loop with dO, V, K in the Q, K, V slots) and the
+// reverse dK/dV pass.
 template <int BK>
 static la2_status backward_sm100_bk(const void* q, const void* k, const void* v, const void* dout,
-                                    void* dq, void* dk, void* dvv, int64_t BH, int64_t N,
+                                    void* dq, void* dk, void* dvv, const Heads& hd, int64_t N,
                                     int causal, float* s_kv, float* s_u, const Plan& p,
                                     int64_t spin, cudaStream_t st) {
   constexpr int D = 128, DV = 128;
   CUtensorMap tq, tk, tv, tdo;
-  if (!make_tmap_3d(&tq, q, BH, N, D, BK) || !make_tmap_3d(&tk, k, BH, N, D, BK) ||
-      !make_tmap_3d(&tv, v, BH, N, DV, BK) || !make_tmap_3d(&tdo, dout, BH, N, DV, BK))
+  if (!make_tmap_3d(&tq, q, hd.BH, N, D, BK) || !make_tmap_3d(&tk, k, hd.BHkv, N, D, BK) ||
+      !make_tmap_3d(&tv, v, hd.BHkv, N, DV, BK) || !make_tmap_3d(&tdo, dout, hd.BH, N, DV, BK))
     return LA2_ERR_CUDA;
   la2_status s = LA2_OK;
   const int nel = D * DV;
@@ -424,33 +490,35 @@ static la2_status backward_sm100_bk(const void* q, const void* k, const void* v,
   const bool dq_split = causal && p.dq_ranges;
   if (dq_split) {
     // dQ = ((dO V^T) ⊙ M) K: the causal forward with (dO, V, K) as (Q, K, V).
-    s = causal_range_split<BK>(dout, v, k, dq, BH, N, s_kv, p.rp, spin, st, K_STATE_TC, K_BWD_DQ_TC);
+    s = causal_range_split<BK>(dout, v, k, dq, hd, N, s_kv, p.rp, spin, st, K_STATE_TC, K_BWD_DQ_TC);
     if (s != LA2_OK) return s;
   }
   if (states) {
-    sm100::Params ps{};
-    ps.N = N;
-    ps.L = p.L;
-    ps.C = p.C;
-    ps.units_per_seq = p.C;
-    ps.spin_limit = spin;
     if (!dq_split) {
-      LaunchTimer t(K_STATE_TC, st);
-      ps.out_states = s_kv;  // K^T V per chunk
-      s = launch_fwd_sm100<BK, D, DV, sm100::MODE_STATE>(tq, tk, tv, tq, ps, BH * p.C, st);
+      s = kv_chunk_states<BK>(tk, tv, s_kv, hd, N, p, spin, st);  // K^T V per chunk
+      if (s != LA2_OK) return s;
     }
-    if (s != LA2_OK) return s;
     {
+      // Q^T dO per chunk of each K/V sequence, summed over its group's query heads
+      sm100::Params ps{};
+      ps.N = N;
+      ps.L = p.L;
+      ps.C = p.C;
+      ps.units_per_seq = p.C;
+      ps.spin_limit = spin;
+      ps.out_states = s_u;
+      ps.H = hd.H;
+      ps.G = hd.G;
+      ps.state_group = hd.G;
       LaunchTimer t(K_STATE_TC, st);
-      ps.out_states = s_u;  // Q^T dO per chunk
-      s = launch_fwd_sm100<BK, D, DV, sm100::MODE_STATE>(tq, tq, tdo, tq, ps, BH * p.C, st);
+      s = launch_fwd_sm100<BK, D, DV, sm100::MODE_STATE>(tq, tq, tdo, tq, ps, hd.BHkv * p.C, st);
     }
     if (s != LA2_OK) return s;
     if (!dq_split && (causal || p.C > kSumInKernel)) {
-      s = run_scan(s_kv, BH, nel, p, causal ? 0 : 2, st);
+      s = run_scan(s_kv, hd.BHkv, nel, p, causal ? 0 : 2, st);
       if (s != LA2_OK) return s;
     }
-    s = run_scan(s_u, BH, nel, p, causal ? 1 : 2, st);
+    s = run_scan(s_u, hd.BHkv, nel, p, causal ? 1 : 2, st);
     if (s != LA2_OK) return s;
   }
   // Otherwise (non-causal, or a forced split beyond the range table) the
@@ -465,39 +533,32 @@ static la2_status backward_sm100_bk(const void* q, const void* k, const void* v,
     pq.units_per_seq = p.C;
     pq.init_count = p.C <= kSumInKernel ? p.C : 1;  // non-causal dQ: summed here or scanned
     pq.spin_limit = spin;
+    pq.H = hd.H;
+    pq.G = hd.G;
+    pq.state_group = 1;
     CUtensorMap tdq = tq;
-    if (sm100::Cfg<BK, D, DV>::TMA_STORE && !make_tmap_3d(&tdq, dq, BH, N, D, 16)) return LA2_ERR_CUDA;
+    if (sm100::Cfg<BK, D, DV>::TMA_STORE && !make_tmap_3d(&tdq, dq, hd.BH, N, D, 16)) return LA2_ERR_CUDA;
     {
       LaunchTimer t(K_BWD_DQ_TC, st);
       s = causal
-              ? launch_fwd_sm100<BK, D, DV, sm100::MODE_CAUSAL, true>(tdo, tv, tk, tdq, pq, BH * p.C, st)
-              : launch_fwd_sm100<BK, D, DV, sm100::MODE_NONCAUSAL, true>(tdo, tv, tk, tdq, pq, BH * p.C,
-                                                                        st);
+              ? launch_fwd_sm100<BK, D, DV, sm100::MODE_CAUSAL, true>(tdo, tv, tk, tdq, pq, hd.BH * p.C, st)
+              : launch_fwd_sm100<BK, D, DV, sm100::MODE_NONCAUSAL, true>(tdo, tv, tk, tdq, pq,
+                                                                        hd.BH * p.C, st);
     }
     if (s != LA2_OK) return s;
   }
-  sm100::BwdParams pb{};
-  pb.dk = static_cast<__nv_bfloat16*>(dk);
-  pb.dv = static_cast<__nv_bfloat16*>(dvv);
-  pb.init_u = states ? s_u : nullptr;
-  pb.N = N;
-  pb.L = p.L;
-  pb.C = p.C;
-  pb.spin_limit = spin;
-  pb.causal = causal;
-  CUtensorMap tdk = tq, tdv = tq;
-  if (sm100::BCfg<BK, D, DV>::TMA_STORE &&
-      (!make_tmap_3d(&tdk, dk, BH, N, D, 16) || !make_tmap_3d(&tdv, dvv, BH, N, DV, 16)))
-    return LA2_ERR_CUDA;
-  LaunchTimer t(K_BWD_DKDV_TC, st);
-  return launch_bwd_dkdv_sm100<BK>(tq, tk, tv, tdo, tdk, tdv, pb, BH * p.C, st);
+  // A group of query heads accumulates into one dK, dV: the scores of each
+  // head need their own TMEM columns, which 64-row tiles leave free.
+  if (hd.G > 1 && BK == 128 && causal)
+    return dkdv_sm100<64>(q, k, v, dout, dk, dvv, hd, N, causal, states ? s_u : nullptr, p, spin, st);
+  return dkdv_sm100<BK>(q, k, v, dout, dk, dvv, hd, N, causal, states ? s_u : nullptr, p, spin, st);
 }
 
-static la2_status forward_sm100(const void* q, const void* k, const void* v, void* o, int64_t BH,
+static la2_status forward_sm100(const void* q, const void* k, const void* v, void* o, const Heads& hd,
                                 int64_t N, int causal, int block, float* states, const Plan& p,
                                 int64_t spin, cudaStream_t st) {
-  return block == 64 ? forward_sm100_bk<64>(q, k, v, o, BH, N, causal, states, p, spin, st)
-                     : forward_sm100_bk<128>(q, k, v, o, BH, N, causal, states, p, spin, st);
+  return block == 64 ? forward_sm100_bk<64>(q, k, v, o, hd, N, causal, states, p, spin, st)
+                     : forward_sm100_bk<128>(q, k, v, o, hd, N, causal, states, p, spin, st);
 }
 
 }  // namespace la2
@@ -508,13 +569,18 @@ using namespace la2;
 
 extern "C" {
 
-size_t la2_workspace_size(int64_t B, int64_t H, int64_t N, int64_t d, int64_t dv, int causal,
-                          int block, la2_dtype dt, int is_backward) {
-  if (check_shape(B, H, N, d, dv, causal, block, dt, is_backward != 0) != LA2_OK) return (size_t)-1;
+size_t la2_workspace_size_gqa(int64_t B, int64_t H, int64_t Hkv, int64_t N, int64_t d, int64_t dv,
+                              int causal, int block, la2_dtype dt, int is_backward) {
+  if (check_shape(B, H, N, d, dv, causal, block, dt, is_backward != 0, Hkv) != LA2_OK) return (size_t)-1;
   if (B == 0 || H == 0 || N == 0) return 0;
   const int sms = device_sm_count();
   if (sms <= 0) return (size_t)-1;
-  return make_plan(B, H, N, d, dv, causal, block, dt, is_backward != 0, sms).ws_bytes;
+  return make_plan(B, H, N, d, dv, causal, block, dt, is_backward != 0, sms, Hkv).ws_bytes;
+}
+
+size_t la2_workspace_size(int64_t B, int64_t H, int64_t N, int64_t d, int64_t dv, int causal,
+                          int block, la2_dtype dt, int is_backward) {
+  return la2_workspace_size_gqa(B, H, H, N, d, dv, causal, block, dt, is_backward);
 }
 
 int64_t la2_plan_ranges(int64_t B, int64_t H, int64_t N, int64_t d, int64_t dv, int causal,
@@ -594,6 +660,9 @@ la2_status la2_kv_state(const void* k, const void* v, float* state, int64_t B, i
     ps.units_per_seq = p.C;
     ps.out_states = chunks;
     ps.spin_limit = spin_limit();
+    ps.H = 1;
+    ps.G = 1;
+    ps.state_group = 1;
     LaunchTimer t(K_STATE_TC, st);
     s = launch_fwd_sm100<64, 128, 128, sm100::MODE_STATE>(tk, tk, tv, tk, ps, BH * p.C, st);
   } else {
@@ -663,52 +732,61 @@ la2_status la2_decode_step(const void* q, const void* k, const void* v, void* o,
   return launch_status();
 }
 
-la2_status la2_forward(const void* q, const void* k, const void* v, void* o, int64_t B, int64_t H,
-                       int64_t N, int64_t d, int64_t dv, int causal, int block, la2_dtype dt,
-                       void* workspace, size_t workspace_bytes, la2_stream_t stream) {
-  la2_status s = check_shape(B, H, N, d, dv, causal, block, dt, false);
+la2_status la2_forward_gqa(const void* q, const void* k, const void* v, void* o, int64_t B,
+                           int64_t H, int64_t Hkv, int64_t N, int64_t d, int64_t dv, int causal,
+                           int block, la2_dtype dt, void* workspace, size_t workspace_bytes,
+                           la2_stream_t stream) {
+  la2_status s = check_shape(B, H, N, d, dv, causal, block, dt, false, Hkv);
   if (s != LA2_OK) return s;
   if (B == 0 || H == 0 || N == 0) return LA2_OK;
   if (!q || !k || !v || !o) return LA2_ERR_INVALID_ARG;
   if (!is_aligned(q, 16) || !is_aligned(k, 16) || !is_aligned(v, 16) || !is_aligned(o, 16))
     return LA2_ERR_INVALID_ARG;
   const size_t es = dt == LA2_BF16 ? 2 : 4;
-  const size_t nq = (size_t)B * H * N * d * es, nv = (size_t)B * H * N * dv * es;
-  if (overlaps(o, nv, q, nq) || overlaps(o, nv, k, nq) || overlaps(o, nv, v, nv))
+  const size_t nq = (size_t)B * H * N * d * es, no = (size_t)B * H * N * dv * es;
+  const size_t nk = (size_t)B * Hkv * N * d * es, nv = (size_t)B * Hkv * N * dv * es;
+  if (overlaps(o, no, q, nq) || overlaps(o, no, k, nk) || overlaps(o, no, v, nv))
     return LA2_ERR_INVALID_ARG;
   const int sms = device_sm_count();
   if (sms <= 0) return LA2_ERR_CUDA;
-  const Plan p = make_plan(B, H, N, d, dv, causal, block, dt, false, sms);
+  const Plan p = make_plan(B, H, N, d, dv, causal, block, dt, false, sms, Hkv);
+  const Heads hd{B * H, B * Hkv, static_cast<int32_t>(H), static_cast<int32_t>(H / Hkv)};
   if (p.ws_bytes > 0) {
     if (!workspace || workspace_bytes < p.ws_bytes) return LA2_ERR_WORKSPACE;
     if (!is_aligned(workspace, 256)) return LA2_ERR_INVALID_ARG;
-    if (overlaps(workspace, p.ws_bytes, o, nv)) return LA2_ERR_INVALID_ARG;
+    if (overlaps(workspace, p.ws_bytes, o, no)) return LA2_ERR_INVALID_ARG;
   }
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const int64_t BH = B * H;
   float* states = p.need_states ? static_cast<float*>(workspace) : nullptr;
   const int nel = (int)(d * dv);
-  if (p.tc) return forward_sm100(q, k, v, o, BH, N, causal, block, states, p, spin_limit(), st);
-  if (p.need_states) {
+  if (p.tc) return forward_sm100(q, k, v, o, hd, N, causal, block, states, p, spin_limit(), st);
+  if (p.need_states) {  // K^T V chunk states of the K/V sequences, then their prefix / total
     s = dt == LA2_BF16
-            ? run_chunk_states<__nv_bfloat16>(k, v, states, BH, N, (int)d, (int)dv, p, st)
-            : run_chunk_states<float>(k, v, states, BH, N, (int)d, (int)dv, p, st);
+            ? run_chunk_states<__nv_bfloat16>(k, v, states, hd.BHkv, N, (int)d, (int)dv, p, st)
+            : run_chunk_states<float>(k, v, states, hd.BHkv, N, (int)d, (int)dv, p, st);
     if (s != LA2_OK) return s;
-    s = run_scan(states, BH, nel, p, causal ? 0 : 2, st);
+    s = run_scan(states, hd.BHkv, nel, p, causal ? 0 : 2, st);
     if (s != LA2_OK) return s;
   }
   return dt == LA2_BF16
-             ? forward_simt<__nv_bfloat16>(q, k, v, o, BH, N, (int)d, (int)dv, causal, block,
+             ? forward_simt<__nv_bfloat16>(q, k, v, o, hd, N, (int)d, (int)dv, causal, block,
                                            states, p, st)
-             : forward_simt<float>(q, k, v, o, BH, N, (int)d, (int)dv, causal, block, states, p,
+             : forward_simt<float>(q, k, v, o, hd, N, (int)d, (int)dv, causal, block, states, p,
                                    st);
 }
 
-la2_status la2_backward(const void* q, const void* k, const void* v, const void* dout, void* dq,
-                        void* dk, void* dvv, int64_t B, int64_t H, int64_t N, int64_t d,
-                        int64_t dv, int causal, int block, la2_dtype dt, void* workspace,
-                        size_t workspace_bytes, la2_stream_t stream) {
-  la2_status s = check_shape(B, H, N, d, dv, causal, block, dt, true);
+la2_status la2_forward(const void* q, const void* k, const void* v, void* o, int64_t B, int64_t H,
+                       int64_t N, int64_t d, int64_t dv, int causal, int block, la2_dtype dt,
+                       void* workspace, size_t workspace_bytes, la2_stream_t stream) {
+  return la2_forward_gqa(q, k, v, o, B, H, H, N, d, dv, causal, block, dt, workspace,
+                         workspace_bytes, stream);
+}
+
+la2_status la2_backward_gqa(const void* q, const void* k, const void* v, const void* dout, void* dq,
+                            void* dk, void* dvv, int64_t B, int64_t H, int64_t Hkv, int64_t N,
+                            int64_t d, int64_t dv, int causal, int block, la2_dtype dt,
+                            void* workspace, size_t workspace_bytes, la2_stream_t stream) {
+  la2_status s = check_shape(B, H, N, d, dv, causal, block, dt, true, Hkv);
   if (s != LA2_OK) return s;
   if (B == 0 || H == 0 || N == 0) return LA2_OK;
   const void* ins[4] = {q, k, v, dout};
@@ -718,9 +796,10 @@ la2_status la2_backward(const void* q, const void* k, const void* v, const void*
   for (void* p : outs)
     if (!p || !is_aligned(p, 16)) return LA2_ERR_INVALID_ARG;
   const size_t es = dt == LA2_BF16 ? 2 : 4;
-  const size_t nq = (size_t)B * H * N * d * es, nv = (size_t)B * H * N * dv * es;
-  const size_t in_sz[4] = {nq, nq, nv, nv};
-  const size_t out_sz[3] = {nq, nq, nv};
+  const size_t nq = (size_t)B * H * N * d * es, nod = (size_t)B * H * N * dv * es;
+  const size_t nk = (size_t)B * Hkv * N * d * es, nv = (size_t)B * Hkv * N * dv * es;
+  const size_t in_sz[4] = {nq, nk, nv, nod};
+  const size_t out_sz[3] = {nq, nk, nv};
   for (int i = 0; i < 3; ++i) {
     for (int j = 0; j < 4; ++j)
       if (overlaps(outs[i], out_sz[i], ins[j], in_sz[j])) return LA2_ERR_INVALID_ARG;
@@ -729,7 +808,7 @@ la2_status la2_backward(const void* q, const void* k, const void* v, const void*
   }
   const int sms = device_sm_count();
   if (sms <= 0) return LA2_ERR_CUDA;
-  const Plan p = make_plan(B, H, N, d, dv, causal, block, dt, true, sms);
+  const Plan p = make_plan(B, H, N, d, dv, causal, block, dt, true, sms, Hkv);
   if (p.ws_bytes > 0) {
     if (!workspace || workspace_bytes < p.ws_bytes) return LA2_ERR_WORKSPACE;
     if (!is_aligned(workspace, 256)) return LA2_ERR_INVALID_ARG;
@@ -737,41 +816,52 @@ la2_status la2_backward(const void* q, const void* k, const void* v, const void*
       if (overlaps(workspace, p.ws_bytes, outs[i], out_sz[i])) return LA2_ERR_INVALID_ARG;
   }
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const int64_t BH = B * H;
+  const Heads hd{B * H, B * Hkv, static_cast<int32_t>(H), static_cast<int32_t>(H / Hkv)};
   const int nel = (int)(d * dv);
+  // chunk states of the K/V sequences: [K^T V | Q^T dO summed over each group]
   float* s_kv = p.need_states ? static_cast<float*>(workspace) : nullptr;
-  float* s_u = p.need_states ? s_kv + (size_t)BH * p.C * nel : nullptr;
+  float* s_u = p.need_states ? s_kv + (size_t)hd.BHkv * p.C * nel : nullptr;
   if (p.tc) {
     float* second = nullptr;  // K^T V chunk states, or the dQ pass's range states
     if (p.need_states) {
       s_u = static_cast<float*>(workspace);
-      second = s_u + (size_t)BH * p.C * nel;
+      second = s_u + (size_t)hd.BHkv * p.C * nel;
     } else if (p.ws_bytes > 0) {
       second = static_cast<float*>(workspace);
     }
-    return block == 64 ? backward_sm100_bk<64>(q, k, v, dout, dq, dk, dvv, BH, N, causal, second,
+    return block == 64 ? backward_sm100_bk<64>(q, k, v, dout, dq, dk, dvv, hd, N, causal, second,
                                                 s_u, p, spin_limit(), st)
-                       : backward_sm100_bk<128>(q, k, v, dout, dq, dk, dvv, BH, N, causal, second,
+                       : backward_sm100_bk<128>(q, k, v, dout, dq, dk, dvv, hd, N, causal, second,
                                                  s_u, p, spin_limit(), st);
   }
   if (p.need_states) {
     const bool bf = dt == LA2_BF16;
-    s = bf ? run_chunk_states<__nv_bfloat16>(k, v, s_kv, BH, N, (int)d, (int)dv, p, st)
-           : run_chunk_states<float>(k, v, s_kv, BH, N, (int)d, (int)dv, p, st);
+    s = bf ? run_chunk_states<__nv_bfloat16>(k, v, s_kv, hd.BHkv, N, (int)d, (int)dv, p, st)
+           : run_chunk_states<float>(k, v, s_kv, hd.BHkv, N, (int)d, (int)dv, p, st);
     if (s != LA2_OK) return s;
-    s = bf ? run_chunk_states<__nv_bfloat16>(q, dout, s_u, BH, N, (int)d, (int)dv, p, st)
-           : run_chunk_states<float>(q, dout, s_u, BH, N, (int)d, (int)dv, p, st);
+    s = bf ? run_chunk_states<__nv_bfloat16>(q, dout, s_u, hd.BHkv, N, (int)d, (int)dv, p, st,
+                                             hd.H, hd.G, hd.G)
+           : run_chunk_states<float>(q, dout, s_u, hd.BHkv, N, (int)d, (int)dv, p, st, hd.H, hd.G,
+                                     hd.G);
     if (s != LA2_OK) return s;
-    s = run_scan(s_kv, BH, nel, p, causal ? 0 : 2, st);
+    s = run_scan(s_kv, hd.BHkv, nel, p, causal ? 0 : 2, st);
     if (s != LA2_OK) return s;
-    s = run_scan(s_u, BH, nel, p, causal ? 1 : 2, st);
+    s = run_scan(s_u, hd.BHkv, nel, p, causal ? 1 : 2, st);
     if (s != LA2_OK) return s;
   }
   return dt == LA2_BF16
-             ? backward_simt<__nv_bfloat16>(q, k, v, dout, dq, dk, dvv, BH, N, (int)d, (int)dv,
+             ? backward_simt<__nv_bfloat16>(q, k, v, dout, dq, dk, dvv, hd, N, (int)d, (int)dv,
                                             causal, block, s_kv, s_u, p, st)
-             : backward_simt<float>(q, k, v, dout, dq, dk, dvv, BH, N, (int)d, (int)dv, causal,
+             : backward_simt<float>(q, k, v, dout, dq, dk, dvv, hd, N, (int)d, (int)dv, causal,
                                     block, s_kv, s_u, p, st);
+}
+
+la2_status la2_backward(const void* q, const void* k, const void* v, const void* dout, void* dq,
+                        void* dk, void* dvv, int64_t B, int64_t H, int64_t N, int64_t d,
+                        int64_t dv, int causal, int block, la2_dtype dt, void* workspace,
+                        size_t workspace_bytes, la2_stream_t stream) {
+  return la2_backward_gqa(q, k, v, dout, dq, dk, dvv, B, H, H, N, d, dv, causal, block, dt,
+                          workspace, workspace_bytes, stream);
 }
 
 la2_status la2_check(la2_stream_t stream) {

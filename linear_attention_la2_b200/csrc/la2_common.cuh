@@ -23,6 +23,24 @@ __device__ __forceinline__ void record_error(int code, int where) {
 
 __device__ __forceinline__ int64_t imin64(int64_t a, int64_t b) { return a < b ? a : b; }
 
+// Grouped K/V heads (GQA; MQA with one K/V head). With H query heads and
+// Hkv = H / G K/V heads, query sequence bh = b*H + h reads K/V sequence
+// b*Hkv + h/G. G = 1 is the plain layout (every query head has its own K/V).
+__host__ __device__ __forceinline__ int64_t kv_seq(int64_t bh, int32_t H, int32_t G) {
+  if (G <= 1) return bh;
+  const int64_t b = bh / H;
+  const int32_t h = static_cast<int32_t>(bh - b * H);
+  return b * (H / G) + h / G;
+}
+// First query sequence of K/V sequence `kv` (the group is kv's G consecutive heads).
+__host__ __device__ __forceinline__ int64_t q_seq0(int64_t kv, int32_t H, int32_t G) {
+  if (G <= 1) return kv;
+  const int32_t Hkv = H / G;
+  const int64_t b = kv / Hkv;
+  const int32_t j = static_cast<int32_t>(kv - b * Hkv);
+  return b * H + static_cast<int64_t>(j) * G;
+}
+
 // Programmatic dependent launch: let the next kernel of the stream start its
 // launch now (its CTAs still wait in pdl_wait for this grid), and wait until
 // the previous kernel of the stream has completed and its memory is visible.

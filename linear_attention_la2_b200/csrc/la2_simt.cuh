@@ -14,6 +14,8 @@
 // (float or bf16) are widened on load and outputs rounded to T on store.
 #pragma once
 
+#include <algorithm>
+
 #include "la2_common.cuh"
 
 namespace la2 {
@@ -24,27 +26,31 @@ constexpr int kSimtThreads = 256;
 // Chunk states: S[bh][c] = sum over rows t of chunk c of a_t^T b_t  (da x db).
 // (a, b) = (K, V) gives the KV state of a chunk; (Q, dO) gives the state the
 // dK/dV pass of the backward carries. One CTA per (bh, c); each thread keeps
-// up to 64 state elements in registers.
+// up to 64 state elements in registers. With `group` > 1, bh is a K/V
+// sequence and its state sums the chunk over the group's query sequences
+// (q_seq0(bh) + j, j < group): the summed suffix state of grouped heads.
 // ----------------------------------------------------------------------------
 constexpr int kStateRowsPerTile = 32;
 
 template <typename T>
 __global__ void __launch_bounds__(kSimtThreads)
 chunk_state_kernel(const T* __restrict__ a, const T* __restrict__ b, float* __restrict__ out,
-                   int64_t N, int da, int db, int64_t L, int64_t C) {
+                   int64_t N, int da, int db, int64_t L, int64_t C, int H, int G, int group) {
   extern __shared__ float smem[];
   float* As = smem;                              // [32][da]
   float* Bs = smem + kStateRowsPerTile * da;     // [32][db]
   const int64_t unit = blockIdx.x;
   const int64_t bh = unit / C, c = unit % C;
   const int64_t t0 = c * L, t1 = imin64(N, t0 + L);
-  const T* ab = a + bh * N * da;
-  const T* bb = b + bh * N * db;
   const int nel = da * db;
   float acc[64];
 #pragma unroll
   for (int r = 0; r < 64; ++r) acc[r] = 0.f;
 
+  for (int j = 0; j < group; ++j) {
+  const int64_t src = group > 1 ? q_seq0(bh, H, G) + j : bh;
+  const T* ab = a + src * N * da;
+  const T* bb = b + src * N * db;
   for (int64_t s0 = t0; s0 < t1; s0 += kStateRowsPerTile) {
     const int rows = (int)imin64(kStateRowsPerTile, t1 - s0);
     for (int i = threadIdx.x; i < kStateRowsPerTile * da; i += blockDim.x) {
@@ -67,6 +73,7 @@ chunk_state_kernel(const T* __restrict__ a, const T* __restrict__ b, float* __re
       }
     }
     __syncthreads();
+  }
   }
   float* o = out + (bh * C + c) * (int64_t)nel;
 #pragma unroll
@@ -145,7 +152,7 @@ template <typename T>
 __global__ void __launch_bounds__(kSimtThreads)
 fwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                 T* __restrict__ o, const float* __restrict__ states, int64_t N, int d, int dv,
-                int Bk, int64_t L, int64_t C, int causal) {
+                int Bk, int64_t L, int64_t C, int causal, int H, int G) {
   extern __shared__ float smem[];
   float* KV = smem;
   T* Qs = reinterpret_cast<T*>(KV + d * dv);
@@ -154,15 +161,16 @@ fwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
   T* S = Vs + Bk * dv;  // masked (Q K^T) block, rounded to T
   const int64_t unit = blockIdx.x;
   const int64_t bh = unit / C, c = unit % C;
+  const int64_t bkv = kv_seq(bh, H, G);  // K/V sequence (and its states)
   const int64_t t0 = c * L, t1 = imin64(N, t0 + L);
   const T* qb = q + bh * N * d;
-  const T* kb = k + bh * N * d;
-  const T* vb = v + bh * N * dv;
+  const T* kb = k + bkv * N * d;
+  const T* vb = v + bkv * N * dv;
   T* ob = o + bh * N * dv;
   const int64_t nel = (int64_t)d * dv;
   const float* init = nullptr;
-  if (!causal) init = states + bh * C * nel;           // total in slot 0
-  else if (states) init = states + (bh * C + c) * nel;  // exclusive prefix
+  if (!causal) init = states + bkv * C * nel;           // total in slot 0
+  else if (states) init = states + (bkv * C + c) * nel;  // exclusive prefix
   load_state(KV, init, (int)nel);
 
   for (int64_t i0 = t0; i0 < t1; i0 += Bk) {
@@ -214,7 +222,7 @@ template <typename T>
 __global__ void __launch_bounds__(kSimtThreads)
 bwd_dq_simt_kernel(const T* __restrict__ k, const T* __restrict__ v, const T* __restrict__ dout,
                    T* __restrict__ dq, const float* __restrict__ states, int64_t N, int d, int dv,
-                   int Bk, int64_t L, int64_t C, int causal) {
+                   int Bk, int64_t L, int64_t C, int causal, int H, int G) {
   extern __shared__ float smem[];
   float* KV = smem;
   T* dOs = reinterpret_cast<T*>(KV + d * dv);
@@ -223,15 +231,16 @@ bwd_dq_simt_kernel(const T* __restrict__ k, const T* __restrict__ v, const T* __
   T* A = Ks + Bk * d;  // masked (dO V^T) block, rounded to T
   const int64_t unit = blockIdx.x;
   const int64_t bh = unit / C, c = unit % C;
+  const int64_t bkv = kv_seq(bh, H, G);
   const int64_t t0 = c * L, t1 = imin64(N, t0 + L);
-  const T* kb = k + bh * N * d;
-  const T* vb = v + bh * N * dv;
+  const T* kb = k + bkv * N * d;
+  const T* vb = v + bkv * N * dv;
   const T* gb = dout + bh * N * dv;
   T* dqb = dq + bh * N * d;
   const int64_t nel = (int64_t)d * dv;
   const float* init = nullptr;
-  if (!causal) init = states + bh * C * nel;
-  else if (states) init = states + (bh * C + c) * nel;
+  if (!causal) init = states + bkv * C * nel;
+  else if (states) init = states + (bkv * C + c) * nel;
   load_state(KV, init, (int)nel);
 
   for (int64_t i0 = t0; i0 < t1; i0 += Bk) {
@@ -278,14 +287,35 @@ bwd_dq_simt_kernel(const T* __restrict__ k, const T* __restrict__ v, const T* __
 //   dK_i = ((dO_i V_i^T) ⊙ M_B)^T Q_i + V_i U^T
 //   dV_i = ((Q_i K_i^T) ⊙ M_B)^T dO_i + K_i U ;  U += Q_i^T dO_i
 // Non-causal: dK_i = V_i U^T, dV_i = K_i U with U = Q^T dO over the sequence.
+// One CTA per (K/V sequence, chunk). With grouped heads (G > 1) the causal
+// terms add up over the group's query heads and U sums all of them (one state
+// for the group). Each thread accumulates strips of 32 columns of one row of
+// dK_i and dV_i in registers (at most two strips of each; the host keeps
+// Bk * ceil(d / 32) and Bk * ceil(dv / 32) within 2 * kSimtThreads).
 // Shared memory: U [d][dv], Q, K [Bk][d], V, dO [Bk][dv], A, P [Bk][Bk].
 // ----------------------------------------------------------------------------
+constexpr int kStrip = 32;
+constexpr int kStripsPerThread = 2;
+
+// acc[c] (+)= sum over t in [t_lo, rows) of W[t * Bk + j] * X[t * w + c0 + c]
+template <typename T>
+__device__ __forceinline__ void strip_masked(float (&acc)[kStrip], const T* W, const T* X, int j, int c0,
+                                             int w, int rows, int Bk) {
+  for (int t = j; t < rows; ++t) {
+    const float a = to_f32(W[t * Bk + j]);
+    const T* x = X + t * w + c0;
+#pragma unroll
+    for (int c = 0; c < kStrip; ++c)
+      if (c0 + c < w) acc[c] = fmaf(a, to_f32(x[c]), acc[c]);
+  }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kSimtThreads)
 bwd_dkdv_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                      const T* __restrict__ dout, T* __restrict__ dk, T* __restrict__ dvv,
                      const float* __restrict__ states, int64_t N, int d, int dv, int Bk,
-                     int64_t L, int64_t C, int causal) {
+                     int64_t L, int64_t C, int causal, int H, int G) {
   extern __shared__ float smem[];
   float* U = smem;
   T* Qs = reinterpret_cast<T*>(U + d * dv);
@@ -295,12 +325,12 @@ bwd_dkdv_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* 
   T* A = dOs + Bk * dv;  // masked (dO V^T) block, rounded to T
   T* P = A + Bk * Bk;    // masked (Q K^T) block, rounded to T
   const int64_t unit = blockIdx.x;
-  const int64_t bh = unit / C, c = unit % C;
+  const int64_t bh = unit / C, c = unit % C;  // the K/V sequence
   const int64_t t0 = c * L, t1 = imin64(N, t0 + L);
-  const T* qb = q + bh * N * d;
+  const int64_t q0 = q_seq0(bh, H, G);
+  const int heads = causal ? G : 1;
   const T* kb = k + bh * N * d;
   const T* vb = v + bh * N * dv;
-  const T* gb = dout + bh * N * dv;
   T* dkb = dk + bh * N * d;
   T* dvb = dvv + bh * N * dv;
   const int64_t nel = (int64_t)d * dv;
@@ -308,6 +338,8 @@ bwd_dkdv_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* 
   if (!causal) init = states + bh * C * nel;
   else if (states) init = states + (bh * C + c) * nel;  // exclusive suffix
   load_state(U, init, (int)nel);
+  // strips: dK strip s = (row s / sk, columns 32 * (s % sk)), likewise dV
+  const int sk = (d + kStrip - 1) / kStrip, sv = (dv + kStrip - 1) / kStrip;
 
   const int64_t nblk = (t1 - t0 + Bk - 1) / Bk;
   for (int64_t bi = nblk - 1; bi >= 0; --bi) {
@@ -315,12 +347,46 @@ bwd_dkdv_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* 
     const int rows = (int)imin64(Bk, t1 - i0);
     load_tile(Ks, kb + i0 * d, rows, Bk, d);
     load_tile(Vs, vb + i0 * dv, rows, Bk, dv);
-    if (causal) {
-      load_tile(Qs, qb + i0 * d, rows, Bk, d);
-      load_tile(dOs, gb + i0 * dv, rows, Bk, dv);
-    }
     __syncthreads();
-    if (causal) {
+    // the later blocks' part, from U before this block's update:
+    // dK[j][cc] = sum_e V[j][e] U[cc][e],  dV[j][e] = sum_cc K[j][cc] U[cc][e]
+    float ak[kStripsPerThread][kStrip], av[kStripsPerThread][kStrip];
+#pragma unroll
+    for (int r = 0; r < kStripsPerThread; ++r) {
+      const int sid = threadIdx.x + r * kSimtThreads;
+      const int j = sid / sk, c0 = (sid % sk) * kStrip;
+#pragma unroll
+      for (int cc = 0; cc < kStrip; ++cc) ak[r][cc] = 0.f;
+      if (j < rows) {
+        for (int e = 0; e < dv; ++e) {
+          const float x = to_f32(Vs[j * dv + e]);
+#pragma unroll
+          for (int cc = 0; cc < kStrip; ++cc)
+            if (c0 + cc < d) ak[r][cc] = fmaf(x, U[(c0 + cc) * dv + e], ak[r][cc]);
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < kStripsPerThread; ++r) {
+      const int sid = threadIdx.x + r * kSimtThreads;
+      const int j = sid / sv, e0 = (sid % sv) * kStrip;
+#pragma unroll
+      for (int e = 0; e < kStrip; ++e) av[r][e] = 0.f;
+      if (j < rows) {
+        for (int cc = 0; cc < d; ++cc) {
+          const float x = to_f32(Ks[j * d + cc]);
+#pragma unroll
+          for (int e = 0; e < kStrip; ++e)
+            if (e0 + e < dv) av[r][e] = fmaf(x, U[cc * dv + e0 + e], av[r][e]);
+        }
+      }
+    }
+    for (int g = 0; causal && g < heads; ++g) {
+      const int64_t hq = q0 + g;
+      __syncthreads();  // U read above (g = 0) or Q, dO of the previous head done with
+      load_tile(Qs, q + hq * N * d + i0 * d, rows, Bk, d);
+      load_tile(dOs, dout + hq * N * dv + i0 * dv, rows, Bk, dv);
+      __syncthreads();
       for (int i = threadIdx.x; i < Bk * Bk; i += blockDim.x) {
         const int t = i / Bk, j = i % Bk;  // t: query row, j: key row
         float a = 0.f, p = 0.f;
@@ -332,34 +398,53 @@ bwd_dkdv_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* 
         P[i] = from_f32<T>(p);
       }
       __syncthreads();
-    }
-    for (int i = threadIdx.x; i < rows * d; i += blockDim.x) {
-      const int j = i / d, cc = i % d;
-      float acc = 0.f;
-      if (causal)
-        for (int t = j; t < rows; ++t) acc = fmaf(to_f32(A[t * Bk + j]), to_f32(Qs[t * d + cc]), acc);
-      for (int e = 0; e < dv; ++e) acc = fmaf(to_f32(Vs[j * dv + e]), U[cc * dv + e], acc);
-      dkb[(i0 + j) * d + cc] = from_f32<T>(acc);
-    }
-    for (int i = threadIdx.x; i < rows * dv; i += blockDim.x) {
-      const int j = i / dv, e = i % dv;
-      float acc = 0.f;
-      if (causal)
-        for (int t = j; t < rows; ++t) acc = fmaf(to_f32(P[t * Bk + j]), to_f32(dOs[t * dv + e]), acc);
-      for (int cc = 0; cc < d; ++cc) acc = fmaf(to_f32(Ks[j * d + cc]), U[cc * dv + e], acc);
-      dvb[(i0 + j) * dv + e] = from_f32<T>(acc);
-    }
-    __syncthreads();
-    if (causal) {
+      // dK[j] += sum_{t >= j} A[t][j] Q[t],  dV[j] += sum_{t >= j} P[t][j] dO[t]
+#pragma unroll
+      for (int r = 0; r < kStripsPerThread; ++r) {
+        const int sid = threadIdx.x + r * kSimtThreads;
+        const int j = sid / sk;
+        if (j < rows) strip_masked(ak[r], A, Qs, j, (sid % sk) * kStrip, d, rows, Bk);
+      }
+#pragma unroll
+      for (int r = 0; r < kStripsPerThread; ++r) {
+        const int sid = threadIdx.x + r * kSimtThreads;
+        const int j = sid / sv;
+        if (j < rows) strip_masked(av[r], P, dOs, j, (sid % sv) * kStrip, dv, rows, Bk);
+      }
       for (int i = threadIdx.x; i < d * dv; i += blockDim.x) {
         const int cc = i / dv, e = i % dv;
         float acc = U[i];
         for (int t = 0; t < rows; ++t) acc = fmaf(to_f32(Qs[t * d + cc]), to_f32(dOs[t * dv + e]), acc);
         U[i] = acc;
       }
-      __syncthreads();
     }
+#pragma unroll
+    for (int r = 0; r < kStripsPerThread; ++r) {
+      const int sid = threadIdx.x + r * kSimtThreads;
+      const int j = sid / sk, c0 = (sid % sk) * kStrip;
+      if (j < rows)
+#pragma unroll
+        for (int cc = 0; cc < kStrip; ++cc)
+          if (c0 + cc < d) dkb[(i0 + j) * d + c0 + cc] = from_f32<T>(ak[r][cc]);
+    }
+#pragma unroll
+    for (int r = 0; r < kStripsPerThread; ++r) {
+      const int sid = threadIdx.x + r * kSimtThreads;
+      const int j = sid / sv, e0 = (sid % sv) * kStrip;
+      if (j < rows)
+#pragma unroll
+        for (int e = 0; e < kStrip; ++e)
+          if (e0 + e < dv) dvb[(i0 + j) * dv + e0 + e] = from_f32<T>(av[r][e]);
+    }
+    __syncthreads();  // K, V, U settled before the next block's loads
   }
+}
+
+// Strips of 32 columns the dK/dV loop keeps per block: every one must have a
+// thread (at most kStripsPerThread each).
+inline bool bwd_dkdv_simt_fits(int d, int dv, int Bk) {
+  const int strips = Bk * ((std::max(d, dv) + kStrip - 1) / kStrip);
+  return strips <= kStripsPerThread * kSimtThreads;
 }
 
 inline size_t fwd_simt_smem(int d, int dv, int Bk, size_t es) {

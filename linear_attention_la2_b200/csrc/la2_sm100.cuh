@@ -318,6 +318,14 @@ struct Params {
   int64_t C;                  // chunks per sequence
   int64_t units_per_seq;      // C (forward) or the number of chunks whose state is needed
   int64_t spin_limit;
+  // Grouped K/V heads: query heads per batch and query heads per K/V head.
+  // Block loops (MODE_CAUSAL, MODE_NONCAUSAL) run one unit per query sequence
+  // and read K, V and the initial states of its K/V sequence (kv_seq).
+  // MODE_STATE runs one unit per state sequence; with state_group > 1 that is
+  // a K/V sequence whose state sums the tiles of its group's state_group query
+  // sequences (the K and V slots then hold Q and dO: the dK/dV pass's U).
+  int32_t H, G;
+  int32_t state_group;
 };
 
 // Shared state of one CTA.
@@ -446,10 +454,14 @@ la2_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   const int64_t t0 = c * prm.L;
   const int64_t t1 = min(prm.N, t0 + prm.L);
   const int nblk = static_cast<int>((t1 - t0 + BK - 1) / BK);
+  // K/V sequence of this unit's loads (a state unit is its own sequence)
+  const int64_t bkv = MODE == MODE_STATE ? bh : kv_seq(bh, prm.H, prm.G);
+  const int sgroup = (MODE == MODE_STATE && prm.state_group > 1) ? prm.state_group : 1;
+  const int nsteps = MODE == MODE_STATE ? nblk * sgroup : nblk;
   const bool has_init = (MODE == MODE_NONCAUSAL) || (MODE == MODE_CAUSAL && prm.init_states && c > 0);
   const float* init = nullptr;
-  if (MODE == MODE_NONCAUSAL) init = prm.init_states + bh * prm.C * (int64_t)(D * DV);
-  else if (has_init) init = prm.init_states + (bh * prm.C + c) * (int64_t)(D * DV);
+  if (MODE == MODE_NONCAUSAL) init = prm.init_states + bkv * prm.C * (int64_t)(D * DV);
+  else if (has_init) init = prm.init_states + (bkv * prm.C + c) * (int64_t)(D * DV);
 
   // ---- setup
   if (threadIdx.x == 0) {
@@ -498,16 +510,21 @@ la2_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     if (lane == 0) {
       int issued_kv = 0, issued_q = 0;
       bool ok = true;
-      for (int i = 0; i < nblk && ok; ++i) {
-        const int row = static_cast<int>(t0 + static_cast<int64_t>(i) * BK);
+      for (int i = 0; i < nsteps && ok; ++i) {
+        // a state unit of a group walks the blocks of each query sequence in turn
+        const int blk = MODE == MODE_STATE ? i % nblk : i;
+        const int zkv = MODE == MODE_STATE && sgroup > 1
+                            ? static_cast<int>(q_seq0(bh, prm.H, prm.G) + i / nblk)
+                            : static_cast<int>(bkv);
+        const int row = static_cast<int>(t0 + static_cast<int64_t>(blk) * BK);
         if (MODE != MODE_NONCAUSAL) {
           const int s = i % CF::KS;
           if (!wait_bar(&b.kv_empty[s], ((i / CF::KS) & 1) ^ 1, lim, b.abort_flag, 1)) { ok = false; break; }
           mbar_expect_tx(&b.kv_full[s], CF::KTILE + CF::VTILE);
           for (int p = 0; p < CF::DP; ++p)
-            tma_load_3d(sK + s * CF::KTILE + p * BK * 128, &tm_k, &b.kv_full[s], 64 * p, row, (int)bh);
+            tma_load_3d(sK + s * CF::KTILE + p * BK * 128, &tm_k, &b.kv_full[s], 64 * p, row, zkv);
           for (int p = 0; p < CF::VP; ++p)
-            tma_load_3d(sV + s * CF::VTILE + p * BK * 128, &tm_v, &b.kv_full[s], 64 * p, row, (int)bh);
+            tma_load_3d(sV + s * CF::VTILE + p * BK * 128, &tm_v, &b.kv_full[s], 64 * p, row, zkv);
           ++issued_kv;
         }
         if (MODE != MODE_STATE) {
@@ -538,7 +555,7 @@ la2_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       const uint32_t tKV = tmem + CF::COL_KV;
       int snap_ph = 0;
       bool ok = true;
-      for (int i = 0; i < nblk && ok; ++i) {
+      for (int i = 0; i < nsteps && ok; ++i) {
         const int qs = i % CF::QS, ks = i % CF::KS;
         const uint32_t qa = smem_u32(sQ + qs * CF::QTILE);
         const uint32_t ka = smem_u32(sK + ks * CF::KTILE);

@@ -14,7 +14,16 @@
 // One CTA per (b, h, chunk); 512 threads: warp 0 TMA, warp 1 MMA issuer
 // (+ TMEM), warps 4-7 mask S^T, A^T -> bf16 P^T, Pd^T (SMEM), warps 8-11 the
 // bf16 snapshot of U, warps 12-15 dK, dV -> HBM. A^T lives in the columns of
-// the dK accumulator until the mask warpgroup has read it.
+// the dK accumulator until the mask warpgroup has read it (Bk=128).
+//
+// Grouped K/V heads (G query heads per K/V head): a K/V head's dK and dV add
+// up over its query heads h, and so do their suffix states: with
+// U = sum_h sum_{l>i} Q_{h,l}^T dO_{h,l} one state serves the whole group,
+//   dV_i = K_i U + sum_h (S_h^T ⊙ M) dO_{h,i},  dK_i = V_i U^T + sum_h (A_h^T ⊙ M) Q_{h,i},
+//   U   += sum_h Q_{h,i}^T dO_{h,i}.
+// The CTA then runs G steps per block (causal), one per query head, loading
+// (Q_h, K, V, dO_h) each time; dK and dV leave once per block. G > 1 needs
+// A^T in its own columns (Bk=64 tiles).
 #pragma once
 
 #include "la2_sm100.cuh"
@@ -56,12 +65,13 @@ struct BCfg {
 };
 
 struct BwdParams {
-  __nv_bfloat16* dk;       // [BH][N][D]
-  __nv_bfloat16* dv;       // [BH][N][DV]
-  const float* init_u;     // [BH][C][D*DV] (state_f4 layout): suffix (causal) or total in slot 0
+  __nv_bfloat16* dk;       // [BHkv][N][D]
+  __nv_bfloat16* dv;       // [BHkv][N][DV]
+  const float* init_u;     // [BHkv][C][D*DV] (state_f4 layout): suffix (causal) or total in slot 0
   int64_t N, L, C;
   int64_t spin_limit;
   int causal;
+  int32_t H, G;            // query heads per batch; query heads per K/V head (q_seq0)
 };
 
 template <int BK, int D, int DV>
@@ -96,10 +106,14 @@ la2_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int64_t unit = blockIdx.x;
-  const int64_t bh = unit / prm.C, c = unit % prm.C;
+  const int64_t bh = unit / prm.C, c = unit % prm.C;  // bh: the K/V sequence
   const int64_t t0 = c * prm.L, t1 = min(prm.N, t0 + prm.L);
   const int nblk = static_cast<int>((t1 - t0 + BK - 1) / BK);
   const bool causal = prm.causal != 0;
+  // query heads walked per block (the non-causal form needs only K, V and U)
+  const int gq = causal && prm.G > 1 ? prm.G : 1;
+  const int nsteps = nblk * gq;
+  const int64_t q0 = q_seq0(bh, prm.H, prm.G);
   const bool has_init = !causal || (prm.init_u && c + 1 < prm.C);
   const float* init = nullptr;
   if (!causal) init = prm.init_u + bh * prm.C * static_cast<int64_t>(D * DV);
@@ -151,8 +165,9 @@ la2_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     if (lane == 0) {
       int issued = 0;
       bool ok = true;
-      for (int s = 0; s < nblk && ok; ++s) {
-        const int i = nblk - 1 - s;  // reverse block order
+      for (int s = 0; s < nsteps && ok; ++s) {
+        const int i = nblk - 1 - s / gq;  // reverse block order
+        const int hq = static_cast<int>(q0 + s % gq);  // query sequence of Q and dO
         const int row = static_cast<int>(t0 + static_cast<int64_t>(i) * BK);
         const int slot = s % CF::NS;
         if (!wait_bar(&st_empty[slot], ((s / CF::NS) & 1) ^ 1, lim, abort_flag, 201)) { ok = false; break; }
@@ -160,9 +175,9 @@ la2_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         const CUtensorMap* maps[4] = {&tm_q, &tm_k, &tm_v, &tm_do};
         for (int t = 0; t < 4; ++t) {
           if (!causal && (t == 0 || t == 3)) continue;  // non-causal needs only K and V
+          const int z = (t == 0 || t == 3) ? hq : static_cast<int>(bh);
           for (int p = 0; p < 2; ++p)
-            tma_load_3d(tile(slot, t) + p * BK * 128, maps[t], &st_full[slot], 64 * p, row,
-                        static_cast<int>(bh));
+            tma_load_3d(tile(slot, t) + p * BK * 128, maps[t], &st_full[slot], 64 * p, row, z);
         }
         ++issued;
       }
@@ -184,14 +199,17 @@ la2_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       const uint32_t snap0 = smem_u32(sSnap), pt0 = smem_u32(sPT), pdt0 = smem_u32(sPdT);
       int snap_ph = 0;
       bool ok = true;
-      for (int s = 0; s < nblk && ok; ++s) {
+      for (int s = 0; s < nsteps && ok; ++s) {
         const int slot = s % CF::NS;
+        const int blk = s / gq;                 // block counter (reverse order)
+        const bool first = s % gq == 0;         // first query head of the block
+        const bool last = s % gq == gq - 1;     // last query head of the block
         const uint32_t aq = smem_u32(tile(slot, 0)), ak = smem_u32(tile(slot, 1));
         const uint32_t av = smem_u32(tile(slot, 2)), ado = smem_u32(tile(slot, 3));
         if (!wait_w(&st_full[slot], (s / CF::NS) & 1, 210)) { ok = false; break; }
         // A^T aliasing dK: the epilogue must have read the last block's dK
-        if (!CF::AT_OWN && !wait_w(g_empty, (s & 1) ^ 1, 211)) { ok = false; break; }
-        const bool have_u = s > 0 || has_init;
+        if (!CF::AT_OWN && !wait_w(g_empty, (blk & 1) ^ 1, 211)) { ok = false; break; }
+        const bool have_u = blk > 0 || has_init;
         if (causal) {
           if (!wait_w(s_read, (s & 1) ^ 1, 212)) { ok = false; break; }
           tc_fence_after();
@@ -207,13 +225,13 @@ la2_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           mma_commit_warp(s_full);
         }
         // the dK/dV accumulators must be free (the epilogue read the last block's)
-        if (CF::AT_OWN && !wait_w(g_empty, (s & 1) ^ 1, 216)) { ok = false; break; }
-        if (have_u && (causal || s == 0)) {
+        if (CF::AT_OWN && first && !wait_w(g_empty, (blk & 1) ^ 1, 216)) { ok = false; break; }
+        if (have_u && first && (causal || s == 0)) {
           if (!wait_w(snap_full, snap_ph, 213)) { ok = false; break; }
           snap_ph ^= 1;
         }
         tc_fence_after();
-        if (have_u) {
+        if (have_u && first) {
           // dV = K U: A = K (K-major, K = d), B[n=e][k=c] = U[c][e] (snapshot, MN-major)
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t off = ((kk >> 2) * BK * 128 + (kk & 3) * 32) >> 4;
@@ -225,14 +243,14 @@ la2_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           // U += Q^T dO (after the snapshot of the old U was taken)
           for (int kk = 0; kk < BK / 16; ++kk)
             mma_bf16_ss_warp(tU, dMN + (aq >> 4) + kk * (2048 >> 4), dMN + (ado >> 4) + kk * (2048 >> 4),
-                        CF::ID_UPD, (have_u || kk > 0) ? 1u : 0u);
+                        CF::ID_UPD, (have_u || !first || kk > 0) ? 1u : 0u);
           // A^T aliasing dK: the mask warpgroup must have read it
           if (!CF::AT_OWN) {
             if (!wait_w(s_read, s & 1, 214)) { ok = false; break; }
             tc_fence_after();
           }
         }
-        if (have_u) {
+        if (have_u && first) {
           // dK = V U^T: A = V (K-major, K = dv), B[n=c][k=e] = U[c][e] (snapshot, K-major)
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t off = ((kk >> 2) * BK * 128 + (kk & 3) * 32) >> 4;
@@ -240,26 +258,27 @@ la2_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
             mma_bf16_ss_warp(tDK, dKm + (av >> 4) + off, dKm + (snap0 >> 4) + soff, CF::ID_KM, kk > 0);
           }
         }
-        // U is updated and no issued MMA reads the snapshot any more: the
-        // state warpgroup may take the next one
-        if (causal) mma_commit_warp(u_updated);
+        // U is updated (by every query head of the block) and no issued MMA
+        // reads the snapshot any more: the state warpgroup may take the next one
+        if (causal && last) mma_commit_warp(u_updated);
         if (causal) {
           if (!wait_w(p_full, s & 1, 215)) { ok = false; break; }
           tc_fence_after();
+          const uint32_t acc0 = (have_u || !first) ? 1u : 0u;
           // dV += P^T dO ; dK += Pd^T Q  (A = masked tiles, K-major, K = BK; B MN-major)
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint32_t off = ((kk >> 2) * BK * 128 + (kk & 3) * 32) >> 4;
             mma_bf16_ss_warp(tDV, dKm + (pt0 >> 4) + off, dMN + (ado >> 4) + kk * (2048 >> 4), CF::ID_MN,
-                        (have_u || kk > 0) ? 1u : 0u);
+                        (acc0 || kk > 0) ? 1u : 0u);
           }
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint32_t off = ((kk >> 2) * BK * 128 + (kk & 3) * 32) >> 4;
             mma_bf16_ss_warp(tDK, dKm + (pdt0 >> 4) + off, dMN + (aq >> 4) + kk * (2048 >> 4), CF::ID_MN,
-                        (have_u || kk > 0) ? 1u : 0u);
+                        (acc0 || kk > 0) ? 1u : 0u);
           }
           mma_commit_warp(p_empty);
         }
-        mma_commit_warp(g_full);
+        if (last) mma_commit_warp(g_full);
         mma_commit_warp(&st_empty[slot]);
       }
       mma_commit_warp(drain);
@@ -272,7 +291,7 @@ la2_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       const uint32_t lane_off = static_cast<uint32_t>(32 * w4) << 16;
       const uint32_t bases[2] = {smem_u32(sPT), smem_u32(sPdT)};
       const uint32_t srcs[2] = {tmem + CF::COL_ST + lane_off, tmem + CF::COL_AT + lane_off};
-      for (int s = 0; s < nblk; ++s) {
+      for (int s = 0; s < nsteps; ++s) {
         if (!__all_sync(0xffffffffu, wait_bar(s_full, s & 1, lim, abort_flag, 220))) break;
         if (!__all_sync(0xffffffffu, wait_bar(p_empty, (s & 1) ^ 1, lim, abort_flag, 221))) break;
         tc_fence_after();

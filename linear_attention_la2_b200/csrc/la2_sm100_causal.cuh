@@ -67,6 +67,7 @@ struct CausalParams {
   float* agg;        // range states [R][D*DV] (prefix_mode 1, or KIND_AGG output); see agg_f4
   int64_t N;
   int64_t spin_limit;
+  int32_t H, G;      // query heads per batch, query heads per K/V head (kv_seq)
 };
 
 enum Kind : int { KIND_MAIN = 0, KIND_AGG = 1 };
@@ -464,16 +465,17 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       bool ok = true;
       while (ok && it.next(st)) {
         const int row = st.blk * BK;
-        const int zz = static_cast<int>(st.bh);
+        const int zz = static_cast<int>(st.bh);                               // Q (and O)
+        const int zkv = static_cast<int>(kv_seq(st.bh, prm.H, prm.G));        // K, V
         const int ks = g % CF::KS;
         if (!wait_bar(&kv_empty[ks], ((g / CF::KS) & 1) ^ 1, lim, abort_flag, 101)) { ok = false; break; }
         LA2_TRACE_POINT(0, g);
         const bool q_here = CF::QWITHKV && !st.pre;
         mbar_expect_tx(&kv_full[ks], CF::KTILE + CF::VTILE + (q_here ? CF::QTILE : 0));
         for (int p = 0; p < CF::DP; ++p)
-          tma_load_3d(sK + ks * CF::KTILE + p * BK * 128, &tm_k, &kv_full[ks], 64 * p, row, zz);
+          tma_load_3d(sK + ks * CF::KTILE + p * BK * 128, &tm_k, &kv_full[ks], 64 * p, row, zkv);
         for (int p = 0; p < CF::VP; ++p)
-          tma_load_3d(sV + ks * CF::VTILE + p * BK * 128, &tm_v, &kv_full[ks], 64 * p, row, zz);
+          tma_load_3d(sV + ks * CF::VTILE + p * BK * 128, &tm_v, &kv_full[ks], 64 * p, row, zkv);
         if (q_here)
           for (int p = 0; p < CF::DP; ++p)
             tma_load_3d(sQ + ks * CF::QTILE + p * BK * 128, &tm_q, &kv_full[ks], 64 * p, row, zz);

@@ -43,6 +43,11 @@ _SIGS = {
                            _vp, _sz, _vp]),
     "la2_backward": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _int,
                             _int, _int, _vp, _sz, _vp]),
+    "la2_workspace_size_gqa": (_sz, [_i64, _i64, _i64, _i64, _i64, _i64, _int, _int, _int, _int]),
+    "la2_forward_gqa": (_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64, _int, _int,
+                               _int, _vp, _sz, _vp]),
+    "la2_backward_gqa": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64,
+                                _i64, _int, _int, _int, _vp, _sz, _vp]),
     "la2_check": (_int, [_vp]),
     "la2_status_string": (ctypes.c_char_p, [_int]),
     "la2_set_chunk_len": (_int, [_i64]),
@@ -73,6 +78,9 @@ la2_workspace_size = _lib.la2_workspace_size
 la2_forward = _lib.la2_forward
 la2_backward = _lib.la2_backward
 la2_check = _lib.la2_check
+la2_workspace_size_gqa = _lib.la2_workspace_size_gqa
+la2_forward_gqa = _lib.la2_forward_gqa
+la2_backward_gqa = _lib.la2_backward_gqa
 la2_set_chunk_len = _lib.la2_set_chunk_len
 la2_plan_ranges = _lib.la2_plan_ranges
 la2_set_spin_limit = _lib.la2_set_spin_limit
@@ -198,55 +206,76 @@ def _check_workspace(ws, need, device):
         raise La2Error(LA2_ERR_INVALID_ARG)
 
 
+def _kv_heads(q, k, v):
+    """K/V head count of a call: k, v [B,Hkv,N,.] with Hkv dividing q's H."""
+    if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
+        raise La2Error(LA2_ERR_INVALID_ARG)
+    H, Hkv = q.shape[1], k.shape[1]
+    if (H > 0 and (Hkv < 1 or H % Hkv)) or (H == 0 and Hkv != 0):
+        raise La2Error(LA2_ERR_INVALID_ARG)
+    return Hkv
+
+
+def workspace_bytes_gqa(B, H, Hkv, N, d, dv, causal, block, dtype_code, is_backward) -> int:
+    n = la2_workspace_size_gqa(B, H, Hkv, N, d, dv, int(causal), block, dtype_code, int(is_backward))
+    if n == ctypes.c_size_t(-1).value:
+        raise La2Error(LA2_ERR_INVALID_ARG)
+    return int(n)
+
+
 def forward(q, k, v, causal: bool = True, block: int = 64, out=None, workspace=None, stream=None):
-    """O = ((Q K^T) ⊙ M) V for [B,H,N,d] CUDA tensors; returns O."""
+    """O = ((Q K^T) ⊙ M) V for [B,H,N,d] CUDA tensors; returns O. k and v may
+    hold fewer heads (grouped K/V heads: query head h reads K/V head
+    h // (H // Hkv))."""
     import torch
 
     _check_inputs(q, k, v)
-    if q.dim() != 4 or v.dim() != 4:
-        raise La2Error(LA2_ERR_INVALID_ARG)
+    Hkv = _kv_heads(q, k, v)
     B, H, N, d = q.shape
     dv = v.shape[-1]
     dt = _dtype_code(q)
-    _check_like(q, q.shape, q.dtype, k)
-    _check_like(q, (B, H, N, dv), q.dtype, v)
+    _check_like(q, (B, Hkv, N, d), q.dtype, k)
+    _check_like(q, (B, Hkv, N, dv), q.dtype, v)
     if out is None:
         out = torch.empty((B, H, N, dv), dtype=q.dtype, device=q.device)
     _check_inputs(out)
     _check_like(q, (B, H, N, dv), q.dtype, out)
-    need = workspace_bytes(B, H, N, d, dv, causal, block, dt, False)
+    need = workspace_bytes_gqa(B, H, Hkv, N, d, dv, causal, block, dt, False)
     ws = workspace if workspace is not None else _workspace(need, q.device, stream)
     _check_workspace(ws, need, q.device)
-    _raise(la2_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, N, d, dv, int(causal), block, dt,
-                       _ptr(ws), ws.numel() if ws is not None else 0, _stream_handle(stream)))
+    _raise(la2_forward_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, Hkv, N, d, dv, int(causal),
+                           block, dt, _ptr(ws), ws.numel() if ws is not None else 0,
+                           _stream_handle(stream)))
     return out
 
 
 def backward(q, k, v, do, causal: bool = True, block: int = 64, outs=None, workspace=None,
              stream=None):
-    """Gradients (dQ, dK, dV) of <dO, O> for the same op; returns a tuple."""
+    """Gradients (dQ, dK, dV) of <dO, O> for the same op; returns a tuple. With
+    grouped K/V heads dK and dV are the sums over each group's query heads."""
     import torch
 
     _check_inputs(q, k, v, do)
-    if q.dim() != 4 or v.dim() != 4:
-        raise La2Error(LA2_ERR_INVALID_ARG)
+    Hkv = _kv_heads(q, k, v)
     B, H, N, d = q.shape
     dv = v.shape[-1]
     dt = _dtype_code(q)
-    _check_like(q, q.shape, q.dtype, k)
-    _check_like(q, (B, H, N, dv), q.dtype, v, do)
+    _check_like(q, (B, Hkv, N, d), q.dtype, k)
+    _check_like(q, (B, Hkv, N, dv), q.dtype, v)
+    _check_like(q, (B, H, N, dv), q.dtype, do)
     if outs is None:
         outs = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
     dq, dk, dvv = outs
     _check_inputs(dq, dk, dvv)
-    _check_like(q, q.shape, q.dtype, dq, dk)
-    _check_like(q, (B, H, N, dv), q.dtype, dvv)
-    need = workspace_bytes(B, H, N, d, dv, causal, block, dt, True)
+    _check_like(q, q.shape, q.dtype, dq)
+    _check_like(q, (B, Hkv, N, d), q.dtype, dk)
+    _check_like(q, (B, Hkv, N, dv), q.dtype, dvv)
+    need = workspace_bytes_gqa(B, H, Hkv, N, d, dv, causal, block, dt, True)
     ws = workspace if workspace is not None else _workspace(need, q.device, stream)
     _check_workspace(ws, need, q.device)
-    _raise(la2_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dvv), B, H, N,
-                        d, dv, int(causal), block, dt, _ptr(ws), ws.numel() if ws is not None else 0,
-                        _stream_handle(stream)))
+    _raise(la2_backward_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dvv), B,
+                            H, Hkv, N, d, dv, int(causal), block, dt, _ptr(ws),
+                            ws.numel() if ws is not None else 0, _stream_handle(stream)))
     return dq, dk, dvv
 
 

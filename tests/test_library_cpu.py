@@ -194,3 +194,32 @@ def test_header_states_the_tensor_core_shapes():
     # bf16 shapes off the tensor-core path are accepted (pointer check fails first)
     assert _fwd(dt=la2.LA2_BF16, d=64, dv=128) == la2.LA2_ERR_INVALID_ARG
     assert _fwd(dt=la2.LA2_BF16, d=128, dv=64, block=128) == la2.LA2_ERR_INVALID_ARG
+
+
+def test_gqa_rejects_bad_head_counts():
+    """H must be a multiple of the K/V head count Hkv >= 1."""
+    bad = ctypes.c_size_t(-1).value
+    ws = la2.la2_workspace_size_gqa
+    for H, Hkv in ((8, 3), (8, 0), (8, -1), (4, 8)):
+        assert ws(1, H, Hkv, 16, 64, 64, 1, 64, la2.LA2_F32, 0) == bad
+        assert la2.la2_forward_gqa(NULL, NULL, NULL, NULL, 1, H, Hkv, 16, 64, 64, 1, 64, la2.LA2_F32,
+                                   NULL, 0, NULL) == la2.LA2_ERR_INVALID_ARG
+        assert la2.la2_backward_gqa(NULL, NULL, NULL, NULL, NULL, NULL, NULL, 1, H, Hkv, 16, 64, 64,
+                                    1, 64, la2.LA2_F32, NULL, 0, NULL) == la2.LA2_ERR_INVALID_ARG
+    # empty problems are still no-ops
+    assert la2.la2_forward_gqa(NULL, NULL, NULL, NULL, 0, 8, 2, 16, 64, 64, 1, 64, la2.LA2_F32, NULL,
+                               0, NULL) == la2.LA2_OK
+    assert ws(1, 0, 0, 16, 64, 64, 1, 64, la2.LA2_F32, 0) == 0
+    # a valid grouping with NULL pointers fails only on the pointers
+    assert la2.la2_forward_gqa(NULL, NULL, NULL, NULL, 1, 8, 2, 16, 64, 64, 1, 64, la2.LA2_F32, NULL,
+                               0, NULL) == la2.LA2_ERR_INVALID_ARG
+
+
+def test_binding_checks_grouped_shapes():
+    import torch
+
+    q = torch.zeros(1, 8, 16, 64)
+    assert la2._kv_heads(q, torch.zeros(1, 2, 16, 64), torch.zeros(1, 2, 16, 64)) == 2
+    for kv in (torch.zeros(1, 3, 16, 64), torch.zeros(1, 0, 16, 64)):
+        with pytest.raises(la2.La2Error):
+            la2._kv_heads(q, kv, kv)
