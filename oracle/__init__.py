@@ -6,7 +6,9 @@ from .la2_oracle import (  # noqa: F401
     backward_rows,
     blocked_forward,
     decode_step,
+    backward_from_states,
     forward,
+    forward_from_state,
     forward_gqa,
     forward_rows,
     kv_state,

@@ -33,7 +33,9 @@ exist to pin the definition (and to check very long sequences where the O(N^2)
 definition is too slow on a CPU), never the other way round. ``kv_state`` (the
 state after a prefill) and ``decode_step`` (one RNN-mode step) are the oracle of
 the inference form; ``forward_gqa`` / ``backward_gqa`` the oracle of grouped K/V
-heads (a layout of the same op: each query head reads the K/V head of its group).
+heads (a layout of the same op: each query head reads the K/V head of its group);
+``forward_from_state`` / ``backward_from_states`` the oracle of one part of a
+sequence whose other parts are summarised by KV states (sequence parallelism).
 
 Parity status: every function here is pinned by ``tests/test_oracle.py``
 (brute force on tiny integer inputs, closed forms, RNN-form equality, block-size
@@ -288,6 +290,37 @@ def decode_step(q, k, v, state):
     new = s + k[..., :, None] * v[..., None, :]
     o = np.einsum("bhd,bhde->bhe", q, new)
     return o, new
+
+
+def forward_from_state(q, k, v, state) -> np.ndarray:
+    """Causal output of a sequence whose earlier tokens are summarised by a KV
+    state ``state [B,H,d,dv]`` (article, point 2: a block's inter-block part is
+    its queries times the state accumulated over everything before it):
+    ``o_t = q_t state + sum_{s <= t} (q_t . k_s) v_s``. With the state of a
+    sequence's first part this is the output of its second part (sequence
+    parallelism: each shard starts from the sum of the earlier shards' states).
+    """
+    st = _f64(state)
+    out = forward(q, k, v, True)
+    return out + np.einsum("bhnd,bhde->bhne", _f64(q), st)
+
+
+def backward_from_states(q, k, v, do, prefix, suffix):
+    """Gradients, for one part of a longer causal sequence, of the loss
+    ``sum_t <dO_t, O_t>`` over the whole sequence: the part's closed forms
+    (``backward``) plus the terms that cross its ends. ``prefix [B,H,d,dv]`` is
+    the KV state of the tokens before the part (its queries read it:
+    ``dq_t += dO_t prefix^T``); ``suffix [B,H,d,dv]`` is ``sum q_t^T dO_t`` over
+    the tokens after it (their queries read this part's keys and values:
+    ``dk_s += v_s suffix^T``, ``dv_s += k_s suffix``).
+    """
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    P, U = _f64(prefix), _f64(suffix)
+    dq, dk, dvv = backward(q, k, v, do, True)
+    dq = dq + np.einsum("bhne,bhde->bhnd", do, P)
+    dk = dk + np.einsum("bhne,bhde->bhnd", v, U)
+    dvv = dvv + np.einsum("bhnd,bhde->bhne", k, U)
+    return dq, dk, dvv
 
 
 def blocked_forward(q, k, v, block: int, causal: bool = True) -> np.ndarray:
