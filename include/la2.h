@@ -138,6 +138,42 @@ LA2_API la2_status la2_backward_gqa(const void *q, const void *k, const void *v,
                                     size_t workspace_bytes, la2_stream_t stream);
 
 /*
+ * Sequence parallelism: one part (a contiguous range of N rows) of longer
+ * causal sequences whose other parts live elsewhere, e.g. on other GPUs
+ * (youleyou.com article, section "小结": sequence-parallel linear attention as
+ * the next step; section "Lightning Attention-2简介", point 2: the part's
+ * inter-block term is its queries times the state of everything before it).
+ * q, k, v, o, dout, dq, dk, dvv: this part, [B,H,N,.] as for la2_forward
+ * (one K/V head per query head). States are fp32, row-major [d][dv] per
+ * (b, h), device memory, 16-byte aligned:
+ *  - prefix_states [n_prefix][B][H][d][dv]: their sum is the KV state
+ *    sum k_t^T v_t of every token before this part (la2_kv_state of each
+ *    earlier part);
+ *  - suffix_states [n_suffix][B][H][d][dv]: their sum is sum q_t^T dO_t over
+ *    every token after this part (la2_kv_state with (q, dO) in the (k, v)
+ *    slots, for each later part).
+ * la2_forward_sp writes the part's causal output o_t = q_t P + sum over the
+ * part's s <= t of (q_t . k_s) v_s; la2_backward_sp the part's gradients of
+ * the whole sequence's L = <dO, O> (dq += dO P^T, dk += v U^T, dv += k U for
+ * the summed prefix P and suffix U). n = 0 means no such parts (NULL allowed);
+ * states must not overlap the outputs. Workspace: la2_workspace_size_sp.
+ * Other conventions and errors as for la2_forward / la2_backward.
+ */
+LA2_API size_t la2_workspace_size_sp(int64_t B, int64_t H, int64_t N, int64_t d, int64_t dv,
+                                     int block, la2_dtype dt, int is_backward);
+LA2_API la2_status la2_forward_sp(const void *q, const void *k, const void *v, void *o,
+                                  const float *prefix_states, int64_t n_prefix, int64_t B,
+                                  int64_t H, int64_t N, int64_t d, int64_t dv, int block,
+                                  la2_dtype dt, void *workspace, size_t workspace_bytes,
+                                  la2_stream_t stream);
+LA2_API la2_status la2_backward_sp(const void *q, const void *k, const void *v, const void *dout,
+                                   void *dq, void *dk, void *dvv, const float *prefix_states,
+                                   int64_t n_prefix, const float *suffix_states, int64_t n_suffix,
+                                   int64_t B, int64_t H, int64_t N, int64_t d, int64_t dv, int block,
+                                   la2_dtype dt, void *workspace, size_t workspace_bytes,
+                                   la2_stream_t stream);
+
+/*
  * Synchronises `stream`, then reports and clears the device-side error word
  * that kernels set when a bounded wait gives up (LA2_ERR_TIMEOUT), or
  * LA2_ERR_CUDA if the stream holds a CUDA error. LA2_OK otherwise.

@@ -149,7 +149,7 @@ static la2_status check_shape(int64_t B, int64_t H, int64_t N, int64_t d, int64_
 }
 
 static Plan make_plan_uncached(int64_t B, int64_t H, int64_t Hkv, int64_t N, int64_t d, int64_t dv,
-                               int causal, int block, la2_dtype dt, bool is_bwd, int sms) {
+                               int causal, int block, la2_dtype dt, bool is_bwd, int sms, bool sp) {
   Plan p;
   const int64_t BH = B * H;
   const int64_t BHkv = B * Hkv;
@@ -179,7 +179,9 @@ static Plan make_plan_uncached(int64_t B, int64_t H, int64_t Hkv, int64_t N, int
   // task indices fit in 32 bits. Otherwise the chunk path below runs, for the
   // forward as for the backward's dQ pass.
   bool range_fits = false;
-  if (p.tc && causal) {
+  // A part of a longer sequence (sequence parallelism) starts from the states
+  // of the other parts: the chunk path, whose state scan takes them as a base.
+  if (p.tc && causal && !sp) {
     p.rp = plan_ranges(BH, N, block, sms, g_chunk_len);
     range_fits = p.rp.R >= 1 && p.rp.R <= sm100::kMaxRanges && BH * T <= 0x7fffffff;
     p.ranges = range_fits;
@@ -191,7 +193,7 @@ static Plan make_plan_uncached(int64_t B, int64_t H, int64_t Hkv, int64_t N, int
   }
   p.L = L;
   p.C = std::max<int64_t>(1, (N + L - 1) / L);
-  p.need_states = (p.C > 1) || !causal;
+  p.need_states = (p.C > 1) || !causal || sp;
   // chunk states belong to K/V sequences (shared by a group's query heads)
   const size_t one = (size_t)BHkv * (size_t)p.C * state_bytes;
   p.ws_bytes = p.need_states ? one * (is_bwd ? 2 : 1) : 0;
@@ -211,29 +213,30 @@ static Plan make_plan_uncached(int64_t B, int64_t H, int64_t Hkv, int64_t N, int
 // count; the range split is a small search, so recent plans are kept.
 struct PlanKey {
   int64_t B, H, Hkv, N, d, dv, chunk_len;
-  int causal, block, dt, is_bwd, sms;
+  int causal, block, dt, is_bwd, sms, sp;
   bool operator==(const PlanKey& o) const {
     return B == o.B && H == o.H && Hkv == o.Hkv && N == o.N && d == o.d && dv == o.dv &&
            chunk_len == o.chunk_len && causal == o.causal && block == o.block && dt == o.dt &&
-           is_bwd == o.is_bwd && sms == o.sms;
+           is_bwd == o.is_bwd && sms == o.sms && sp == o.sp;
   }
 };
 
 static Plan make_plan(int64_t B, int64_t H, int64_t N, int64_t d, int64_t dv, int causal, int block,
-                      la2_dtype dt, bool is_bwd, int sms, int64_t Hkv = -1) {
+                      la2_dtype dt, bool is_bwd, int sms, int64_t Hkv = -1, bool sp = false) {
   if (Hkv < 0) Hkv = H;
   constexpr int kSlots = 16;
   static PlanKey keys[kSlots];
   static Plan plans[kSlots];
   static int used = 0, next_slot = 0;
   static std::mutex mu;
-  const PlanKey k{B, H, Hkv, N, d, dv, g_chunk_len, causal, block, static_cast<int>(dt), is_bwd ? 1 : 0, sms};
+  const PlanKey k{B, H, Hkv, N, d, dv, g_chunk_len, causal, block, static_cast<int>(dt), is_bwd ? 1 : 0,
+                  sms, sp ? 1 : 0};
   {
     std::lock_guard<std::mutex> lock(mu);
     for (int i = 0; i < used; ++i)
       if (keys[i] == k) return plans[i];
   }
-  Plan p = make_plan_uncached(B, H, Hkv, N, d, dv, causal, block, dt, is_bwd, sms);
+  Plan p = make_plan_uncached(B, H, Hkv, N, d, dv, causal, block, dt, is_bwd, sms, sp);
   std::lock_guard<std::mutex> lock(mu);
   keys[next_slot] = k;
   plans[next_slot] = p;
@@ -257,6 +260,17 @@ struct Heads {
   int32_t H, G;
 };
 
+// States of the other parts of each sequence (sequence parallelism): the sum
+// of n_pre states [n_pre][nseq][d][dv] before this part (the causal prefix,
+// K^T V) and of n_suf states after it (sum Q^T dO, the backward's suffix).
+struct Ext {
+  const float* pre = nullptr;
+  int64_t n_pre = 0;
+  const float* suf = nullptr;
+  int64_t n_suf = 0;
+  bool on = false;
+};
+
 template <typename T>
 static la2_status run_chunk_states(const void* a, const void* b, float* out, int64_t nseq, int64_t N,
                                    int da, int db, const Plan& p, cudaStream_t st, int32_t H = 1,
@@ -268,10 +282,13 @@ static la2_status run_chunk_states(const void* a, const void* b, float* out, int
   return launch_status();
 }
 
-static la2_status run_scan(float* s, int64_t nseq, int nel, const Plan& p, int mode, cudaStream_t st) {
+static la2_status run_scan(float* s, int64_t nseq, int nel, const Plan& p, int mode, cudaStream_t st,
+                           const float* ext = nullptr, int64_t n_ext = 0, int d = 0, int dv = 0,
+                           int f4_layout = 0) {
   dim3 grid((nel + kSimtThreads - 1) / kSimtThreads, (unsigned)nseq);
   LaunchTimer t(K_CHUNK_SCAN, st);
-  if (launch_pdl(chunk_scan_kernel, grid, dim3(kSimtThreads), 0, st, s, p.C, nel, mode) != cudaSuccess)
+  if (launch_pdl(chunk_scan_kernel, grid, dim3(kSimtThreads), 0, st, s, p.C, nel, mode,
+                 n_ext > 0 ? ext : nullptr, n_ext, nseq, d, dv, f4_layout) != cudaSuccess)
     return LA2_ERR_CUDA;
   return launch_status();
 }
@@ -391,7 +408,7 @@ static la2_status kv_chunk_states(const CUtensorMap& tk, const CUtensorMap& tv, 
 template <int BK>
 static la2_status forward_sm100_bk(const void* q, const void* k, const void* v, void* o,
                                    const Heads& hd, int64_t N, int causal, float* states,
-                                   const Plan& p, int64_t spin, cudaStream_t st) {
+                                   const Plan& p, int64_t spin, cudaStream_t st, const Ext& ext) {
   if (causal && p.ranges)
     return causal_range_split<BK>(q, k, v, o, hd, N, states, p.rp, spin, st, K_STATE_TC, K_FWD_TC);
   constexpr int D = 128, DV = 128;
@@ -418,10 +435,11 @@ static la2_status forward_sm100_bk(const void* q, const void* k, const void* v, 
     if (p.need_states) {
       s = kv_chunk_states<BK>(tk, tv, states, hd, N, p, spin, st);
       if (s != LA2_OK) return s;
-      s = run_scan(states, hd.BHkv, nel, p, 0, st);
+      s = run_scan(states, hd.BHkv, nel, p, 0, st, ext.pre, ext.n_pre, D, DV, 1);
       if (s != LA2_OK) return s;
     }
     prm.init_states = p.need_states ? states : nullptr;
+    prm.init_all = ext.on ? 1 : 0;
     prm.units_per_seq = p.C;
     LaunchTimer t(K_FWD_TC, st);
     return launch_fwd_sm100<BK, D, DV, sm100::MODE_CAUSAL>(tq, tk, tv, to_c, prm, hd.BH * p.C, st);
@@ -445,7 +463,7 @@ static la2_status forward_sm100_bk(const void* q, const void* k, const void* v, 
 template <int TB>
 static la2_status dkdv_sm100(const void* q, const void* k, const void* v, const void* dout, void* dk,
                              void* dvv, const Heads& hd, int64_t N, int causal, const float* s_u,
-                             const Plan& p, int64_t spin, cudaStream_t st) {
+                             const Plan& p, int64_t spin, cudaStream_t st, bool init_all) {
   constexpr int D = 128, DV = 128;
   CUtensorMap tq, tk, tv, tdo;
   if (!make_tmap_3d(&tq, q, hd.BH, N, D, TB) || !make_tmap_3d(&tk, k, hd.BHkv, N, D, TB) ||
@@ -462,6 +480,7 @@ static la2_status dkdv_sm100(const void* q, const void* k, const void* v, const 
   pb.causal = causal;
   pb.H = hd.H;
   pb.G = hd.G;
+  pb.init_all = init_all ? 1 : 0;
   CUtensorMap tdk = tq, tdv = tq;
   if (sm100::BCfg<TB, D, DV>::TMA_STORE &&
       (!make_tmap_3d(&tdk, dk, hd.BHkv, N, D, 16) || !make_tmap_3d(&tdv, dvv, hd.BHkv, N, DV, 16)))
@@ -478,7 +497,7 @@ template <int BK>
 static la2_status backward_sm100_bk(const void* q, const void* k, const void* v, const void* dout,
                                     void* dq, void* dk, void* dvv, const Heads& hd, int64_t N,
                                     int causal, float* s_kv, float* s_u, const Plan& p,
-                                    int64_t spin, cudaStream_t st) {
+                                    int64_t spin, cudaStream_t st, const Ext& ext) {
   constexpr int D = 128, DV = 128;
   CUtensorMap tq, tk, tv, tdo;
   if (!make_tmap_3d(&tq, q, hd.BH, N, D, BK) || !make_tmap_3d(&tk, k, hd.BHkv, N, D, BK) ||
@@ -515,10 +534,10 @@ static la2_status backward_sm100_bk(const void* q, const void* k, const void* v,
     }
     if (s != LA2_OK) return s;
     if (!dq_split && (causal || p.C > kSumInKernel)) {
-      s = run_scan(s_kv, hd.BHkv, nel, p, causal ? 0 : 2, st);
+      s = run_scan(s_kv, hd.BHkv, nel, p, causal ? 0 : 2, st, ext.pre, ext.n_pre, D, DV, 1);
       if (s != LA2_OK) return s;
     }
-    s = run_scan(s_u, hd.BHkv, nel, p, causal ? 1 : 2, st);
+    s = run_scan(s_u, hd.BHkv, nel, p, causal ? 1 : 2, st, ext.suf, ext.n_suf, D, DV, 1);
     if (s != LA2_OK) return s;
   }
   // Otherwise (non-causal, or a forced split beyond the range table) the
@@ -536,6 +555,7 @@ static la2_status backward_sm100_bk(const void* q, const void* k, const void* v,
     pq.H = hd.H;
     pq.G = hd.G;
     pq.state_group = 1;
+    pq.init_all = ext.on ? 1 : 0;
     CUtensorMap tdq = tq;
     if (sm100::Cfg<BK, D, DV>::TMA_STORE && !make_tmap_3d(&tdq, dq, hd.BH, N, D, 16)) return LA2_ERR_CUDA;
     {
@@ -550,15 +570,17 @@ static la2_status backward_sm100_bk(const void* q, const void* k, const void* v,
   // A group of query heads accumulates into one dK, dV: the scores of each
   // head need their own TMEM columns, which 64-row tiles leave free.
   if (hd.G > 1 && BK == 128 && causal)
-    return dkdv_sm100<64>(q, k, v, dout, dk, dvv, hd, N, causal, states ? s_u : nullptr, p, spin, st);
-  return dkdv_sm100<BK>(q, k, v, dout, dk, dvv, hd, N, causal, states ? s_u : nullptr, p, spin, st);
+    return dkdv_sm100<64>(q, k, v, dout, dk, dvv, hd, N, causal, states ? s_u : nullptr, p, spin, st,
+                          ext.on);
+  return dkdv_sm100<BK>(q, k, v, dout, dk, dvv, hd, N, causal, states ? s_u : nullptr, p, spin, st,
+                        ext.on);
 }
 
 static la2_status forward_sm100(const void* q, const void* k, const void* v, void* o, const Heads& hd,
                                 int64_t N, int causal, int block, float* states, const Plan& p,
-                                int64_t spin, cudaStream_t st) {
-  return block == 64 ? forward_sm100_bk<64>(q, k, v, o, hd, N, causal, states, p, spin, st)
-                     : forward_sm100_bk<128>(q, k, v, o, hd, N, causal, states, p, spin, st);
+                                int64_t spin, cudaStream_t st, const Ext& ext) {
+  return block == 64 ? forward_sm100_bk<64>(q, k, v, o, hd, N, causal, states, p, spin, st, ext)
+                     : forward_sm100_bk<128>(q, k, v, o, hd, N, causal, states, p, spin, st, ext);
 }
 
 }  // namespace la2
@@ -732,10 +754,21 @@ la2_status la2_decode_step(const void* q, const void* k, const void* v, void* o,
   return launch_status();
 }
 
-la2_status la2_forward_gqa(const void* q, const void* k, const void* v, void* o, int64_t B,
-                           int64_t H, int64_t Hkv, int64_t N, int64_t d, int64_t dv, int causal,
-                           int block, la2_dtype dt, void* workspace, size_t workspace_bytes,
-                           la2_stream_t stream) {
+}  // extern "C"
+
+namespace la2 {
+
+static bool ext_ok(const float* p, int64_t n, size_t one, const void* out, size_t nout) {
+  if (n < 0) return false;
+  if (n == 0) return true;
+  if (!p || !is_aligned(p, 16)) return false;
+  return !overlaps(p, (size_t)n * one, out, nout);
+}
+
+static la2_status forward_impl(const void* q, const void* k, const void* v, void* o, int64_t B,
+                               int64_t H, int64_t Hkv, int64_t N, int64_t d, int64_t dv, int causal,
+                               int block, la2_dtype dt, void* workspace, size_t workspace_bytes,
+                               la2_stream_t stream, const Ext& ext) {
   la2_status s = check_shape(B, H, N, d, dv, causal, block, dt, false, Hkv);
   if (s != LA2_OK) return s;
   if (B == 0 || H == 0 || N == 0) return LA2_OK;
@@ -747,9 +780,11 @@ la2_status la2_forward_gqa(const void* q, const void* k, const void* v, void* o,
   const size_t nk = (size_t)B * Hkv * N * d * es, nv = (size_t)B * Hkv * N * dv * es;
   if (overlaps(o, no, q, nq) || overlaps(o, no, k, nk) || overlaps(o, no, v, nv))
     return LA2_ERR_INVALID_ARG;
+  if (!ext_ok(ext.pre, ext.n_pre, (size_t)B * Hkv * d * dv * sizeof(float), o, no))
+    return LA2_ERR_INVALID_ARG;
   const int sms = device_sm_count();
   if (sms <= 0) return LA2_ERR_CUDA;
-  const Plan p = make_plan(B, H, N, d, dv, causal, block, dt, false, sms, Hkv);
+  const Plan p = make_plan(B, H, N, d, dv, causal, block, dt, false, sms, Hkv, ext.on);
   const Heads hd{B * H, B * Hkv, static_cast<int32_t>(H), static_cast<int32_t>(H / Hkv)};
   if (p.ws_bytes > 0) {
     if (!workspace || workspace_bytes < p.ws_bytes) return LA2_ERR_WORKSPACE;
@@ -759,13 +794,13 @@ la2_status la2_forward_gqa(const void* q, const void* k, const void* v, void* o,
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   float* states = p.need_states ? static_cast<float*>(workspace) : nullptr;
   const int nel = (int)(d * dv);
-  if (p.tc) return forward_sm100(q, k, v, o, hd, N, causal, block, states, p, spin_limit(), st);
+  if (p.tc) return forward_sm100(q, k, v, o, hd, N, causal, block, states, p, spin_limit(), st, ext);
   if (p.need_states) {  // K^T V chunk states of the K/V sequences, then their prefix / total
     s = dt == LA2_BF16
             ? run_chunk_states<__nv_bfloat16>(k, v, states, hd.BHkv, N, (int)d, (int)dv, p, st)
             : run_chunk_states<float>(k, v, states, hd.BHkv, N, (int)d, (int)dv, p, st);
     if (s != LA2_OK) return s;
-    s = run_scan(states, hd.BHkv, nel, p, causal ? 0 : 2, st);
+    s = run_scan(states, hd.BHkv, nel, p, causal ? 0 : 2, st, ext.pre, ext.n_pre, (int)d, (int)dv, 0);
     if (s != LA2_OK) return s;
   }
   return dt == LA2_BF16
@@ -775,6 +810,39 @@ la2_status la2_forward_gqa(const void* q, const void* k, const void* v, void* o,
                                    st);
 }
 
+}  // namespace la2
+
+extern "C" {
+
+la2_status la2_forward_gqa(const void* q, const void* k, const void* v, void* o, int64_t B,
+                           int64_t H, int64_t Hkv, int64_t N, int64_t d, int64_t dv, int causal,
+                           int block, la2_dtype dt, void* workspace, size_t workspace_bytes,
+                           la2_stream_t stream) {
+  return forward_impl(q, k, v, o, B, H, Hkv, N, d, dv, causal, block, dt, workspace, workspace_bytes,
+                      stream, Ext{});
+}
+
+la2_status la2_forward_sp(const void* q, const void* k, const void* v, void* o,
+                          const float* prefix_states, int64_t n_prefix, int64_t B, int64_t H,
+                          int64_t N, int64_t d, int64_t dv, int block, la2_dtype dt,
+                          void* workspace, size_t workspace_bytes, la2_stream_t stream) {
+  Ext ext;
+  ext.pre = prefix_states;
+  ext.n_pre = n_prefix;
+  ext.on = true;
+  return forward_impl(q, k, v, o, B, H, H, N, d, dv, 1, block, dt, workspace, workspace_bytes, stream,
+                      ext);
+}
+
+size_t la2_workspace_size_sp(int64_t B, int64_t H, int64_t N, int64_t d, int64_t dv, int block,
+                             la2_dtype dt, int is_backward) {
+  if (check_shape(B, H, N, d, dv, 1, block, dt, is_backward != 0) != LA2_OK) return (size_t)-1;
+  if (B == 0 || H == 0 || N == 0) return 0;
+  const int sms = device_sm_count();
+  if (sms <= 0) return (size_t)-1;
+  return make_plan(B, H, N, d, dv, 1, block, dt, is_backward != 0, sms, H, true).ws_bytes;
+}
+
 la2_status la2_forward(const void* q, const void* k, const void* v, void* o, int64_t B, int64_t H,
                        int64_t N, int64_t d, int64_t dv, int causal, int block, la2_dtype dt,
                        void* workspace, size_t workspace_bytes, la2_stream_t stream) {
@@ -782,10 +850,15 @@ la2_status la2_forward(const void* q, const void* k, const void* v, void* o, int
                          workspace_bytes, stream);
 }
 
-la2_status la2_backward_gqa(const void* q, const void* k, const void* v, const void* dout, void* dq,
-                            void* dk, void* dvv, int64_t B, int64_t H, int64_t Hkv, int64_t N,
-                            int64_t d, int64_t dv, int causal, int block, la2_dtype dt,
-                            void* workspace, size_t workspace_bytes, la2_stream_t stream) {
+}  // extern "C"
+
+namespace la2 {
+
+static la2_status backward_impl(const void* q, const void* k, const void* v, const void* dout,
+                                void* dq, void* dk, void* dvv, int64_t B, int64_t H, int64_t Hkv,
+                                int64_t N, int64_t d, int64_t dv, int causal, int block,
+                                la2_dtype dt, void* workspace, size_t workspace_bytes,
+                                la2_stream_t stream, const Ext& ext) {
   la2_status s = check_shape(B, H, N, d, dv, causal, block, dt, true, Hkv);
   if (s != LA2_OK) return s;
   if (B == 0 || H == 0 || N == 0) return LA2_OK;
@@ -806,9 +879,14 @@ la2_status la2_backward_gqa(const void* q, const void* k, const void* v, const v
     for (int j = i + 1; j < 3; ++j)
       if (overlaps(outs[i], out_sz[i], outs[j], out_sz[j])) return LA2_ERR_INVALID_ARG;
   }
+  const size_t one = (size_t)B * Hkv * d * dv * sizeof(float);
+  for (int i = 0; i < 3; ++i)
+    if (!ext_ok(ext.pre, ext.n_pre, one, outs[i], out_sz[i]) ||
+        !ext_ok(ext.suf, ext.n_suf, one, outs[i], out_sz[i]))
+      return LA2_ERR_INVALID_ARG;
   const int sms = device_sm_count();
   if (sms <= 0) return LA2_ERR_CUDA;
-  const Plan p = make_plan(B, H, N, d, dv, causal, block, dt, true, sms, Hkv);
+  const Plan p = make_plan(B, H, N, d, dv, causal, block, dt, true, sms, Hkv, ext.on);
   if (p.ws_bytes > 0) {
     if (!workspace || workspace_bytes < p.ws_bytes) return LA2_ERR_WORKSPACE;
     if (!is_aligned(workspace, 256)) return LA2_ERR_INVALID_ARG;
@@ -830,9 +908,9 @@ la2_status la2_backward_gqa(const void* q, const void* k, const void* v, const v
       second = static_cast<float*>(workspace);
     }
     return block == 64 ? backward_sm100_bk<64>(q, k, v, dout, dq, dk, dvv, hd, N, causal, second,
-                                                s_u, p, spin_limit(), st)
+                                                s_u, p, spin_limit(), st, ext)
                        : backward_sm100_bk<128>(q, k, v, dout, dq, dk, dvv, hd, N, causal, second,
-                                                 s_u, p, spin_limit(), st);
+                                                 s_u, p, spin_limit(), st, ext);
   }
   if (p.need_states) {
     const bool bf = dt == LA2_BF16;
@@ -844,9 +922,9 @@ la2_status la2_backward_gqa(const void* q, const void* k, const void* v, const v
            : run_chunk_states<float>(q, dout, s_u, hd.BHkv, N, (int)d, (int)dv, p, st, hd.H, hd.G,
                                      hd.G);
     if (s != LA2_OK) return s;
-    s = run_scan(s_kv, hd.BHkv, nel, p, causal ? 0 : 2, st);
+    s = run_scan(s_kv, hd.BHkv, nel, p, causal ? 0 : 2, st, ext.pre, ext.n_pre, (int)d, (int)dv, 0);
     if (s != LA2_OK) return s;
-    s = run_scan(s_u, hd.BHkv, nel, p, causal ? 1 : 2, st);
+    s = run_scan(s_u, hd.BHkv, nel, p, causal ? 1 : 2, st, ext.suf, ext.n_suf, (int)d, (int)dv, 0);
     if (s != LA2_OK) return s;
   }
   return dt == LA2_BF16
@@ -854,6 +932,33 @@ la2_status la2_backward_gqa(const void* q, const void* k, const void* v, const v
                                             causal, block, s_kv, s_u, p, st)
              : backward_simt<float>(q, k, v, dout, dq, dk, dvv, hd, N, (int)d, (int)dv, causal,
                                     block, s_kv, s_u, p, st);
+}
+
+}  // namespace la2
+
+extern "C" {
+
+la2_status la2_backward_gqa(const void* q, const void* k, const void* v, const void* dout, void* dq,
+                            void* dk, void* dvv, int64_t B, int64_t H, int64_t Hkv, int64_t N,
+                            int64_t d, int64_t dv, int causal, int block, la2_dtype dt,
+                            void* workspace, size_t workspace_bytes, la2_stream_t stream) {
+  return backward_impl(q, k, v, dout, dq, dk, dvv, B, H, Hkv, N, d, dv, causal, block, dt, workspace,
+                       workspace_bytes, stream, Ext{});
+}
+
+la2_status la2_backward_sp(const void* q, const void* k, const void* v, const void* dout, void* dq,
+                           void* dk, void* dvv, const float* prefix_states, int64_t n_prefix,
+                           const float* suffix_states, int64_t n_suffix, int64_t B, int64_t H,
+                           int64_t N, int64_t d, int64_t dv, int block, la2_dtype dt,
+                           void* workspace, size_t workspace_bytes, la2_stream_t stream) {
+  Ext ext;
+  ext.pre = prefix_states;
+  ext.n_pre = n_prefix;
+  ext.suf = suffix_states;
+  ext.n_suf = n_suffix;
+  ext.on = true;
+  return backward_impl(q, k, v, dout, dq, dk, dvv, B, H, H, N, d, dv, 1, block, dt, workspace,
+                       workspace_bytes, stream, ext);
 }
 
 la2_status la2_backward(const void* q, const void* k, const void* v, const void* dout, void* dq,

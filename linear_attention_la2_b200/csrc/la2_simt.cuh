@@ -88,9 +88,20 @@ chunk_state_kernel(const T* __restrict__ a, const T* __restrict__ b, float* __re
 //   mode 0: exclusive prefix  P_c = sum_{c' < c} S_c'   (causal, forward order)
 //   mode 1: exclusive suffix  R_c = sum_{c' > c} S_c'   (causal, reverse order)
 //   mode 2: total into slot 0  T = sum_c S_c             (non-causal)
+// `ext` (optional) adds a base to every prefix / suffix: the sum of n_ext
+// states [n_ext][nseq][d][dv] (row-major fp32) of the parts of the sequence
+// before (mode 0) or after (mode 1) this one. `f4_layout` says the chunk
+// states are in the tensor-core layout (state_f4: float4 j of row r at j*d + r).
 // ----------------------------------------------------------------------------
+__device__ __forceinline__ int64_t state_row_major_index(int e, int d, int dv, int f4_layout) {
+  if (!f4_layout) return e;
+  const int f4 = e >> 2, j = f4 / d, r = f4 - j * d;
+  return static_cast<int64_t>(r) * dv + 4 * j + (e & 3);
+}
+
 __global__ void __launch_bounds__(kSimtThreads)
-chunk_scan_kernel(float* __restrict__ s, int64_t C, int nel, int mode) {
+chunk_scan_kernel(float* __restrict__ s, int64_t C, int nel, int mode, const float* __restrict__ ext,
+                  int64_t n_ext, int64_t nseq, int d, int dv, int f4_layout) {
   pdl_launch_dependents();
   pdl_wait();
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
@@ -98,6 +109,10 @@ chunk_scan_kernel(float* __restrict__ s, int64_t C, int nel, int mode) {
   float* p = s + (int64_t)blockIdx.y * C * nel + e;
   constexpr int U = 8;  // independent loads in flight per thread
   float run = 0.f;
+  if (ext) {
+    const int64_t rm = state_row_major_index(e, d, dv, f4_layout);
+    for (int64_t i = 0; i < n_ext; ++i) run += ext[(i * nseq + blockIdx.y) * nel + rm];
+  }
   if (mode == 2) {
     for (int64_t c0 = 0; c0 < C; c0 += U) {
       float x[U];

@@ -164,6 +164,16 @@ __device__ __forceinline__ void mma_bf16_ss_warp(uint32_t d_tmem, uint64_t a_des
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// D[tmem] (+)= A[tmem] * B[smem]: the A operand (M rows in TMEM lanes, two
+// bf16 of consecutive k per 32-bit column) is read from tensor memory.
+__device__ __forceinline__ void mma_bf16_ts_warp(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                                 uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p, e;\n elect.sync _|e, 0xffffffff;\n setp.ne.b32 p, %4, 0;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 __device__ __forceinline__ void mma_commit_warp(uint64_t* bar) {
   asm volatile(
       "{\n .reg .pred e;\n elect.sync _|e, 0xffffffff;\n"
@@ -202,6 +212,15 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       : "memory");
 }
 #undef LA2_W8
+// Thread t writes 16 consecutive 32-bit columns of TMEM lane (lane field of taddr) + t.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+      "%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -326,6 +345,9 @@ struct Params {
   // sequences (the K and V slots then hold Q and dO: the dK/dV pass's U).
   int32_t H, G;
   int32_t state_group;
+  // MODE_CAUSAL: every chunk, the first included, starts from its slot of
+  // init_states (a sequence part whose earlier parts are summarised there).
+  int32_t init_all;
 };
 
 // Shared state of one CTA.
@@ -458,7 +480,8 @@ la2_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   const int64_t bkv = MODE == MODE_STATE ? bh : kv_seq(bh, prm.H, prm.G);
   const int sgroup = (MODE == MODE_STATE && prm.state_group > 1) ? prm.state_group : 1;
   const int nsteps = MODE == MODE_STATE ? nblk * sgroup : nblk;
-  const bool has_init = (MODE == MODE_NONCAUSAL) || (MODE == MODE_CAUSAL && prm.init_states && c > 0);
+  const bool has_init = (MODE == MODE_NONCAUSAL) ||
+                        (MODE == MODE_CAUSAL && prm.init_states && (c > 0 || prm.init_all));
   const float* init = nullptr;
   if (MODE == MODE_NONCAUSAL) init = prm.init_states + bkv * prm.C * (int64_t)(D * DV);
   else if (has_init) init = prm.init_states + (bkv * prm.C + c) * (int64_t)(D * DV);

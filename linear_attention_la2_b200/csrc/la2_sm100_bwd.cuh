@@ -72,6 +72,7 @@ struct BwdParams {
   int64_t spin_limit;
   int causal;
   int32_t H, G;            // query heads per batch; query heads per K/V head (q_seq0)
+  int32_t init_all;        // causal: the last chunk too starts from its slot of init_u
 };
 
 template <int BK, int D, int DV>
@@ -114,7 +115,7 @@ la2_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   const int gq = causal && prm.G > 1 ? prm.G : 1;
   const int nsteps = nblk * gq;
   const int64_t q0 = q_seq0(bh, prm.H, prm.G);
-  const bool has_init = !causal || (prm.init_u && c + 1 < prm.C);
+  const bool has_init = !causal || (prm.init_u && (c + 1 < prm.C || prm.init_all));
   const float* init = nullptr;
   if (!causal) init = prm.init_u + bh * prm.C * static_cast<int64_t>(D * DV);
   else if (has_init) init = prm.init_u + (bh * prm.C + c) * static_cast<int64_t>(D * DV);

@@ -198,10 +198,16 @@ struct CCfg {
   // The state-only pass (KIND_AGG) holds no Q, P, snapshot or O tiles and
   // spends that space on a deeper K/V ring: its loads are latency-bound.
   static constexpr bool AGG = KIND == KIND_AGG;
-  static constexpr int QS = BK == 64 ? 3 : 1;
+  // Bk=128: P lives in tensor memory (the P V MMA reads its A operand there)
+  // and O has one TMEM buffer; the shared memory a P tile would take carries a
+  // second Q slot instead, so Q rides with K and V in a 2-deep ring and the
+  // next block's Q arrives while the current block computes.
+  static constexpr bool P_TMEM = BK == 128 && !AGG;
+  static constexpr int QS = BK == 64 ? 3 : 2;
   static constexpr int KS = AGG ? (BK == 64 ? 6 : 3) : (BK == 64 ? 3 : 2);
   static constexpr int NSB = BK == 64 ? 2 : 1;    // S buffers (TMEM)
-  static constexpr int NPB = BK == 64 ? 2 : 1;    // P buffers (SMEM)
+  static constexpr int NPB = BK == 64 ? 2 : 1;    // P buffers (SMEM at Bk=64, TMEM at Bk=128)
+  static constexpr int NOB = P_TMEM ? 1 : 2;      // O buffers (TMEM)
   // One snapshot buffer suffices: the state role writes snapshot m+1 only after
   // update(m) completed, and update(m) is issued after QKV(m) read snapshot m.
   static constexpr int NSNAP = 1;
@@ -212,8 +218,9 @@ struct CCfg {
   static constexpr int OSTAGE = TMA_STORE ? 2 : 0;
   // Q rides in the K/V ring (one barrier per step) when the rings are as deep.
   static constexpr bool QWITHKV = QS == KS;
-  // With two P buffers the P-free signal is the O-full commit of the same block.
-  static constexpr bool MERGE_OP = NPB == 2;
+  // With as many P as O buffers the P-free signal is the O-full commit of the
+  // block that read the P buffer (P V is the last MMA writing that O).
+  static constexpr bool MERGE_OP = NPB == NOB;
   static constexpr int DP = D / 64;
   static constexpr int VP = DV / 64;
   static constexpr int QTILE = BK * D * 2;
@@ -226,13 +233,14 @@ struct CCfg {
   static constexpr int OFF_K = OFF_Q + (AGG ? 0 : QS * QTILE);
   static constexpr int OFF_V = OFF_K + KS * KTILE;
   static constexpr int OFF_P = OFF_V + KS * VTILE;
-  static constexpr int OFF_SNAP = OFF_P + (AGG ? 0 : NPB * PTILE);
+  static constexpr int OFF_SNAP = OFF_P + ((AGG || P_TMEM) ? 0 : NPB * PTILE);
   static constexpr int OFF_OST = OFF_SNAP + (AGG ? 0 : NSNAP * SNAP);
   static constexpr int OFF_BAR = OFF_OST + OSTAGE * OTILE;
   static constexpr int NBAR = 2 * QS + 2 * KS + 15;  // rings + 6 pairs + 3 singles
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
   static constexpr uint32_t COL_KV = 0;
-  static constexpr uint32_t COL_O = 128;  // two buffers of 128 columns
+  static constexpr uint32_t COL_O = 128;  // NOB buffers of 128 columns
+  static constexpr uint32_t COL_P = 256;  // P_TMEM: BK rows x BK bf16 (BK / 2 columns)
   static constexpr uint32_t COL_S = 384;  // NSB buffers of BK columns
   static constexpr uint32_t ID_S = make_idesc(BK, BK, false, false);
   static constexpr uint32_t ID_QKV = make_idesc(BK, DV, false, true);
@@ -240,6 +248,8 @@ struct CCfg {
   static constexpr uint32_t ID_PV = make_idesc(BK, DV, false, true);
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
   static_assert(COL_S + NSB * BK <= kTmemCols, "TMEM budget");
+  static_assert(COL_O + NOB * 128 <= (P_TMEM ? COL_P : COL_S) && COL_P + BK / 2 <= COL_S,
+                "TMEM columns of O, P and S overlap");
 };
 
 template <int D>
@@ -545,6 +555,7 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         LA2_TRACE_POINT(5, mm);
         if (!CF::QWITHKV && !wait_w(&q_full[mm % CF::QS], (mm / CF::QS) & 1, 111)) return false;
         if (!wait_w(&kv_full[gg % CF::KS], (gg / CF::KS) & 1, 112)) return false;
+        LA2_TRACE_POINT(15, mm);
         // S buffer mm % NSB is free: the mask role read S(mm - NSB) before it
         // arrived on p_full(mm - 1), which this warp waited for before PV(mm - 1).
         tc_fence_after();
@@ -583,9 +594,10 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
               !wait_w(&snap_full[sb], (sn / CF::NSNAP) & 1, 115)) { ok = false; break; }
           if (!wait_ack()) { ok = false; break; }
           LA2_TRACE_POINT(2, m);
-          const uint32_t ob = m & 1;
+          const uint32_t ob = m % CF::NOB;
           const uint32_t tO = tmem + CF::COL_O + ob * 128;
-          if (!wait_w(&o_empty[ob], ((m >> 1) & 1) ^ 1, 116)) { ok = false; break; }
+          if (!wait_w(&o_empty[ob], ((m / CF::NOB) & 1) ^ 1, 116)) { ok = false; break; }
+          LA2_TRACE_POINT(13, m);
           tc_fence_after();
           if (needs_snap) {
             const uint64_t a = dKm + ((sQ0 + qslot(m, g) * CF::QTILE) >> 4);
@@ -607,7 +619,14 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           if (!wait_w(&p_full[pb], (m / CF::NPB) & 1, 117)) { ok = false; break; }
           LA2_TRACE_POINT(4, m);
           tc_fence_after();
-          {
+          if constexpr (CF::P_TMEM) {
+            // A = P from TMEM: the k-th 16-column slice of P is 8 TMEM columns in
+            const uint64_t b = dK_mn + ((sV0 + ks * CF::VTILE) >> 4);
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk)
+              mma_bf16_ts_warp(tO, tmem + CF::COL_P + kk * 8, b + kk * (2048 >> 4), CF::ID_PV,
+                               (needs_snap || kk > 0) ? 1u : 0u);
+          } else {
             const uint64_t a = dKm + ((sP0 + pb * CF::PTILE) >> 4);
             const uint64_t b = dK_mn + ((sV0 + ks * CF::VTILE) >> 4);
 #pragma unroll
@@ -620,6 +639,7 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           mma_commit_warp(&o_full[ob]);
           if (!CF::MERGE_OP) mma_commit_warp(&p_empty[pb]);
           mma_commit_warp(&kv_empty[ks]);
+          LA2_TRACE_POINT(14, m);
           ++m;
         }
         ++g;
@@ -648,6 +668,31 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         uint64_t* p_free = CF::MERGE_OP ? o_full : p_empty;
         if (!__all_sync(0xffffffffu, wait_bar(&p_free[pb], ((m / CF::NPB) & 1) ^ 1, lim, abort_flag, 121))) break;
         tc_fence_after();
+        if constexpr (CF::P_TMEM) {
+          // P rows into TMEM next to S: lane r, column j holds bf16 P[r][2j], P[r][2j+1]
+          const uint32_t tP = tmem + CF::COL_P + lane_off;
+#pragma unroll
+          for (int c32 = 0; c32 < BK / 32; ++c32) {
+            uint32_t v[32];
+            tmem_ld32(tS + c32 * 32, v);
+            tmem_ld_wait();
+            uint32_t w[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int col = c32 * 32 + 2 * e;
+              const float a = (col <= r) ? __uint_as_float(v[2 * e]) : 0.f;
+              const float bb = (col + 1 <= r) ? __uint_as_float(v[2 * e + 1]) : 0.f;
+              w[e] = pack_bf16x2(a, bb);
+            }
+            tmem_st16(tP + c32 * 16, w);
+          }
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(&p_full[pb]);
+          if (threadIdx.x % 128 == 0) LA2_TRACE_POINT(8, m);
+          ++m;
+          continue;
+        }
         const uint32_t pbase = smem_u32(sP + pb * CF::PTILE);
 #pragma unroll
         for (int c32 = 0; c32 < BK / 32; ++c32) {
@@ -790,9 +835,9 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       uint32_t m = 0;
       while (it.next(st)) {
         if (st.pre) continue;
-        const uint32_t ob = m & 1;
+        const uint32_t ob = m % CF::NOB;
         const uint32_t tO = tmem + CF::COL_O + ob * 128 + lane_off;
-        if (!__all_sync(0xffffffffu, wait_bar(&o_full[ob], (m >> 1) & 1, lim, abort_flag, 140))) break;
+        if (!__all_sync(0xffffffffu, wait_bar(&o_full[ob], (m / CF::NOB) & 1, lim, abort_flag, 140))) break;
         if (threadIdx.x % 128 == 0) LA2_TRACE_POINT(11, m);
         tc_fence_after();
         if constexpr (CF::TMA_STORE) {
@@ -845,6 +890,30 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         const int64_t row = static_cast<int64_t>(st.blk) * BK + r;
         const bool valid = r >= 0 && row < prm.N;
         uint4* dst = reinterpret_cast<uint4*>(prm.o + (st.bh * prm.N + (valid ? row : 0)) * DV);
+        if constexpr (CF::NOB == 1) {
+          // One O buffer: read the whole row out of TMEM (packed to bf16) and
+          // release the buffer to the next block's Q KV before the stores.
+          uint32_t pk[DV / 2];
+#pragma unroll
+          for (int c32 = 0; c32 < DV / 32; ++c32) {
+            uint32_t v[32];
+            tmem_ld32(tO + c32 * 32, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              pk[c32 * 16 + e] = pack_bf16x2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
+          }
+          tc_fence_before();
+          mbar_arrive(&o_empty[ob]);
+          if (valid) {
+#pragma unroll
+            for (int q = 0; q < DV / 8; ++q)
+              dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+          }
+          if (threadIdx.x % 128 == 0) LA2_TRACE_POINT(12, m);
+          ++m;
+          continue;
+        }
 #pragma unroll
         for (int c32 = 0; c32 < DV / 32; ++c32) {
           uint32_t v[32];

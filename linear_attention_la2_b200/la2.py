@@ -48,6 +48,11 @@ _SIGS = {
                                _int, _vp, _sz, _vp]),
     "la2_backward_gqa": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64,
                                 _i64, _int, _int, _int, _vp, _sz, _vp]),
+    "la2_workspace_size_sp": (_sz, [_i64, _i64, _i64, _i64, _i64, _int, _int, _int]),
+    "la2_forward_sp": (_int, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64, _int,
+                              _int, _vp, _sz, _vp]),
+    "la2_backward_sp": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _i64, _i64, _i64,
+                               _i64, _i64, _i64, _int, _int, _vp, _sz, _vp]),
     "la2_check": (_int, [_vp]),
     "la2_status_string": (ctypes.c_char_p, [_int]),
     "la2_set_chunk_len": (_int, [_i64]),
@@ -81,6 +86,9 @@ la2_check = _lib.la2_check
 la2_workspace_size_gqa = _lib.la2_workspace_size_gqa
 la2_forward_gqa = _lib.la2_forward_gqa
 la2_backward_gqa = _lib.la2_backward_gqa
+la2_workspace_size_sp = _lib.la2_workspace_size_sp
+la2_forward_sp = _lib.la2_forward_sp
+la2_backward_sp = _lib.la2_backward_sp
 la2_set_chunk_len = _lib.la2_set_chunk_len
 la2_plan_ranges = _lib.la2_plan_ranges
 la2_set_spin_limit = _lib.la2_set_spin_limit
@@ -330,3 +338,78 @@ def decode_step(q, k, v, state, out=None, stream=None):
 
 def check(stream=None):
     _raise(la2_check(_stream_handle(stream)))
+
+
+def _states_arg(states, q):
+    """(pointer, count) of a [n,B,H,d,dv] float32 stack of states (None: none)."""
+    import torch
+
+    if states is None or states.shape[0] == 0:
+        return _vp(0), 0
+    B, H, _, d = q.shape
+    _check_inputs(states)
+    if states.dim() != 5 or tuple(states.shape[1:4]) != (B, H, d) or states.dtype != torch.float32 \
+            or states.device != q.device:
+        raise La2Error(LA2_ERR_INVALID_ARG)
+    return _ptr(states), int(states.shape[0])
+
+
+def forward_sp(q, k, v, prefix_states=None, block: int = 64, out=None, workspace=None, stream=None):
+    """Causal output of one part of longer sequences: ``prefix_states``
+    [n,B,H,d,dv] float32 sum to the KV state of everything before the part."""
+    import torch
+
+    _check_inputs(q, k, v)
+    if q.dim() != 4 or v.dim() != 4:
+        raise La2Error(LA2_ERR_INVALID_ARG)
+    B, H, N, d = q.shape
+    dv = v.shape[-1]
+    dt = _dtype_code(q)
+    _check_like(q, q.shape, q.dtype, k)
+    _check_like(q, (B, H, N, dv), q.dtype, v)
+    if out is None:
+        out = torch.empty((B, H, N, dv), dtype=q.dtype, device=q.device)
+    _check_inputs(out)
+    _check_like(q, (B, H, N, dv), q.dtype, out)
+    pp, npre = _states_arg(prefix_states, q)
+    need = la2_workspace_size_sp(B, H, N, d, dv, block, dt, 0)
+    if need == ctypes.c_size_t(-1).value:
+        raise La2Error(LA2_ERR_INVALID_ARG)
+    ws = workspace if workspace is not None else _workspace(need, q.device, stream)
+    _check_workspace(ws, need, q.device)
+    _raise(la2_forward_sp(_ptr(q), _ptr(k), _ptr(v), _ptr(out), pp, npre, B, H, N, d, dv, block, dt,
+                          _ptr(ws), ws.numel() if ws is not None else 0, _stream_handle(stream)))
+    return out
+
+
+def backward_sp(q, k, v, do, prefix_states=None, suffix_states=None, block: int = 64, outs=None,
+                workspace=None, stream=None):
+    """Gradients of one part of longer sequences: ``prefix_states`` sum to the
+    KV state before the part, ``suffix_states`` to sum q^T dO after it."""
+    import torch
+
+    _check_inputs(q, k, v, do)
+    if q.dim() != 4 or v.dim() != 4:
+        raise La2Error(LA2_ERR_INVALID_ARG)
+    B, H, N, d = q.shape
+    dv = v.shape[-1]
+    dt = _dtype_code(q)
+    _check_like(q, q.shape, q.dtype, k)
+    _check_like(q, (B, H, N, dv), q.dtype, v, do)
+    if outs is None:
+        outs = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
+    dq, dk, dvv = outs
+    _check_inputs(dq, dk, dvv)
+    _check_like(q, q.shape, q.dtype, dq, dk)
+    _check_like(q, (B, H, N, dv), q.dtype, dvv)
+    pp, npre = _states_arg(prefix_states, q)
+    sp, nsuf = _states_arg(suffix_states, q)
+    need = la2_workspace_size_sp(B, H, N, d, dv, block, dt, 1)
+    if need == ctypes.c_size_t(-1).value:
+        raise La2Error(LA2_ERR_INVALID_ARG)
+    ws = workspace if workspace is not None else _workspace(need, q.device, stream)
+    _check_workspace(ws, need, q.device)
+    _raise(la2_backward_sp(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dvv), pp,
+                           npre, sp, nsuf, B, H, N, d, dv, block, dt, _ptr(ws),
+                           ws.numel() if ws is not None else 0, _stream_handle(stream)))
+    return dq, dk, dvv
