@@ -356,9 +356,10 @@ static la2_status causal_range_split(const void* q, const void* k, const void* v
     return LA2_ERR_CUDA;
   sm100::RangeTable rt;
   if (!fill_range_table(rp, &rt)) return LA2_ERR_UNSUPPORTED;
-  // O tiles leave through per-warp TMA stores of 16 rows at Bk=64.
+  // O tiles leave through per-warp TMA stores: 16 rows a warp at Bk=64, 32 at Bk=128.
   CUtensorMap to = tq;
-  if (sm100::CCfg<BK, D, DV>::TMA_STORE && !make_tmap_3d(&to, o, hd.BH, N, DV, 16))
+  using CF = sm100::CCfg<BK, D, DV>;
+  if ((CF::TMA_STORE || CF::O_IN_Q) && !make_tmap_3d(&to, o, hd.BH, N, DV, CF::O_IN_Q ? 32 : 16))
     return LA2_ERR_CUDA;
   sm100::CausalParams cp{};
   cp.o = static_cast<__nv_bfloat16*>(o);

@@ -216,8 +216,13 @@ struct CCfg {
   // queue that the MMA warp's barrier and tcgen05 instructions also use).
   static constexpr bool TMA_STORE = BK == 64 && !AGG;
   static constexpr int OSTAGE = TMA_STORE ? 2 : 0;
-  // Q rides in the K/V ring (one barrier per step) when the rings are as deep.
-  static constexpr bool QWITHKV = QS == KS;
+  // Bk=128: O(m) is staged in Q(m)'s tile (dead once P V(m) completed; same
+  // size and swizzled layout) and leaves by TMA stores; the epilogue, not the
+  // MMA warp, then releases the Q slot, after its stores have read the tile.
+  static constexpr bool O_IN_Q = BK == 128 && !AGG;
+  // Q rides in the K/V ring (one barrier per step) when the rings are as deep
+  // and the MMA warp releases Q.
+  static constexpr bool QWITHKV = QS == KS && !O_IN_Q;
   // With as many P as O buffers the P-free signal is the O-full commit of the
   // block that read the P buffer (P V is the last MMA writing that O).
   static constexpr bool MERGE_OP = NPB == NOB;
@@ -400,7 +405,10 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < CF::QS; ++s) { mbar_init(&q_full[s], 1); mbar_init(&q_empty[s], 1); }
+    for (int s = 0; s < CF::QS; ++s) {
+      mbar_init(&q_full[s], 1);
+      mbar_init(&q_empty[s], CF::O_IN_Q ? 4 : 1);  // O_IN_Q: one arrival per epilogue warp
+    }
     for (int s = 0; s < CF::KS; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&s_full[s], 1);
@@ -419,7 +427,7 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   }
   if (warp == kWarpProducer && lane == 0) {
     if (KIND == KIND_MAIN) tma_prefetch(&tm_q);
-    if (KIND == KIND_MAIN && CF::TMA_STORE) tma_prefetch(&tm_o);
+    if (KIND == KIND_MAIN && (CF::TMA_STORE || CF::O_IN_Q)) tma_prefetch(&tm_o);
     tma_prefetch(&tm_k);
     tma_prefetch(&tm_v);
   }
@@ -610,7 +618,7 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
             mma_commit_warp(&snap_free[sb]);
             ++sn;
           }
-          if (!CF::QWITHKV) mma_commit_warp(&q_empty[m % CF::QS]);
+          if (!CF::QWITHKV && !CF::O_IN_Q) mma_commit_warp(&q_empty[m % CF::QS]);
           update(ks, needs_snap);
           mma_commit_warp(kv_updated);
           if (st.seg_last) ack_pending = true;
@@ -890,25 +898,48 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         const int64_t row = static_cast<int64_t>(st.blk) * BK + r;
         const bool valid = r >= 0 && row < prm.N;
         uint4* dst = reinterpret_cast<uint4*>(prm.o + (st.bh * prm.N + (valid ? row : 0)) * DV);
-        if constexpr (CF::NOB == 1) {
+        if constexpr (CF::O_IN_Q) {
           // One O buffer: read the whole row out of TMEM (packed to bf16) and
-          // release the buffer to the next block's Q KV before the stores.
-          uint32_t pk[DV / 2];
+          // release the buffer to the next block's Q KV first; then stage the
+          // row in Q(m)'s tile (128B-swizzled 64-column panels, as TMA wrote Q)
+          // and store this warp's 32 rows with TMA.
+          (void)valid;
+          (void)dst;
+          const uint32_t qs = m % CF::QS;
+          uint8_t* stage = sQ + qs * CF::QTILE;
 #pragma unroll
           for (int c32 = 0; c32 < DV / 32; ++c32) {
             uint32_t v[32];
             tmem_ld32(tO + c32 * 32, v);
             tmem_ld_wait();
+            if (c32 == DV / 32 - 1) {  // every TMEM read of O(m) is done
+              tc_fence_before();
+              mbar_arrive(&o_empty[ob]);
+            }
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-              pk[c32 * 16 + e] = pack_bf16x2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
+            for (int q = 0; q < 4; ++q) {  // 16-byte chunk ch of row r
+              const int ch = c32 * 4 + q;
+              const int panel = ch >> 3, cj = ch & 7;
+              st_shared_v4(smem_u32(stage + panel * BK * 128) + r * 128 + ((cj ^ (r & 7)) << 4),
+                           pack_bf16x2(__uint_as_float(v[8 * q]), __uint_as_float(v[8 * q + 1])),
+                           pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3])),
+                           pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5])),
+                           pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7])));
+            }
           }
-          tc_fence_before();
-          mbar_arrive(&o_empty[ob]);
-          if (valid) {
+          fence_proxy_async();
+          __syncwarp();
+          if (lane == 0) {
+            const int64_t y = static_cast<int64_t>(st.blk) * BK + 32 * w4;
+            if (y < prm.N) {  // rows past N are clipped by the tensor map
 #pragma unroll
-            for (int q = 0; q < DV / 8; ++q)
-              dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+              for (int p = 0; p < DV / 64; ++p)
+                tma_store_3d(&tm_o, stage + p * BK * 128 + 32 * w4 * 128, 64 * p,
+                             static_cast<int>(y), static_cast<int>(st.bh));
+            }
+            bulk_commit_group();
+            bulk_wait_group_read<0>();  // the tile may take Q(m + QS) once read
+            mbar_arrive(&q_empty[qs]);
           }
           if (threadIdx.x % 128 == 0) LA2_TRACE_POINT(12, m);
           ++m;
@@ -934,7 +965,7 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (threadIdx.x % 128 == 0) LA2_TRACE_POINT(12, m);
         ++m;
       }
-      if (CF::TMA_STORE && lane == 0) bulk_wait_group<0>();  // stores done before exit
+      if ((CF::TMA_STORE || CF::O_IN_Q) && lane == 0) bulk_wait_group<0>();  // stores done before exit
     }
   }
 
