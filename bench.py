@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--workload", default="bf16_long_512k")
     ap.add_argument("--block", type=int, default=0, help="override the workload's block size")
     ap.add_argument("--N", type=int, default=0, help="override the sequence length")
+    ap.add_argument("--causal", type=int, default=1, choices=[0, 1],
+                    help="0: the non-causal form O = Q (K^T V) of the same workload")
     ap.add_argument("--impl", default="la2", choices=["la2", "reference"])
     ap.add_argument("--sweep", action="store_true",
                     help="also print one line per sequence-length sweep point, the 512K case and "
@@ -306,10 +308,11 @@ def run_reference(args):
     if rank != 0:
         return 0
     w = workload_from_args(args)
-    _, _, text = oracle_sample_plan(w)
+    causal = bool(args.causal)
+    _, _, text = oracle_sample_plan(w, causal)
     total, tokens = 0.0, 0
     for i in range(args.warmup + args.steps):
-        n, t = oracle_sample(w, i)
+        n, t = oracle_sample(w, i, causal)
         if i >= args.warmup:
             total += t
             tokens += n
@@ -319,7 +322,7 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": config_of(w),
+        "config": config_of(w, causal),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": _oracle_cores(),
                          "kind": "oracle", "sample": f"each step: {text}, on host cores"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -361,7 +364,8 @@ def run_gpu(args):
     w = workload_from_args(args)
     hbm, tf_burst, tf_sust, peak_kind = peaks()
 
-    line = bench_workload(args, w, dev, la2, world, rank, local, hbm, peak_kind, main=True)
+    line = bench_workload(args, w, dev, la2, world, rank, local, hbm, peak_kind, main=True,
+                          causal=bool(args.causal))
     if rank == 0:
         print(json.dumps(line), flush=True)
     if args.sweep:
@@ -557,7 +561,7 @@ def bench_workload(args, w, dev, la2, world, rank, local, hbm, peak_kind, main, 
         line["metric"] = FWDBWD_METRIC
         line["config"]["workload"] += " (+ backward)"
     if main and not args.no_e2e and not w.backward:
-        line["e2e"] = e2e_measure(args, w, dev, la2, world, base, ws, ws_bytes, dt)
+        line["e2e"] = e2e_measure(args, w, dev, la2, world, base, ws, ws_bytes, dt, causal)
     if main and rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_oracle_rate(w, budget_s=10.0, causal=causal)
     return line
@@ -670,7 +674,7 @@ def bench_decode(args, dev, la2, world, hbm, peak_kind):
     }
 
 
-def e2e_measure(args, w, dev, la2, world, base, ws, ws_bytes, dt):
+def e2e_measure(args, w, dev, la2, world, base, ws, ws_bytes, dt, causal=True):
     """Same metric through the public binding with host buffers: every step copies
     Q, K, V from pinned host memory, runs the forward and reads O back."""
     import torch
@@ -687,7 +691,7 @@ def e2e_measure(args, w, dev, la2, world, base, ws, ws_bytes, dt):
         dq.copy_(hq, non_blocking=True)
         dk.copy_(hk, non_blocking=True)
         dvv.copy_(hv, non_blocking=True)
-        la2.forward(dq, dk, dvv, causal=True, block=w.block, out=do, workspace=ws if ws_bytes else None)
+        la2.forward(dq, dk, dvv, causal=causal, block=w.block, out=do, workspace=ws if ws_bytes else None)
         ho.copy_(do, non_blocking=True)
 
     for _ in range(max(1, args.warmup)):

@@ -464,7 +464,8 @@ static la2_status forward_sm100_bk(const void* q, const void* k, const void* v, 
 template <int TB>
 static la2_status dkdv_sm100(const void* q, const void* k, const void* v, const void* dout, void* dk,
                              void* dvv, const Heads& hd, int64_t N, int causal, const float* s_u,
-                             const Plan& p, int64_t spin, cudaStream_t st, bool init_all) {
+                             const Plan& p, int64_t spin, cudaStream_t st, bool init_all,
+                             bool sum_states) {
   constexpr int D = 128, DV = 128;
   CUtensorMap tq, tk, tv, tdo;
   if (!make_tmap_3d(&tq, q, hd.BH, N, D, TB) || !make_tmap_3d(&tk, k, hd.BHkv, N, D, TB) ||
@@ -482,6 +483,7 @@ static la2_status dkdv_sm100(const void* q, const void* k, const void* v, const 
   pb.H = hd.H;
   pb.G = hd.G;
   pb.init_all = init_all ? 1 : 0;
+  pb.sum_states = sum_states ? 1 : 0;
   CUtensorMap tdk = tq, tdv = tq;
   if (sm100::BCfg<TB, D, DV>::TMA_STORE &&
       (!make_tmap_3d(&tdk, dk, hd.BHkv, N, D, 16) || !make_tmap_3d(&tdv, dvv, hd.BHkv, N, DV, 16)))
@@ -508,6 +510,7 @@ static la2_status backward_sm100_bk(const void* q, const void* k, const void* v,
   const int nel = D * DV;
   const bool states = p.need_states;
   const bool dq_split = causal && p.dq_ranges;
+  const bool u_summed = states && !ext.on && p.C <= kSumInKernel;
   if (dq_split) {
     // dQ = ((dO V^T) ⊙ M) K: the causal forward with (dO, V, K) as (Q, K, V).
     s = causal_range_split<BK>(dout, v, k, dq, hd, N, s_kv, p.rp, spin, st, K_STATE_TC, K_BWD_DQ_TC);
@@ -538,8 +541,13 @@ static la2_status backward_sm100_bk(const void* q, const void* k, const void* v,
       s = run_scan(s_kv, hd.BHkv, nel, p, causal ? 0 : 2, st, ext.pre, ext.n_pre, D, DV, 1);
       if (s != LA2_OK) return s;
     }
-    s = run_scan(s_u, hd.BHkv, nel, p, causal ? 1 : 2, st, ext.suf, ext.n_suf, D, DV, 1);
-    if (s != LA2_OK) return s;
+    // A few chunk states per sequence: the dK/dV pass adds up the later (or,
+    // without the mask, all) chunks' states itself; many, or with external
+    // states of other parts: scan first.
+    if (!u_summed) {
+      s = run_scan(s_u, hd.BHkv, nel, p, causal ? 1 : 2, st, ext.suf, ext.n_suf, D, DV, 1);
+      if (s != LA2_OK) return s;
+    }
   }
   // Otherwise (non-causal, or a forced split beyond the range table) the
   // block loop over chunks from the scanned K^T V prefix (or total) states.
@@ -572,9 +580,9 @@ static la2_status backward_sm100_bk(const void* q, const void* k, const void* v,
   // head need their own TMEM columns, which 64-row tiles leave free.
   if (hd.G > 1 && BK == 128 && causal)
     return dkdv_sm100<64>(q, k, v, dout, dk, dvv, hd, N, causal, states ? s_u : nullptr, p, spin, st,
-                          ext.on);
+                          ext.on, u_summed);
   return dkdv_sm100<BK>(q, k, v, dout, dk, dvv, hd, N, causal, states ? s_u : nullptr, p, spin, st,
-                        ext.on);
+                        ext.on, u_summed);
 }
 
 static la2_status forward_sm100(const void* q, const void* k, const void* v, void* o, const Heads& hd,

@@ -73,6 +73,9 @@ struct BwdParams {
   int causal;
   int32_t H, G;            // query heads per batch; query heads per K/V head (q_seq0)
   int32_t init_all;        // causal: the last chunk too starts from its slot of init_u
+  // 1: init_u holds the raw chunk states (no scan ran); a chunk adds up the
+  // states of the later chunks of its sequence (causal) or all of them.
+  int32_t sum_states;
 };
 
 template <int BK, int D, int DV>
@@ -117,8 +120,17 @@ la2_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   const int64_t q0 = q_seq0(bh, prm.H, prm.G);
   const bool has_init = !causal || (prm.init_u && (c + 1 < prm.C || prm.init_all));
   const float* init = nullptr;
-  if (!causal) init = prm.init_u + bh * prm.C * static_cast<int64_t>(D * DV);
-  else if (has_init) init = prm.init_u + (bh * prm.C + c) * static_cast<int64_t>(D * DV);
+  // states added at init: one scanned slot, or the raw states of chunks
+  // [c0, C) of the sequence (the later chunks, or all of them without the mask)
+  int64_t c0 = 0, nsum = 1;
+  if (!causal) {
+    init = prm.init_u + bh * prm.C * static_cast<int64_t>(D * DV);
+    nsum = prm.sum_states ? prm.C : 1;
+  } else if (has_init) {
+    c0 = prm.sum_states ? c + 1 : c;
+    nsum = prm.sum_states ? prm.C - c - 1 : 1;
+    init = prm.init_u + (bh * prm.C + c0) * static_cast<int64_t>(D * DV);
+  }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < CF::NS; ++s) { mbar_init(&st_full[s], 1); mbar_init(&st_empty[s], 1); }
@@ -348,16 +360,23 @@ la2_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     if (has_init) {
 #pragma unroll 1
       for (int c32 = 0; c32 < DV / 32; ++c32) {
-        uint32_t u[32];
-        const float4* src = reinterpret_cast<const float4*>(init);
+        float acc[32];
 #pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) {
-          const float4 x = src[state_f4<D>(r, c32 * 8 + q4)];
-          u[4 * q4] = __float_as_uint(x.x);
-          u[4 * q4 + 1] = __float_as_uint(x.y);
-          u[4 * q4 + 2] = __float_as_uint(x.z);
-          u[4 * q4 + 3] = __float_as_uint(x.w);
+        for (int j = 0; j < 32; ++j) acc[j] = 0.f;
+        for (int64_t cc = 0; cc < nsum; ++cc) {  // chunk states in chunk order
+          const float4* src = reinterpret_cast<const float4*>(init + cc * static_cast<int64_t>(D * DV));
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4) {
+            const float4 x = src[state_f4<D>(r, c32 * 8 + q4)];
+            acc[4 * q4] += x.x;
+            acc[4 * q4 + 1] += x.y;
+            acc[4 * q4 + 2] += x.z;
+            acc[4 * q4 + 3] += x.w;
+          }
         }
+        uint32_t u[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) u[j] = __float_as_uint(acc[j]);
         if (causal) tmem_st32(tU + c32 * 32, u);
         put_row(u, c32 * 32);
       }
