@@ -359,7 +359,9 @@ static la2_status causal_range_split(const void* q, const void* k, const void* v
   // O tiles leave through per-warp TMA stores: 16 rows a warp at Bk=64, 32 at Bk=128.
   CUtensorMap to = tq;
   using CF = sm100::CCfg<BK, D, DV>;
-  if ((CF::TMA_STORE || CF::O_IN_Q) && !make_tmap_3d(&to, o, hd.BH, N, DV, CF::O_IN_Q ? 32 : 16))
+  // (Bk=64 with O transposed in TMEM: one store of the whole 64-row tile.)
+  if ((CF::TMA_STORE || CF::O_IN_Q) &&
+      !make_tmap_3d(&to, o, hd.BH, N, DV, CF::O_IN_Q ? 32 : (CF::OT ? BK : 16)))
     return LA2_ERR_CUDA;
   sm100::CausalParams cp{};
   cp.o = static_cast<__nv_bfloat16*>(o);

@@ -241,19 +241,24 @@ struct CCfg {
   static constexpr int OFF_SNAP = OFF_P + ((AGG || P_TMEM) ? 0 : NPB * PTILE);
   static constexpr int OFF_OST = OFF_SNAP + (AGG ? 0 : NSNAP * SNAP);
   static constexpr int OFF_BAR = OFF_OST + OSTAGE * OTILE;
-  static constexpr int NBAR = 2 * QS + 2 * KS + 15;  // rings + 6 pairs + 3 singles
+  static constexpr int NBAR = 2 * QS + 2 * KS + 19;  // rings + 8 pairs + 3 singles
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
   static constexpr uint32_t COL_KV = 0;
   static constexpr uint32_t COL_O = 128;  // NOB buffers of 128 columns
   static constexpr uint32_t COL_P = 256;  // P_TMEM: BK rows x BK bf16 (BK / 2 columns)
   static constexpr uint32_t COL_S = 384;  // NSB buffers of BK columns
+  // Bk=64: O is accumulated transposed, O^T = KV^T Q^T + V^T P^T (M = dv = 128
+  // rows of the tensor datapath instead of M = Bk = 64: the two O products at
+  // full rate), BK columns per buffer; the epilogue transposes while staging.
+  static constexpr bool OT = BK == 64 && !AGG;
+  static constexpr uint32_t O_COLS = OT ? BK : 128;  // TMEM columns of one O buffer
   static constexpr uint32_t ID_S = make_idesc(BK, BK, false, false);
-  static constexpr uint32_t ID_QKV = make_idesc(BK, DV, false, true);
+  static constexpr uint32_t ID_QKV = OT ? make_idesc(DV, BK, true, false) : make_idesc(BK, DV, false, true);
   static constexpr uint32_t ID_UPD = make_idesc(D, DV, true, true);
-  static constexpr uint32_t ID_PV = make_idesc(BK, DV, false, true);
+  static constexpr uint32_t ID_PV = OT ? make_idesc(DV, BK, true, false) : make_idesc(BK, DV, false, true);
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
   static_assert(COL_S + NSB * BK <= kTmemCols, "TMEM budget");
-  static_assert(COL_O + NOB * 128 <= (P_TMEM ? COL_P : COL_S) && COL_P + BK / 2 <= COL_S,
+  static_assert(COL_O + NOB * O_COLS <= (P_TMEM ? COL_P : COL_S) && COL_P + BK / 2 <= COL_S,
                 "TMEM columns of O, P and S overlap");
 };
 
@@ -401,7 +406,9 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   uint64_t* kv_updated = o_empty + 2;
   uint64_t* seg_ack = kv_updated + 1;
   uint64_t* drain = seg_ack + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* stage_free = drain + 1;       // [2] transposing epilogue: staging tile free
+  uint64_t* stage_full = stage_free + 2;  // [2] transposing epilogue: staging tile written
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(stage_full + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   if (threadIdx.x == 0) {
@@ -422,6 +429,10 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     mbar_init(kv_updated, 1);
     mbar_init(seg_ack, 128);
     mbar_init(drain, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&stage_free[s], 1);
+      mbar_init(&stage_full[s], 128);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -603,17 +614,20 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           if (!wait_ack()) { ok = false; break; }
           LA2_TRACE_POINT(2, m);
           const uint32_t ob = m % CF::NOB;
-          const uint32_t tO = tmem + CF::COL_O + ob * 128;
+          const uint32_t tO = tmem + CF::COL_O + ob * CF::O_COLS;
           if (!wait_w(&o_empty[ob], ((m / CF::NOB) & 1) ^ 1, 116)) { ok = false; break; }
           LA2_TRACE_POINT(13, m);
           tc_fence_after();
           if (needs_snap) {
-            const uint64_t a = dKm + ((sQ0 + qslot(m, g) * CF::QTILE) >> 4);
-            const uint64_t b = dSnap + ((sS0 + sb * CF::SNAP) >> 4);
+            const uint64_t q = dKm + ((sQ0 + qslot(m, g) * CF::QTILE) >> 4);
+            const uint64_t kv = dSnap + ((sS0 + sb * CF::SNAP) >> 4);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               const uint32_t off = ((kk >> 2) * BK * 128 + (kk & 3) * 32) >> 4;
-              mma_bf16_ss_warp(tO, a + off, b + kk * (2048 >> 4), CF::ID_QKV, kk > 0);
+              if constexpr (CF::OT)  // O^T += KV^T Q^T: A = snapshot (MN-major), B = Q (K-major)
+                mma_bf16_ss_warp(tO, kv + kk * (2048 >> 4), q + off, CF::ID_QKV, kk > 0);
+              else
+                mma_bf16_ss_warp(tO, q + off, kv + kk * (2048 >> 4), CF::ID_QKV, kk > 0);
             }
             mma_commit_warp(&snap_free[sb]);
             ++sn;
@@ -635,13 +649,17 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
               mma_bf16_ts_warp(tO, tmem + CF::COL_P + kk * 8, b + kk * (2048 >> 4), CF::ID_PV,
                                (needs_snap || kk > 0) ? 1u : 0u);
           } else {
-            const uint64_t a = dKm + ((sP0 + pb * CF::PTILE) >> 4);
-            const uint64_t b = dK_mn + ((sV0 + ks * CF::VTILE) >> 4);
+            const uint64_t pp = dKm + ((sP0 + pb * CF::PTILE) >> 4);
+            const uint64_t vv = dK_mn + ((sV0 + ks * CF::VTILE) >> 4);
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk) {
               const uint32_t off = ((kk >> 2) * BK * 128 + (kk & 3) * 32) >> 4;
-              mma_bf16_ss_warp(tO, a + off, b + kk * (2048 >> 4), CF::ID_PV,
-                          (needs_snap || kk > 0) ? 1u : 0u);
+              if constexpr (CF::OT)  // O^T += V^T P^T: A = V (MN-major), B = P (K-major)
+                mma_bf16_ss_warp(tO, vv + kk * (2048 >> 4), pp + off, CF::ID_PV,
+                                 (needs_snap || kk > 0) ? 1u : 0u);
+              else
+                mma_bf16_ss_warp(tO, pp + off, vv + kk * (2048 >> 4), CF::ID_PV,
+                                 (needs_snap || kk > 0) ? 1u : 0u);
             }
           }
           mma_commit_warp(&o_full[ob]);
@@ -844,10 +862,60 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       while (it.next(st)) {
         if (st.pre) continue;
         const uint32_t ob = m % CF::NOB;
-        const uint32_t tO = tmem + CF::COL_O + ob * 128 + lane_off;
+        const uint32_t tO = tmem + CF::COL_O + ob * CF::O_COLS + lane_off;
         if (!__all_sync(0xffffffffu, wait_bar(&o_full[ob], (m / CF::NOB) & 1, lim, abort_flag, 140))) break;
         if (threadIdx.x % 128 == 0) LA2_TRACE_POINT(11, m);
         tc_fence_after();
+        if constexpr (CF::OT) {
+          // Thread (w4, lane) holds column e = 32 w4 + lane of O for the BK rows of
+          // the block (TMEM lane e, one column per row). It writes them into the
+          // staging tile in the TMA layout (128B-swizzled 64-column panels, rows =
+          // tokens); thread 0 then stores the whole tile.
+          // The four epilogue warps meet on mbarriers (bounded waits, so an
+          // abort elsewhere cannot leave a warp waiting for ever).
+          const int e = 32 * w4 + lane;
+          const uint32_t sb = m & 1, sph = (m >> 1) & 1;
+          uint8_t* stage = smem + CF::OFF_OST + sb * CF::OTILE;
+          if (threadIdx.x % 128 == 0) {
+            bulk_wait_group_read<1>();  // block m-2's store has read this tile
+            mbar_arrive(&stage_free[sb]);
+          }
+          if (!__all_sync(0xffffffffu, wait_bar(&stage_free[sb], sph, lim, abort_flag, 141))) break;
+          const uint32_t col_base = smem_u32(stage + (e >> 6) * BK * 128) + (e & 7) * 2;
+          const int chunk = (e & 63) >> 3;
+#pragma unroll
+          for (int c32 = 0; c32 < BK / 32; ++c32) {
+            uint32_t v[32];
+            tmem_ld32(tO + c32 * 32, v);
+            tmem_ld_wait();
+            if (c32 == BK / 32 - 1) {  // every TMEM read of O(m) is done
+              tc_fence_before();
+              mbar_arrive(&o_empty[ob]);
+            }
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int t = c32 * 32 + j;  // token row of the block
+              st_shared_u16(col_base + t * 128 + ((chunk ^ (t & 7)) << 4),
+                            bf16_bits(__uint_as_float(v[j])));
+            }
+          }
+          fence_proxy_async();
+          mbar_arrive(&stage_full[sb]);
+          if (w4 == 0) {  // the first epilogue warp stores the tile (warp-uniform wait)
+            if (!__all_sync(0xffffffffu, wait_bar(&stage_full[sb], sph, lim, abort_flag, 142))) break;
+            if (lane == 0) {
+              const int64_t y = static_cast<int64_t>(st.blk) * BK;
+#pragma unroll
+              for (int p = 0; p < DV / 64; ++p)  // rows past N are clipped by the tensor map
+                tma_store_3d(&tm_o, stage + p * BK * 128, 64 * p, static_cast<int>(y),
+                             static_cast<int>(st.bh));
+              bulk_commit_group();
+            }
+          }
+          if (threadIdx.x % 128 == 0) LA2_TRACE_POINT(12, m);
+          ++m;
+          continue;
+        }
         if constexpr (CF::TMA_STORE) {
           // Warp w4 owns rows 16*w4 .. 16*w4+15 of the block: it stages them
           // (128B-swizzled, panels of 64 columns) and stores them itself.
