@@ -170,6 +170,25 @@ static Plan make_plan_uncached(int64_t B, int64_t H, int64_t Hkv, int64_t N, int
     int64_t C = one_wave ? std::max<int64_t>(1, target / std::max<int64_t>(BHu, 1))
                          : std::max<int64_t>(1, (target + BHu - 1) / std::max<int64_t>(BHu, 1));
     C = std::min<int64_t>(C, std::max<int64_t>(1, T / 4));
+    if (p.tc && is_bwd) {
+      // The dK/dV pass runs one CTA per (sequence, chunk), in waves of `sms`
+      // CTAs: pick the chunk count whose waves times chunk length (plus a fixed
+      // cost per chunk: initial state, pipeline fill) is smallest, so that a
+      // nearly empty last wave does not stretch the pass (64 sequences x 5
+      // chunks on 148 SMs ran 3 waves where 2 chunks run in one).
+      constexpr double kChunkCost = 3.0;  // blocks
+      const int64_t G = std::max(sms, 1), cmax = std::max<int64_t>(1, T / 4);
+      double best = 0.0;
+      for (int64_t c = 1; c <= cmax; ++c) {
+        const int64_t units = BHu * c;
+        const double cost = static_cast<double>((units + G - 1) / G) *
+                            (static_cast<double>((T + c - 1) / c) + kChunkCost);
+        if (c == 1 || cost < best) {
+          best = cost;
+          C = c;
+        }
+      }
+    }
     L = ((T + C - 1) / C) * block;
   }
   L = std::max<int64_t>(L, block);
@@ -487,8 +506,10 @@ static la2_status dkdv_sm100(const void* q, const void* k, const void* v, const 
   pb.init_all = init_all ? 1 : 0;
   pb.sum_states = sum_states ? 1 : 0;
   CUtensorMap tdk = tq, tdv = tq;
-  if (sm100::BCfg<TB, D, DV>::TMA_STORE &&
-      (!make_tmap_3d(&tdk, dk, hd.BHkv, N, D, 16) || !make_tmap_3d(&tdv, dvv, hd.BHkv, N, DV, 16)))
+  using BC = sm100::BCfg<TB, D, DV>;
+  const int srows = BC::OT ? TB : 16;  // transposed accumulators: one store of the whole tile
+  if (BC::TMA_STORE &&
+      (!make_tmap_3d(&tdk, dk, hd.BHkv, N, D, srows) || !make_tmap_3d(&tdv, dvv, hd.BHkv, N, DV, srows)))
     return LA2_ERR_CUDA;
   LaunchTimer t(K_BWD_DKDV_TC, st);
   return launch_bwd_dkdv_sm100<TB>(tq, tk, tv, tdo, tdk, tdv, pb, hd.BHkv * p.C, st);

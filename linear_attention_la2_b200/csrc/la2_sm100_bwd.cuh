@@ -48,11 +48,18 @@ struct BCfg {
   static constexpr bool TMA_STORE = BK == 64;
   static constexpr int OFF_OST = OFF_SNAP + SNAP;
   static constexpr int OFF_BAR = OFF_OST + (TMA_STORE ? 2 * TILE : 0);
-  static constexpr int NBAR = 2 * NS + 12;
+  static constexpr int NBAR = 2 * NS + 13;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
+  // Bk=64: dV and dK are accumulated transposed, dV^T = U^T K^T + dO^T P and
+  // dK^T = U V^T + Q^T Pd (M = dv = d = 128 rows of the tensor datapath instead of
+  // M = Bk = 64: four of the block's products at full rate); the epilogue
+  // transposes while staging each tile for one TMA store.
+  static constexpr bool OT = BK == 64;
   // TMEM columns: U, dV, dK, S^T, A^T
-  static constexpr uint32_t COL_U = 0, COL_DV = 128, COL_DK = 256, COL_ST = 384;
-  // Bk=64: A^T gets the last 64 columns, so the next block's S^T and A^T need
+  static constexpr uint32_t COL_U = 0;
+  static constexpr uint32_t G_COLS = OT ? BK : 128;  // columns of one dV or dK accumulator
+  static constexpr uint32_t COL_DV = 128, COL_DK = COL_DV + G_COLS, COL_ST = COL_DK + G_COLS;
+  // Bk=64: A^T gets its own columns, so the next block's S^T and A^T need
   // not wait for the epilogue to read dK; Bk=128: A^T aliases dK.
   static constexpr bool AT_OWN = BK == 64;
   static constexpr uint32_t COL_AT = AT_OWN ? COL_ST + BK : COL_DK;
@@ -61,6 +68,8 @@ struct BCfg {
   static constexpr uint32_t ID_MN = make_idesc(BK, 128, false, true);   // X[K-major] * Y[MN-major]
   static constexpr uint32_t ID_KM = make_idesc(BK, 128, false, false);  // X[K-major] * Y[K-major]
   static constexpr uint32_t ID_UPD = make_idesc(D, DV, true, true);     // Q^T dO
+  static constexpr uint32_t ID_T_MK = make_idesc(128, BK, true, false);   // X[MN-major] * Y[K-major]
+  static constexpr uint32_t ID_T_KK = make_idesc(128, BK, false, false);  // X[K-major] * Y[K-major]
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
 };
 
@@ -104,8 +113,8 @@ la2_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   uint64_t* g_full = u_updated + 1;       // dK, dV complete
   uint64_t* g_empty = g_full + 1;
   uint64_t* drain = g_empty + 1;
-  uint64_t* spare = drain + 1;
-  (void)spare;
+  uint64_t* stage_free = drain + 1;       // transposing epilogue: staging tiles free
+  uint64_t* stage_full = stage_free + 1;  // transposing epilogue: staging tiles written
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + CF::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -143,6 +152,8 @@ la2_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     mbar_init(g_full, 1);
     mbar_init(g_empty, 128);
     mbar_init(drain, 1);
+    mbar_init(stage_free, 1);
+    mbar_init(stage_full, 128);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -245,11 +256,16 @@ la2_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         }
         tc_fence_after();
         if (have_u && first) {
-          // dV = K U: A = K (K-major, K = d), B[n=e][k=c] = U[c][e] (snapshot, MN-major)
+          // dV = K U: A = K (K-major, K = d), B[n=e][k=c] = U[c][e] (snapshot, MN-major);
+          // transposed: dV^T = U^T K^T, A[m=e][k=c] = U[c][e] (MN-major), B = K (K-major)
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t off = ((kk >> 2) * BK * 128 + (kk & 3) * 32) >> 4;
-            mma_bf16_ss_warp(tDV, dKm + (ak >> 4) + off, dSnapMN + (snap0 >> 4) + kk * (2048 >> 4), CF::ID_MN,
-                        kk > 0);
+            if constexpr (CF::OT)
+              mma_bf16_ss_warp(tDV, dSnapMN + (snap0 >> 4) + kk * (2048 >> 4), dKm + (ak >> 4) + off,
+                               CF::ID_T_MK, kk > 0);
+            else
+              mma_bf16_ss_warp(tDV, dKm + (ak >> 4) + off, dSnapMN + (snap0 >> 4) + kk * (2048 >> 4),
+                               CF::ID_MN, kk > 0);
           }
         }
         if (causal) {
@@ -265,10 +281,14 @@ la2_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         }
         if (have_u && first) {
           // dK = V U^T: A = V (K-major, K = dv), B[n=c][k=e] = U[c][e] (snapshot, K-major)
+          // transposed: dK^T = U V^T, A[m=c][k=e] = U[c][e] (K-major), B = V (K-major)
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t off = ((kk >> 2) * BK * 128 + (kk & 3) * 32) >> 4;
             const uint32_t soff = ((kk >> 2) * D * 128 + (kk & 3) * 32) >> 4;
-            mma_bf16_ss_warp(tDK, dKm + (av >> 4) + off, dKm + (snap0 >> 4) + soff, CF::ID_KM, kk > 0);
+            if constexpr (CF::OT)
+              mma_bf16_ss_warp(tDK, dKm + (snap0 >> 4) + soff, dKm + (av >> 4) + off, CF::ID_T_KK, kk > 0);
+            else
+              mma_bf16_ss_warp(tDK, dKm + (av >> 4) + off, dKm + (snap0 >> 4) + soff, CF::ID_KM, kk > 0);
           }
         }
         // U is updated (by every query head of the block) and no issued MMA
@@ -278,16 +298,27 @@ la2_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           if (!wait_w(p_full, s & 1, 215)) { ok = false; break; }
           tc_fence_after();
           const uint32_t acc0 = (have_u || !first) ? 1u : 0u;
-          // dV += P^T dO ; dK += Pd^T Q  (A = masked tiles, K-major, K = BK; B MN-major)
+          // dV += P^T dO ; dK += Pd^T Q  (A = masked tiles, K-major, K = BK; B MN-major);
+          // transposed: dV^T += dO^T P, dK^T += Q^T Pd (A MN-major, B = masked tiles)
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint32_t off = ((kk >> 2) * BK * 128 + (kk & 3) * 32) >> 4;
-            mma_bf16_ss_warp(tDV, dKm + (pt0 >> 4) + off, dMN + (ado >> 4) + kk * (2048 >> 4), CF::ID_MN,
-                        (acc0 || kk > 0) ? 1u : 0u);
+            const uint32_t acc = (acc0 || kk > 0) ? 1u : 0u;
+            if constexpr (CF::OT)
+              mma_bf16_ss_warp(tDV, dMN + (ado >> 4) + kk * (2048 >> 4), dKm + (pt0 >> 4) + off,
+                               CF::ID_T_MK, acc);
+            else
+              mma_bf16_ss_warp(tDV, dKm + (pt0 >> 4) + off, dMN + (ado >> 4) + kk * (2048 >> 4),
+                               CF::ID_MN, acc);
           }
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint32_t off = ((kk >> 2) * BK * 128 + (kk & 3) * 32) >> 4;
-            mma_bf16_ss_warp(tDK, dKm + (pdt0 >> 4) + off, dMN + (aq >> 4) + kk * (2048 >> 4), CF::ID_MN,
-                        (acc0 || kk > 0) ? 1u : 0u);
+            const uint32_t acc = (acc0 || kk > 0) ? 1u : 0u;
+            if constexpr (CF::OT)
+              mma_bf16_ss_warp(tDK, dMN + (aq >> 4) + kk * (2048 >> 4), dKm + (pdt0 >> 4) + off,
+                               CF::ID_T_MK, acc);
+            else
+              mma_bf16_ss_warp(tDK, dKm + (pdt0 >> 4) + off, dMN + (aq >> 4) + kk * (2048 >> 4),
+                               CF::ID_MN, acc);
           }
           mma_commit_warp(p_empty);
         }
@@ -411,6 +442,61 @@ la2_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       const int i = nblk - 1 - s;
       if (!__all_sync(0xffffffffu, wait_bar(g_full, s & 1, lim, abort_flag, 240))) break;
       tc_fence_after();
+      if constexpr (CF::OT) {
+        // Thread (w4, lane) holds column x = 32 w4 + lane of dV and of dK for the
+        // BK rows of the block (TMEM lane x, one column per row). It writes them
+        // into the two staging tiles in the TMA layout (128B-swizzled 64-column
+        // panels, rows = keys); the first warp then stores both tiles. The four
+        // warps meet on mbarriers with bounded waits.
+        const int x = 32 * w4 + lane;
+        const uint32_t ph = s & 1;
+        if (threadIdx.x % 128 == 0) {
+          bulk_wait_group_read<0>();  // the last block's stores have read the tiles
+          mbar_arrive(stage_free);
+        }
+        if (!__all_sync(0xffffffffu, wait_bar(stage_free, ph, lim, abort_flag, 241))) break;
+        const int chunk = (x & 63) >> 3;
+        for (int which = 0; which < 2; ++which) {
+          const uint32_t src = tmem + (which == 0 ? CF::COL_DV : CF::COL_DK) + lane_off;
+          const uint32_t col_base =
+              smem_u32(smem + CF::OFF_OST + which * CF::TILE + (x >> 6) * BK * 128) + (x & 7) * 2;
+#pragma unroll
+          for (int c32 = 0; c32 < BK / 32; ++c32) {
+            uint32_t v[32];
+            tmem_ld32(src + c32 * 32, v);
+            tmem_ld_wait();
+            if (which == 1 && c32 == BK / 32 - 1) {  // every TMEM read of this block is done
+              tc_fence_before();
+              mbar_arrive(g_empty);
+            }
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int t = c32 * 32 + j;  // key row of the block
+              st_shared_u16(col_base + t * 128 + ((chunk ^ (t & 7)) << 4),
+                            bf16_bits(__uint_as_float(v[j])));
+            }
+          }
+        }
+        fence_proxy_async();
+        mbar_arrive(stage_full);
+        if (w4 == 0) {
+          if (!__all_sync(0xffffffffu, wait_bar(stage_full, ph, lim, abort_flag, 242))) break;
+          if (lane == 0) {
+            // chunks end on block boundaries or at N (the tensor maps clip at N)
+            const int64_t y = t0 + static_cast<int64_t>(i) * BK;
+            for (int which = 0; which < 2; ++which) {
+              uint8_t* stage = smem + CF::OFF_OST + which * CF::TILE;
+              const CUtensorMap* map = which == 0 ? &tm_dv : &tm_dk;
+#pragma unroll
+              for (int p = 0; p < 2; ++p)
+                tma_store_3d(map, stage + p * BK * 128, 64 * p, static_cast<int>(y),
+                             static_cast<int>(bh));
+            }
+            bulk_commit_group();
+          }
+        }
+        continue;
+      }
       if constexpr (CF::TMA_STORE) {
         // Warp w4 stages its 16 rows of dV and dK (128B-swizzled 64-column
         // panels) and stores them with TMA.
