@@ -1063,6 +1063,10 @@ int la2_version(void) { return (0 << 16) | 1; }
 LA2_API int la2_trace_read(unsigned long long* dst) {
   return cudaMemcpyFromSymbol(dst, sm100::g_trace, sizeof(sm100::g_trace)) == cudaSuccess ? 0 : 1;
 }
+// Copies the per-CTA stamps (start, first main step, end) of the last traced launch (4 x 160 u64).
+LA2_API int la2_trace_cta_read(unsigned long long* dst) {
+  return cudaMemcpyFromSymbol(dst, sm100::g_trace_cta, sizeof(sm100::g_trace_cta)) == cudaSuccess ? 0 : 1;
+}
 #endif
 
 }  // extern "C"

@@ -40,16 +40,29 @@ namespace sm100 {
 
 // Optional per-step timestamps of CTA 0 (globaltimer, ns) for pipeline
 // studies: build with -DLA2_TRACE and read them with la2_trace_read().
+// Per-step events are those of CTA LA2_TRACE_CTA (default 0); LA2_TRACE_CTA_POINT
+// stamps one event per CTA (start, first main step, end).
 #ifdef LA2_TRACE
-constexpr int kTraceEvents = 16, kTraceSteps = 512;
+#ifndef LA2_TRACE_CTA
+#define LA2_TRACE_CTA 0
+#endif
+constexpr int kTraceEvents = 16, kTraceSteps = 512, kTraceCtas = 160;
 __device__ unsigned long long g_trace[kTraceEvents][kTraceSteps];
-#define LA2_TRACE_POINT(ev, idx)                                                  \
+__device__ unsigned long long g_trace_cta[4][kTraceCtas];
+#define LA2_TRACE_POINT(ev, idx)                                                             \
+  do {                                                                                       \
+    if (blockIdx.x == LA2_TRACE_CTA && (idx) < kTraceSteps) g_trace[ev][idx] = globaltimer_ns(); \
+  } while (0)
+#define LA2_TRACE_CTA_POINT(ev)                                                   \
   do {                                                                            \
-    if (blockIdx.x == 0 && (idx) < kTraceSteps) g_trace[ev][idx] = globaltimer_ns(); \
+    if (blockIdx.x < kTraceCtas) g_trace_cta[ev][blockIdx.x] = globaltimer_ns(); \
   } while (0)
 #else
 #define LA2_TRACE_POINT(ev, idx) \
   do {                           \
+  } while (0)
+#define LA2_TRACE_CTA_POINT(ev) \
+  do {                          \
   } while (0)
 #endif
 
@@ -455,6 +468,7 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   // parameters; from here on global memory is read and written.
   pdl_launch_dependents();
   pdl_wait();
+  if (threadIdx.x == 0) LA2_TRACE_CTA_POINT(0);
 
   // Range-state mode: a CTA's range (at most one per CTA) that starts inside
   // a sequence gets its initial state from the consumer warpgroups before
@@ -597,6 +611,7 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (st.pre) {
           if (!wait_w(&kv_full[ks], (g / CF::KS) & 1, 114)) { ok = false; break; }
           if (!wait_ack()) { ok = false; break; }
+          LA2_TRACE_POINT(1, g);
           tc_fence_after();
           update(ks, !st.pre_first);
           if (st.pre_last) {
@@ -605,6 +620,7 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           }
           mma_commit_warp(&kv_empty[ks]);
         } else {
+          if (m == 0 && lane == 0) LA2_TRACE_CTA_POINT(1);
           if (!s_ready && !issue_s(m, g)) { ok = false; break; }
           s_ready = false;
           const bool needs_snap = !(st.seg_first && st.init == 0);
@@ -1034,6 +1050,7 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         ++m;
       }
       if ((CF::TMA_STORE || CF::O_IN_Q) && lane == 0) bulk_wait_group<0>();  // stores done before exit
+      if (threadIdx.x % 128 == 0) LA2_TRACE_CTA_POINT(2);
     }
   }
 
@@ -1049,10 +1066,12 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
 
 // ------------------------------------------------------------------ host side
 
-// Cost model of the range split, in units of one main block (measured on a
-// loaded B200 at Bk=64: main block ~1.2 us, pre-pass block ~0.6 us; a pre-pass
-// block moves half the bytes and its loads stay latency-bound).
-constexpr double kPrepassCost = 0.5;
+// Cost model of the range split, in units of one main block. Per-step
+// timelines of a CTA with a pre-pass, all CTAs loaded (B4 H16 N2K, B2 H32 N8K,
+// B1 H32 N1K at Bk=64): a pre-pass step takes 0.42-0.54 us against 1.38-1.63 us
+// for a main step (its K and V mostly come from L2, read at the same time by
+// the CTA whose range holds those blocks), about 0.35 of a main block.
+constexpr double kPrepassCost = 0.35;
 constexpr double kRangeStateCost = 0.5;  // separate state launch, per block
 constexpr double kLaunchCost = 8.0;      // extra launch + initial-state sum, in Bk=64 main blocks
 
