@@ -1066,12 +1066,14 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
 
 // ------------------------------------------------------------------ host side
 
-// Cost model of the range split, in units of one main block. Per-step
-// timelines of a CTA with a pre-pass, all CTAs loaded (B4 H16 N2K, B2 H32 N8K,
-// B1 H32 N1K at Bk=64): a pre-pass step takes 0.42-0.54 us against 1.38-1.63 us
-// for a main step (its K and V mostly come from L2, read at the same time by
-// the CTA whose range holds those blocks), about 0.35 of a main block.
-constexpr double kPrepassCost = 0.35;
+// Cost model of the range split, in units of one main block. Under the plans
+// it produces, a pre-pass step takes 0.42-0.54 us against 1.38-1.63 us for a
+// main step (per-step timelines of a CTA with a pre-pass, all CTAs loaded, at
+// Bk=64; its K and V mostly come from L2, read at the same time by the CTA
+// whose range holds them). A cost of 0.35 picked plans with more pre-passing
+// ranges, under which the steps got dearer (B4 H16 N2K 37 -> 39 us, B1 H32 N4K
+// 49 -> 67 us per step): 0.5 stays.
+constexpr double kPrepassCost = 0.5;
 constexpr double kRangeStateCost = 0.5;  // separate state launch, per block
 constexpr double kLaunchCost = 8.0;      // extra launch + initial-state sum, in Bk=64 main blocks
 
