@@ -107,6 +107,10 @@ struct Plan {
   size_t ws_bytes = 0;
   bool ranges = false;  // persistent range split (tensor-core causal forward)
   bool dq_ranges = false;  // tensor-core causal backward: dQ through the range split
+  // Tensor-core causal backward, dK/dV in two chunks per K/V sequence, rows
+  // [0, dk_split) and [dk_split, N): the first builds its suffix state in the
+  // kernel (no suffix-state pass, no scan). 0: chunks of L rows.
+  int64_t dk_split = 0;
   RangePlan rp;
 };
 
@@ -224,6 +228,37 @@ static Plan make_plan_uncached(int64_t B, int64_t H, int64_t Hkv, int64_t N, int
     const size_t agg = p.dq_ranges && p.rp.prefix_mode == 1 ? (size_t)p.rp.R * state_bytes : 0;
     const size_t kv = p.need_states ? one : 0;
     p.ws_bytes = (p.need_states ? one : 0) + std::max(agg, kv);
+    // dK/dV split in two with the suffix state built in the kernel, when one
+    // wave holds both chunks of every K/V sequence and the model prefers it.
+    // Costs in dK/dV block steps (one query head of one block): a chunk of c
+    // blocks costs c G + kChunkCost; the suffix-state pass costs kUPass per
+    // block it reads; an in-kernel pre-pass step kPrePass. The first chunk
+    // takes the share a of the blocks that balances a + kPrePass (T - a)
+    // against T - a.
+    constexpr double kChunkCost = 3.0, kUPass = 0.38, kPrePass = 0.25;
+    const int64_t G = std::max<int64_t>(1, H / std::max<int64_t>(1, Hkv));
+    // (64-row dK/dV tiles only: their two-stage ring keeps the pre-pass loads
+    // in flight; the 128-row kernel has one stage)
+    const bool tiles64 = block == 64 || G > 1;
+    if (p.dq_ranges && tiles64 && T >= 2 && 2 * BHkv <= sms && g_chunk_len == 0) {
+      const int64_t waves = (BHkv * p.C + sms - 1) / sms;
+      const double per = static_cast<double>((T + p.C - 1) / p.C);
+      // (one chunk per sequence needs no suffix states)
+      const double cost_a = static_cast<double>(waves) *
+                            (per * G * (1.0 + (p.C > 1 ? kUPass : 0.0)) + kChunkCost);
+      const int64_t a = std::min<int64_t>(
+          T - 1, std::max<int64_t>(1, std::llround(static_cast<double>(T) * (1.0 - kPrePass) /
+                                                    (2.0 - kPrePass))));
+      const double cost_b = std::max(static_cast<double>(a) + kPrePass * static_cast<double>(T - a),
+                                     static_cast<double>(T - a)) * G + kChunkCost;
+      if (cost_b < cost_a) {
+        p.dk_split = a * block;
+        p.C = 2;
+        p.L = a * block;
+        p.need_states = false;
+        p.ws_bytes = agg;
+      }
+    }
   }
   return p;
 }
@@ -505,6 +540,7 @@ static la2_status dkdv_sm100(const void* q, const void* k, const void* v, const 
   pb.G = hd.G;
   pb.init_all = init_all ? 1 : 0;
   pb.sum_states = sum_states ? 1 : 0;
+  pb.split = causal ? p.dk_split : 0;
   CUtensorMap tdk = tq, tdv = tq;
   using BC = sm100::BCfg<TB, D, DV>;
   const int srows = BC::OT ? TB : 16;  // transposed accumulators: one store of the whole tile
@@ -539,7 +575,7 @@ static la2_status backward_sm100_bk(const void* q, const void* k, const void* v,
     s = causal_range_split<BK>(dout, v, k, dq, hd, N, s_kv, p.rp, spin, st, K_STATE_TC, K_BWD_DQ_TC);
     if (s != LA2_OK) return s;
   }
-  if (states) {
+  if (states) {  // (a dK/dV split builds its suffix state in the kernel: no states)
     if (!dq_split) {
       s = kv_chunk_states<BK>(tk, tv, s_kv, hd, N, p, spin, st);  // K^T V per chunk
       if (s != LA2_OK) return s;
@@ -756,10 +792,11 @@ la2_status la2_decode_step(const void* q, const void* k, const void* v, void* o,
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   LaunchTimer t(K_DECODE, st);
   // Four columns per lane when rows of the state, v and o allow 16-, 8- or
-  // 16-byte vector accesses.
+  // 16-byte vector accesses and every row of a thread fits in its registers.
   const dim3 block(32 * kDecodeWarps);
   cudaError_t e;
-  if (dv % 4 == 0 && is_aligned(state, 16) && is_aligned(v, 4 * es) && is_aligned(o, es)) {
+  if (dv % 4 == 0 && d <= kDecodeWarps * kRows && is_aligned(state, 16) && is_aligned(v, 4 * es) &&
+      is_aligned(o, es)) {
     const dim3 grid4((unsigned)BH, (unsigned)((dv + 127) / 128));
     if (dt == LA2_BF16)
       e = launch_pdl(decode_step_v4_kernel<__nv_bfloat16>, grid4, block, 0, st,

@@ -16,6 +16,7 @@
 namespace la2 {
 
 constexpr int kDecodeWarps = 8;
+constexpr int kRows = 128 / kDecodeWarps;  // state rows per thread at the largest d
 
 // grid (B*H, ceil(dv / 32)); block 256. Lane l of every warp owns column
 // 32*blockIdx.y + l; warp w owns state rows w, w + 8, ... The eight partial
@@ -71,7 +72,7 @@ __device__ __forceinline__ float4 load4<__nv_bfloat16>(const __nv_bfloat16* p) {
 }
 
 template <typename T>
-__global__ void __launch_bounds__(32 * kDecodeWarps)
+__global__ void __launch_bounds__(32 * kDecodeWarps, 3)
 decode_step_v4_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                       T* __restrict__ o, float* __restrict__ state, int d, int dv) {
   pdl_launch_dependents();
@@ -86,20 +87,34 @@ decode_step_v4_kernel(const T* __restrict__ q, const T* __restrict__ k, const T*
   if (j < dv) {
     const float4 vj = load4<T>(v + bh * dv + j);
     float* col = state + bh * static_cast<int64_t>(d) * dv + j;
-#pragma unroll 16  // every row of a thread in flight at d = 128
-    for (int i = w; i < d; i += kDecodeWarps) {
-      float4* p = reinterpret_cast<float4*>(col + static_cast<int64_t>(i) * dv);
-      const float ki = to_f32(kb[i]), qi = to_f32(qb[i]);
-      float4 x = *p;
-      x.x += ki * vj.x;
-      x.y += ki * vj.y;
-      x.z += ki * vj.z;
-      x.w += ki * vj.w;
-      *p = x;
-      acc.x += qi * x.x;
-      acc.y += qi * x.y;
-      acc.z += qi * x.z;
-      acc.w += qi * x.w;
+    // A group of this thread's rows is loaded before any is written back: the
+    // writes go through the same pointer, so a fused load-update-store loop
+    // would keep one row in flight per thread (d <= 128: at most kRows rows,
+    // in two groups so that three CTAs fit on an SM).
+#pragma unroll
+    for (int g = 0; g < 2; ++g) {
+      float4 x[kRows / 2];
+#pragma unroll
+      for (int t = 0; t < kRows / 2; ++t) {
+        const int i = w + (g * kRows / 2 + t) * kDecodeWarps;
+        if (i < d) x[t] = *reinterpret_cast<const float4*>(col + static_cast<int64_t>(i) * dv);
+      }
+#pragma unroll
+      for (int t = 0; t < kRows / 2; ++t) {
+        const int i = w + (g * kRows / 2 + t) * kDecodeWarps;
+        if (i < d) {
+          const float ki = to_f32(kb[i]), qi = to_f32(qb[i]);
+          x[t].x += ki * vj.x;
+          x[t].y += ki * vj.y;
+          x[t].z += ki * vj.z;
+          x[t].w += ki * vj.w;
+          *reinterpret_cast<float4*>(col + static_cast<int64_t>(i) * dv) = x[t];
+          acc.x += qi * x[t].x;
+          acc.y += qi * x[t].y;
+          acc.z += qi * x[t].z;
+          acc.w += qi * x[t].w;
+        }
+      }
     }
   }
   part[w][lane] = acc;

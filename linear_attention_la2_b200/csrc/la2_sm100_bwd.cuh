@@ -85,6 +85,11 @@ struct BwdParams {
   // 1: init_u holds the raw chunk states (no scan ran); a chunk adds up the
   // states of the later chunks of its sequence (causal) or all of them.
   int32_t sum_states;
+  // Causal, C = 2: chunk 0 is rows [0, split), chunk 1 rows [split, N), and
+  // chunk 0 builds U itself by a pre-pass over the blocks of chunk 1 (U +=
+  // Q^T dO, Q and dO loads only) before its own blocks: no suffix states are
+  // read (init_u unused). 0: chunks of L rows, U from init_u.
+  int64_t split;
 };
 
 template <int BK, int D, int DV>
@@ -120,14 +125,24 @@ la2_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
 
   const int64_t unit = blockIdx.x;
   const int64_t bh = unit / prm.C, c = unit % prm.C;  // bh: the K/V sequence
-  const int64_t t0 = c * prm.L, t1 = min(prm.N, t0 + prm.L);
-  const int nblk = static_cast<int>((t1 - t0 + BK - 1) / BK);
   const bool causal = prm.causal != 0;
+  const bool split = causal && prm.split > 0;
+  const int64_t t0 = split ? (c == 0 ? 0 : prm.split) : c * prm.L;
+  const int64_t t1 = split ? (c == 0 ? prm.split : prm.N) : min(prm.N, t0 + prm.L);
+  const int nblk = static_cast<int>((t1 - t0 + BK - 1) / BK);
   // query heads walked per block (the non-causal form needs only K, V and U)
   const int gq = causal && prm.G > 1 ? prm.G : 1;
   const int nsteps = nblk * gq;
   const int64_t q0 = q_seq0(bh, prm.H, prm.G);
-  const bool has_init = !causal || (prm.init_u && (c + 1 < prm.C || prm.init_all));
+  // In-kernel suffix state: chunk 0 of a split walks the later blocks first
+  // (t1 is a multiple of BK there), from the last block of the sequence down.
+  // Its steps need only Q and dO: two of them share a stage of the ring
+  // (tiles 0, 3 and 1, 2), so twice as many of their loads are in flight.
+  const int64_t nblk_seq = (prm.N + BK - 1) / BK;
+  const int npre = split && c == 0 ? static_cast<int>(nblk_seq - t1 / BK) * gq : 0;
+  const int npair = (npre + 1) / 2;  // ring steps of the pre-pass
+  const bool has_init = !causal || (!split && prm.init_u && (c + 1 < prm.C || prm.init_all));
+  const bool has_u0 = has_init || npre > 0;  // U is non-zero before the first own block
   const float* init = nullptr;
   // states added at init: one scanned slot, or the raw states of chunks
   // [c0, C) of the sequence (the later chunks, or all of them without the mask)
@@ -189,12 +204,28 @@ la2_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     if (lane == 0) {
       int issued = 0;
       bool ok = true;
-      for (int s = 0; s < nsteps && ok; ++s) {
-        const int i = nblk - 1 - s / gq;  // reverse block order
-        const int hq = static_cast<int>(q0 + s % gq);  // query sequence of Q and dO
-        const int row = static_cast<int>(t0 + static_cast<int64_t>(i) * BK);
+      for (int s = 0; s < npair + nsteps && ok; ++s) {
         const int slot = s % CF::NS;
         if (!wait_bar(&st_empty[slot], ((s / CF::NS) & 1) ^ 1, lim, abort_flag, 201)) { ok = false; break; }
+        if (s < npair) {  // suffix pre-pass: Q and dO of one or two later (block, head) steps
+          const int n2 = min(2, npre - 2 * s);
+          mbar_expect_tx(&st_full[slot], 2 * n2 * CF::TILE);
+          for (int e = 0; e < n2; ++e) {
+            const int sp = 2 * s + e;
+            const int hq = static_cast<int>(q0 + sp % gq);
+            const int row = static_cast<int>((nblk_seq - 1 - sp / gq) * BK);
+            const int tq = e == 0 ? 0 : 1, tdo = e == 0 ? 3 : 2;
+            for (int p = 0; p < 2; ++p) {
+              tma_load_3d(tile(slot, tq) + p * BK * 128, &tm_q, &st_full[slot], 64 * p, row, hq);
+              tma_load_3d(tile(slot, tdo) + p * BK * 128, &tm_do, &st_full[slot], 64 * p, row, hq);
+            }
+          }
+          ++issued;
+          continue;
+        }
+        const int sm = s - npair;
+        const int hq = static_cast<int>(q0 + sm % gq);  // query sequence of Q and dO
+        const int row = static_cast<int>(t0 + static_cast<int64_t>(nblk - 1 - sm / gq) * BK);  // reverse order
         mbar_expect_tx(&st_full[slot], causal ? 4 * CF::TILE : 2 * CF::TILE);
         const CUtensorMap* maps[4] = {&tm_q, &tm_k, &tm_v, &tm_do};
         for (int t = 0; t < 4; ++t) {
@@ -223,17 +254,36 @@ la2_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       const uint32_t snap0 = smem_u32(sSnap), pt0 = smem_u32(sPT), pdt0 = smem_u32(sPdT);
       int snap_ph = 0;
       bool ok = true;
-      for (int s = 0; s < nsteps && ok; ++s) {
+      // Suffix pre-pass: U = sum of Q^T dO over the later blocks (fresh U on
+      // the first step); its completion is the first u_updated phase.
+      for (int s = 0; s < npair && ok; ++s) {
         const int slot = s % CF::NS;
+        if (!wait_w(&st_full[slot], (s / CF::NS) & 1, 217)) { ok = false; break; }
+        tc_fence_after();
+        const int n2 = min(2, npre - 2 * s);
+        for (int e = 0; e < n2; ++e) {
+          const uint32_t aq = smem_u32(tile(slot, e == 0 ? 0 : 1));
+          const uint32_t ado = smem_u32(tile(slot, e == 0 ? 3 : 2));
+          for (int kk = 0; kk < BK / 16; ++kk)
+            mma_bf16_ss_warp(tU, dMN + (aq >> 4) + kk * (2048 >> 4), dMN + (ado >> 4) + kk * (2048 >> 4),
+                             CF::ID_UPD, (s > 0 || e > 0 || kk > 0) ? 1u : 0u);
+        }
+        if (s == npair - 1) mma_commit_warp(u_updated);
+        mma_commit_warp(&st_empty[slot]);
+      }
+      for (int sm = 0; sm < nsteps && ok; ++sm) {
+        const int s = sm;                       // own-block step (mask and P barriers)
+        const int gs = npair + sm;              // step of the stage ring
+        const int slot = gs % CF::NS;
         const int blk = s / gq;                 // block counter (reverse order)
         const bool first = s % gq == 0;         // first query head of the block
         const bool last = s % gq == gq - 1;     // last query head of the block
         const uint32_t aq = smem_u32(tile(slot, 0)), ak = smem_u32(tile(slot, 1));
         const uint32_t av = smem_u32(tile(slot, 2)), ado = smem_u32(tile(slot, 3));
-        if (!wait_w(&st_full[slot], (s / CF::NS) & 1, 210)) { ok = false; break; }
+        if (!wait_w(&st_full[slot], (gs / CF::NS) & 1, 210)) { ok = false; break; }
         // A^T aliasing dK: the epilogue must have read the last block's dK
         if (!CF::AT_OWN && !wait_w(g_empty, (blk & 1) ^ 1, 211)) { ok = false; break; }
-        const bool have_u = blk > 0 || has_init;
+        const bool have_u = blk > 0 || has_u0;
         if (causal) {
           if (!wait_w(s_read, (s & 1) ^ 1, 212)) { ok = false; break; }
           tc_fence_after();
@@ -416,9 +466,27 @@ la2_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       tc_fence_before();
       mbar_arrive(snap_full);
     }
-    if (causal) {
+    bool ok_pre = true;
+    if (npre > 0) {  // U from the suffix pre-pass: snapshot it once it is complete
+      ok_pre = __all_sync(0xffffffffu, wait_bar(u_updated, 0, lim, abort_flag, 231));
+      if (ok_pre) {
+        tc_fence_after();
+#pragma unroll
+        for (int c32 = 0; c32 < DV / 32; ++c32) {
+          uint32_t v[32];
+          tmem_ld32(tU + c32 * 32, v);
+          tmem_ld_wait();
+          put_row(v, c32 * 32);
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        mbar_arrive(snap_full);
+      }
+    }
+    if (causal && ok_pre) {
+      const int ph0 = npre > 0 ? 1 : 0;  // the pre-pass took the first u_updated phase
       for (int s = 0; s + 1 < nblk; ++s) {
-        if (!__all_sync(0xffffffffu, wait_bar(u_updated, s & 1, lim, abort_flag, 230))) break;
+        if (!__all_sync(0xffffffffu, wait_bar(u_updated, (s + ph0) & 1, lim, abort_flag, 230))) break;
         // the snapshot buffer is free: every MMA reading it was issued before
         // the update whose completion u_updated reports
         tc_fence_after();

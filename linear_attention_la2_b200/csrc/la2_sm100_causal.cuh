@@ -1066,14 +1066,15 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
 
 // ------------------------------------------------------------------ host side
 
-// Cost model of the range split, in units of one main block. Under the plans
-// it produces, a pre-pass step takes 0.42-0.54 us against 1.38-1.63 us for a
-// main step (per-step timelines of a CTA with a pre-pass, all CTAs loaded, at
-// Bk=64; its K and V mostly come from L2, read at the same time by the CTA
-// whose range holds them). A cost of 0.35 picked plans with more pre-passing
-// ranges, under which the steps got dearer (B4 H16 N2K 37 -> 39 us, B1 H32 N4K
-// 49 -> 67 us per step): 0.5 stays.
-constexpr double kPrepassCost = 0.5;
+// Cost model of the range split, in units of one main block. Under load a
+// pre-pass step takes 0.42-0.54 us against 1.38-1.63 us for a main step
+// (per-step timelines of a CTA with a pre-pass at Bk=64; its K and V mostly
+// come from L2, read at the same time by the CTA whose range holds them). A
+// sweep of the cost on B4 H16 N2K, B1 H32 N1K and N4K (Bk 64 and 128) put the
+// best single value at 0.4: 0.5 kept ranges that start at block 0 too long
+// (N1K Bk=64: 16.4 -> 14.5 us per step at 0.4), while 0.35 and below split
+// B4 H16 N2K into ranges that span two sequences (35.3 -> 36.5 us).
+constexpr double kPrepassCost = 0.4;
 constexpr double kRangeStateCost = 0.5;  // separate state launch, per block
 constexpr double kLaunchCost = 8.0;      // extra launch + initial-state sum, in Bk=64 main blocks
 

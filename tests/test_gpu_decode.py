@@ -97,3 +97,26 @@ def test_decode_step_full_workload(la2):
     ref_o, ref_s = oracle.decode_step(q, k, v, s0)
     assert oracle.relative_frobenius(o.cpu().double().numpy(), ref_o) <= 1e-2
     assert oracle.relative_frobenius(state.cpu().double().numpy(), ref_s) <= 1e-6
+
+
+@pytest.mark.parametrize("dt,d,dv", [("f32", 160, 36), ("f32", 128, 64), ("bf16", 96, 128),
+                                     ("bf16", 200, 128)])
+def test_decode_step_from_random_state(la2, dt, d, dv):
+    """Decode steps from a random fp32 state, without a prefill: d above 128 runs
+    the one-column-per-lane kernel, d <= 128 with dv % 4 == 0 the kernel that holds
+    all of a thread's state rows in registers."""
+    B, H, T = 3, 2, 4
+    g = torch.Generator().manual_seed(d + dv)
+    tdt = torch.bfloat16 if dt == "bf16" else torch.float32
+    q, k, v = ((torch.randn((B, H, T, n), generator=g) / np.sqrt(d)).to(tdt) for n in (d, d, dv))
+    s = torch.randn((B, H, d, dv), generator=g) * 0.1
+    state = s.cuda()
+    outs = [la2.decode_step(q[:, :, t].cuda(), k[:, :, t].cuda(), v[:, :, t].cuda(), state)
+            for t in range(T)]
+    torch.cuda.synchronize()
+    la2.check()
+    tol = 1e-2 if dt == "bf16" else 1e-5
+    for t in range(T):
+        ref_o, s = oracle.decode_step(q[:, :, t], k[:, :, t], v[:, :, t], s)
+        assert oracle.relative_frobenius(outs[t].cpu().double().numpy(), ref_o) <= tol
+    assert oracle.relative_frobenius(state.cpu().double().numpy(), s) <= 1e-6
