@@ -1076,7 +1076,11 @@ la2_causal_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
 // B4 H16 N2K into ranges that span two sequences (35.3 -> 36.5 us).
 constexpr double kPrepassCost = 0.4;
 constexpr double kRangeStateCost = 0.5;  // separate state launch, per block
-constexpr double kLaunchCost = 8.0;      // extra launch + initial-state sum, in Bk=64 main blocks
+// Extra launch + initial-state sum, in Bk=64 main blocks: fitted so that the
+// plans follow measured winners (B1 H32 N4K Bk=64: range states over ranges
+// aligned to the sequences 43.9 us, pre-pass 46.5 us per step; B4 H16 N2K,
+// B1 H32 N1K and B2 H32 N8K: pre-pass, 17-50 % faster than range states).
+constexpr double kLaunchCost = 4.0;
 
 struct RangePlan {
   int R = 0;
@@ -1087,7 +1091,9 @@ struct RangePlan {
 };
 
 // Greedy split of `total` tasks into ranges of cost <= tau; a range that
-// starts at block b of a sequence pays b pre-pass blocks. Returns the count.
+// starts at block b of a sequence pays b pre-pass blocks. Returns the count,
+// or kMaxRanges + 1 when tau is infeasible (a range would have to start where
+// its pre-pass alone leaves no room for one main block).
 inline int greedy_ranges(int64_t total, int64_t T, double tau, std::vector<int64_t>* starts) {
   int64_t f = 0;
   int n = 0;
@@ -1095,7 +1101,8 @@ inline int greedy_ranges(int64_t total, int64_t T, double tau, std::vector<int64
   while (f < total) {
     const int64_t blk = f % T;
     const double budget = tau - static_cast<double>(blk) * kPrepassCost;
-    int64_t take = budget >= 1.0 ? static_cast<int64_t>(budget) : 1;
+    if (budget < 1.0) return sm100::kMaxRanges + 1;
+    const int64_t take = static_cast<int64_t>(budget);
     if (starts) starts->push_back(f);
     f = std::min(total, f + take);
     ++n;
@@ -1131,8 +1138,20 @@ inline RangePlan plan_ranges(int64_t BH, int64_t N, int block, int sms, int64_t 
   std::vector<int64_t> pre_starts;
   const int n_pre = greedy_ranges(total, T, hi, &pre_starts);
   const double tau_pre = hi;
-  // (b) range-state plan: equal split; a separate launch computes range states
-  const int n_eq = static_cast<int>(std::min<int64_t>(G, total));
+  // (b) range-state plan: equal split; a separate launch computes range states.
+  // With a few ranges per sequence (at most 8) the ranges are aligned to the
+  // sequences (the same count in each), when that leaves at least 3/4 of the
+  // SMs busy: no range then holds the end of one sequence and the start of
+  // the next, and every sequence's last range (1/k of the K/V) needs no
+  // state. Measured against the split over all SMs: B1 H32 N4K and N16K at
+  // Bk=128 2-4 % faster, N64K Bk=128 2.6 %, N64K Bk=64 unchanged. With many
+  // ranges per sequence the saving is small and the SMs left idle cost more
+  // (B1 H8 N512K: 144 ranges up to 3 % slower than 148 under the power cap).
+  int n_eq = static_cast<int>(std::min<int64_t>(G, total));
+  if (BH <= G && G / BH <= 8) {
+    const int64_t aligned = BH * (G / BH);
+    if (4 * aligned >= 3 * static_cast<int64_t>(G) && aligned <= total) n_eq = static_cast<int>(aligned);
+  }
   // the launch cost is a time: in units of this block size's main block
   const double launch = kLaunchCost * 64.0 / static_cast<double>(block);
   const double tau_eq = static_cast<double>(total) / n_eq * (1.0 + kRangeStateCost) + launch;
