@@ -194,7 +194,10 @@ struct StepIter {
       }
     }
     s.bh = pre_bh;
-    s.blk = pre_blk;
+    // The state launch walks each range from its last block down: when it
+    // ends, L2 still holds the K and V it read last, the first blocks of the
+    // ranges, which the main launch reads first. (The state is a sum.)
+    s.blk = KIND == KIND_AGG ? pre_lo + pre_end - 1 - pre_blk : pre_blk;
     s.range = r;
     s.pre = 1;
     s.pre_first = pre_blk == pre_lo;
