@@ -665,7 +665,8 @@ def bench_decode(args, dev, la2, world, hbm, peak_kind):
                                "fp32 state", "B": B, "H": H, "d": d, "dv": dv,
                    "l2": f"state {B * H * d * dv * 4 / 1e6:.0f} MB > L2"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved / hbm, "traffic": None, "kernel": "la2_decode_step",
+                     "frac": achieved / hbm, "traffic": recorded_traffic("la2_decode_step", c["name"]),
+                     "kernel": "la2_decode_step",
                      "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)"},
         "gpu_launches": sum(v["launches"] for v in per_kernel.values()) * args.steps
         // max(1, profiled_steps), "kernels": per_kernel,
