@@ -37,6 +37,18 @@ heads (a layout of the same op: each query head reads the K/V head of its group)
 ``forward_from_state`` / ``backward_from_states`` the oracle of one part of a
 sequence whose other parts are summarised by KV states (sequence parallelism).
 
+Decay (``forward_decay``, ``backward_decay``, ``recurrent_forward_decay``) is a
+reading, not an article formula: the article has no decay, and the only nearby
+text on the pages is a one-line mention of data-dependent gating (gated linear
+attention). The reading is the plainest decayed form of the same op: per head h
+a rate ``lam_h`` in [0, 1] multiplies the KV state before each token,
+``KV_t = lam KV_{t-1} + k_t^T v_t``, i.e. the causal mask becomes
+``D[t, s] = lam^(t - s)`` for ``s <= t``. It reduces to the article's op at
+``lam = 1``. Its pins are mathematical (``tests/test_oracle_decay.py``): equality
+of the left product and the recurrence, ``lam = 1`` against ``forward``,
+``lam = 0`` against its closed form, brute force on integers at ``lam = 1/2``,
+exact directional derivatives.
+
 Parity status: every function here is pinned by ``tests/test_oracle.py``
 (brute force on tiny integer inputs, closed forms, RNN-form equality, block-size
 invariance, associativity, exact directional derivatives, autograd).
@@ -203,6 +215,87 @@ def recurrent_forward(q, k, v) -> np.ndarray:
             kv = np.zeros((d, v.shape[3]))
             for t in range(N):
                 kv += np.outer(k[b, h, t], v[b, h, t])
+                out[b, h, t] = q[b, h, t] @ kv
+    return out
+
+
+def _decay_rates(lam, H: int) -> np.ndarray:
+    lam = np.asarray(_f64(lam), dtype=np.float64).reshape(-1)
+    if lam.shape != (H,):
+        raise ValueError("one decay rate per head expected")
+    return lam
+
+
+def _decay_matrix(lam: float, rows: np.ndarray, N: int) -> np.ndarray:
+    """``D[t, s] = lam^(t - s)`` for ``s <= t``, else 0 (rows t given, all s)."""
+    gap = rows[:, None] - np.arange(N)[None, :]
+    return np.where(gap >= 0, lam ** np.maximum(gap, 0), 0.0)
+
+
+def forward_decay(q, k, v, lam) -> np.ndarray:
+    """Decayed causal left product ``O = ((Q K^T) ⊙ D) V`` for every (b, h).
+
+    Row t of O is ``sum_{s<=t} lam_h^(t-s) (q_t . k_s) v_s`` with one rate
+    ``lam_h`` per head (a reading: see the module notes).
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    _check(q, k, v)
+    B, H, N, _ = q.shape
+    lam = _decay_rates(lam, H)
+    out = np.empty(q.shape[:3] + (v.shape[3],), dtype=np.float64)
+    for b in range(B):
+        for h in range(H):
+            K, V = k[b, h], v[b, h]
+            for r0 in range(0, N, ROW_GROUP):
+                r1 = min(N, r0 + ROW_GROUP)
+                S = (q[b, h, r0:r1] @ K.T) * _decay_matrix(lam[h], np.arange(r0, r1), N)
+                out[b, h, r0:r1] = S @ V
+    return out
+
+
+def backward_decay(q, k, v, do, lam):
+    """Closed-form gradients of ``L = <dO, O>`` for ``O = ((Q K^T) ⊙ D) V``.
+
+    With ``P = (Q K^T) ⊙ D`` and ``dP = (dO V^T) ⊙ D``:
+    ``dQ = dP K``, ``dK = dP^T Q``, ``dV = P^T dO``.
+    """
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    _check(q, k, v)
+    B, H, N, _ = q.shape
+    lam = _decay_rates(lam, H)
+    dq, dk, dvv = np.empty_like(q), np.empty_like(k), np.empty_like(v)
+    for b in range(B):
+        for h in range(H):
+            Q, K, V, dO = q[b, h], k[b, h], v[b, h], do[b, h]
+            dk_acc, dv_acc = np.zeros_like(K), np.zeros_like(V)
+            for r0 in range(0, N, ROW_GROUP):
+                r1 = min(N, r0 + ROW_GROUP)
+                D = _decay_matrix(lam[h], np.arange(r0, r1), N)
+                P = (Q[r0:r1] @ K.T) * D
+                dP = (dO[r0:r1] @ V.T) * D
+                dq[b, h, r0:r1] = dP @ K
+                dk_acc += dP.T @ Q[r0:r1]
+                dv_acc += P.T @ dO[r0:r1]
+            dk[b, h] = dk_acc
+            dvv[b, h] = dv_acc
+    return dq, dk, dvv
+
+
+def recurrent_forward_decay(q, k, v, lam) -> np.ndarray:
+    """RNN form of the decayed op: ``KV_t = lam KV_{t-1} + k_t^T v_t``, ``o_t = q_t KV_t``.
+
+    A pin for ``forward_decay`` only (one token at a time, zero initial state).
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    _check(q, k, v)
+    B, H, N, d = q.shape
+    lam = _decay_rates(lam, H)
+    out = np.empty(q.shape[:3] + (v.shape[3],))
+    for b in range(B):
+        for h in range(H):
+            kv = np.zeros((d, v.shape[3]))
+            for t in range(N):
+                kv = lam[h] * kv + np.outer(k[b, h, t], v[b, h, t])
                 out[b, h, t] = q[b, h, t] @ kv
     return out
 
