@@ -174,6 +174,35 @@ LA2_API la2_status la2_backward_sp(const void *q, const void *k, const void *v, 
                                    la2_stream_t stream);
 
 /*
+ * Decayed causal form (a reading: the article gives no decay; its pages mention
+ * data-dependent gating only, for gated linear attention). Per query head h a
+ * rate lambda[h] multiplies the KV state before each token:
+ *   KV_t = lambda KV_{t-1} + k_t^T v_t,   o_t = q_t KV_t,
+ * i.e. o = ((q k^T) ⊙ D) v with D[t][s] = lambda^(t-s) for s <= t, 0 above;
+ * lambda = 1 is la2_forward's causal op. `lambda`: H fp32 rates in [0, 1],
+ * device memory, 4-byte aligned, read only (powers are taken with powf; rates
+ * outside [0, 1] are not rejected and follow the same formula). One K/V head per
+ * query head; q, k, v, o, dout, dq, dk, dvv as for la2_forward / la2_backward
+ * (causal only). Runs on CUDA cores for every shape and dtype la2_forward takes,
+ * with the shared-memory limits of that path: bf16 d = dv = 128 at block 128
+ * fits the forward but not the backward (LA2_ERR_UNSUPPORTED). Workspace:
+ * la2_workspace_size_decay. Other conventions and errors as for la2_forward /
+ * la2_backward; `lambda` must not overlap the outputs.
+ */
+LA2_API size_t la2_workspace_size_decay(int64_t B, int64_t H, int64_t N, int64_t d, int64_t dv,
+                                        int block, la2_dtype dt, int is_backward);
+LA2_API la2_status la2_forward_decay(const void *q, const void *k, const void *v, void *o,
+                                     const float *lambda, int64_t B, int64_t H, int64_t N,
+                                     int64_t d, int64_t dv, int block, la2_dtype dt,
+                                     void *workspace, size_t workspace_bytes, la2_stream_t stream);
+LA2_API la2_status la2_backward_decay(const void *q, const void *k, const void *v,
+                                      const void *dout, void *dq, void *dk, void *dvv,
+                                      const float *lambda, int64_t B, int64_t H, int64_t N,
+                                      int64_t d, int64_t dv, int block, la2_dtype dt,
+                                      void *workspace, size_t workspace_bytes,
+                                      la2_stream_t stream);
+
+/*
  * Synchronises `stream`, then reports and clears the device-side error word
  * that kernels set when a bounded wait gives up (LA2_ERR_TIMEOUT), or
  * LA2_ERR_CUDA if the stream holds a CUDA error. LA2_OK otherwise.

@@ -328,21 +328,23 @@ struct Ext {
 template <typename T>
 static la2_status run_chunk_states(const void* a, const void* b, float* out, int64_t nseq, int64_t N,
                                    int da, int db, const Plan& p, cudaStream_t st, int32_t H = 1,
-                                   int32_t G = 1, int group = 1) {
+                                   int32_t G = 1, int group = 1, const float* lam = nullptr,
+                                   int decay = 0) {
   const size_t smem = chunk_state_smem(da, db);
   LaunchTimer t(K_CHUNK_STATE, st);
   chunk_state_kernel<T><<<(unsigned)(nseq * p.C), kSimtThreads, smem, st>>>(
-      static_cast<const T*>(a), static_cast<const T*>(b), out, N, da, db, p.L, p.C, H, G, group);
+      static_cast<const T*>(a), static_cast<const T*>(b), out, N, da, db, p.L, p.C, H, G, group,
+      lam, decay);
   return launch_status();
 }
 
 static la2_status run_scan(float* s, int64_t nseq, int nel, const Plan& p, int mode, cudaStream_t st,
                            const float* ext = nullptr, int64_t n_ext = 0, int d = 0, int dv = 0,
-                           int f4_layout = 0) {
+                           int f4_layout = 0, const float* lam = nullptr, int H = 1) {
   dim3 grid((nel + kSimtThreads - 1) / kSimtThreads, (unsigned)nseq);
   LaunchTimer t(K_CHUNK_SCAN, st);
   if (launch_pdl(chunk_scan_kernel, grid, dim3(kSimtThreads), 0, st, s, p.C, nel, mode,
-                 n_ext > 0 ? ext : nullptr, n_ext, nseq, d, dv, f4_layout) != cudaSuccess)
+                 n_ext > 0 ? ext : nullptr, n_ext, nseq, d, dv, f4_layout, lam, H, p.L) != cudaSuccess)
     return LA2_ERR_CUDA;
   return launch_status();
 }
@@ -350,15 +352,15 @@ static la2_status run_scan(float* s, int64_t nseq, int nel, const Plan& p, int m
 template <typename T>
 static la2_status forward_simt(const void* q, const void* k, const void* v, void* o, const Heads& hd,
                                int64_t N, int d, int dv, int causal, int block, float* states,
-                               const Plan& p, cudaStream_t st) {
-  const size_t smem = fwd_simt_smem(d, dv, block, sizeof(T));
+                               const Plan& p, cudaStream_t st, const float* lam = nullptr) {
+  const size_t smem = fwd_simt_smem(d, dv, block, sizeof(T), lam != nullptr);
   if (cudaFuncSetAttribute(fwd_simt_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
     return LA2_ERR_CUDA;
   LaunchTimer t(K_FWD_SIMT, st);
   fwd_simt_kernel<T><<<(unsigned)(hd.BH * p.C), kSimtThreads, smem, st>>>(
       static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v),
-      static_cast<T*>(o), states, N, d, dv, block, p.L, p.C, causal, hd.H, hd.G);
+      static_cast<T*>(o), states, N, d, dv, block, p.L, p.C, causal, hd.H, hd.G, lam);
   return launch_status();
 }
 
@@ -366,9 +368,9 @@ template <typename T>
 static la2_status backward_simt(const void* q, const void* k, const void* v, const void* dout,
                                 void* dq, void* dk, void* dvv, const Heads& hd, int64_t N, int d,
                                 int dv, int causal, int block, float* s_kv, float* s_u,
-                                const Plan& p, cudaStream_t st) {
-  const size_t smem_q = bwd_dq_simt_smem(d, dv, block, sizeof(T));
-  const size_t smem_kv = bwd_dkdv_simt_smem(d, dv, block, sizeof(T));
+                                const Plan& p, cudaStream_t st, const float* lam = nullptr) {
+  const size_t smem_q = bwd_dq_simt_smem(d, dv, block, sizeof(T), lam != nullptr);
+  const size_t smem_kv = bwd_dkdv_simt_smem(d, dv, block, sizeof(T), lam != nullptr);
   if (cudaFuncSetAttribute(bwd_dq_simt_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem_q) != cudaSuccess ||
       cudaFuncSetAttribute(bwd_dkdv_simt_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -378,7 +380,7 @@ static la2_status backward_simt(const void* q, const void* k, const void* v, con
     LaunchTimer t(K_BWD_DQ_SIMT, st);
     bwd_dq_simt_kernel<T><<<(unsigned)(hd.BH * p.C), kSimtThreads, smem_q, st>>>(
         static_cast<const T*>(k), static_cast<const T*>(v), static_cast<const T*>(dout),
-        static_cast<T*>(dq), s_kv, N, d, dv, block, p.L, p.C, causal, hd.H, hd.G);
+        static_cast<T*>(dq), s_kv, N, d, dv, block, p.L, p.C, causal, hd.H, hd.G, lam);
   }
   la2_status s = launch_status();
   if (s != LA2_OK) return s;
@@ -387,7 +389,7 @@ static la2_status backward_simt(const void* q, const void* k, const void* v, con
     bwd_dkdv_simt_kernel<T><<<(unsigned)(hd.BHkv * p.C), kSimtThreads, smem_kv, st>>>(
         static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v),
         static_cast<const T*>(dout), static_cast<T*>(dk), static_cast<T*>(dvv), s_u, N, d, dv,
-        block, p.L, p.C, causal, hd.H, hd.G);
+        block, p.L, p.C, causal, hd.H, hd.G, lam);
   }
   return launch_status();
 }
@@ -1003,9 +1005,139 @@ static la2_status backward_impl(const void* q, const void* k, const void* v, con
                                     block, s_kv, s_u, p, st);
 }
 
+// ------------------------------------------------------------------ decayed form
+
+// CUDA-core plan of the decayed form: chunks of L rows (about two units per
+// SM, at least four blocks a chunk), chunk states decayed to a chunk edge and
+// their decayed scan when a sequence has more than one chunk.
+static Plan plan_decay(int64_t B, int64_t H, int64_t N, int64_t d, int64_t dv, int block,
+                       bool is_bwd, int sms) {
+  Plan p;
+  const int64_t BH = B * H, T = (N + block - 1) / block;
+  int64_t L;
+  if (g_chunk_len > 0) {
+    L = ((g_chunk_len + block - 1) / block) * block;
+  } else {
+    int64_t C = std::max<int64_t>(1, (2 * (int64_t)std::max(sms, 1) + BH - 1) / std::max<int64_t>(BH, 1));
+    C = std::min<int64_t>(C, std::max<int64_t>(1, T / 4));
+    L = ((T + C - 1) / C) * block;
+  }
+  p.L = std::max<int64_t>(L, block);
+  p.C = std::max<int64_t>(1, (N + p.L - 1) / p.L);
+  p.need_states = p.C > 1;
+  p.ws_bytes = p.need_states ? (size_t)BH * p.C * d * dv * sizeof(float) * (is_bwd ? 2 : 1) : 0;
+  return p;
+}
+
+static la2_status check_decay_shape(int64_t B, int64_t H, int64_t N, int64_t d, int64_t dv,
+                                    int block, la2_dtype dt, bool is_bwd) {
+  const la2_status s = check_shape(B, H, N, d, dv, 1, block, dt, is_bwd);
+  if (s != LA2_OK) return s;
+  const size_t es = dt == LA2_BF16 ? 2 : 4, lim = 227 * 1024;
+  if (fwd_simt_smem((int)d, (int)dv, block, es, true) > lim) return LA2_ERR_UNSUPPORTED;
+  if (is_bwd && (bwd_dq_simt_smem((int)d, (int)dv, block, es, true) > lim ||
+                 bwd_dkdv_simt_smem((int)d, (int)dv, block, es, true) > lim ||
+                 !bwd_dkdv_simt_fits((int)d, (int)dv, block)))
+    return LA2_ERR_UNSUPPORTED;
+  return LA2_OK;
+}
+
+static la2_status decay_impl(const void* q, const void* k, const void* v, const void* dout, void* o,
+                             void* dq, void* dk, void* dvv, const float* lam, int64_t B, int64_t H,
+                             int64_t N, int64_t d, int64_t dv, int block, la2_dtype dt,
+                             void* workspace, size_t workspace_bytes, la2_stream_t stream,
+                             bool is_bwd) {
+  la2_status s = check_decay_shape(B, H, N, d, dv, block, dt, is_bwd);
+  if (s != LA2_OK) return s;
+  if (B == 0 || H == 0 || N == 0) return LA2_OK;
+  const size_t es = dt == LA2_BF16 ? 2 : 4;
+  const size_t nq = (size_t)B * H * N * d * es, nv = (size_t)B * H * N * dv * es;
+  const void* ins[4] = {q, k, v, is_bwd ? dout : q};
+  const size_t in_sz[4] = {nq, nq, nv, is_bwd ? nv : nq};
+  void* outs[3] = {is_bwd ? dq : o, is_bwd ? dk : nullptr, is_bwd ? dvv : nullptr};
+  const size_t out_sz[3] = {is_bwd ? nq : nv, nq, nv};
+  const int nout = is_bwd ? 3 : 1;
+  for (const void* x : ins)
+    if (!x || !is_aligned(x, 16)) return LA2_ERR_INVALID_ARG;
+  if (!lam || !is_aligned(lam, 4)) return LA2_ERR_INVALID_ARG;
+  const size_t nl = (size_t)H * sizeof(float);
+  for (int i = 0; i < nout; ++i) {
+    if (!outs[i] || !is_aligned(outs[i], 16)) return LA2_ERR_INVALID_ARG;
+    for (int j = 0; j < 4; ++j)
+      if (overlaps(outs[i], out_sz[i], ins[j], in_sz[j])) return LA2_ERR_INVALID_ARG;
+    for (int j = i + 1; j < nout; ++j)
+      if (overlaps(outs[i], out_sz[i], outs[j], out_sz[j])) return LA2_ERR_INVALID_ARG;
+    if (overlaps(outs[i], out_sz[i], lam, nl)) return LA2_ERR_INVALID_ARG;
+  }
+  const int sms = device_sm_count();
+  if (sms <= 0) return LA2_ERR_CUDA;
+  const Plan p = plan_decay(B, H, N, d, dv, block, is_bwd, sms);
+  if (p.ws_bytes > 0) {
+    if (!workspace || workspace_bytes < p.ws_bytes) return LA2_ERR_WORKSPACE;
+    if (!is_aligned(workspace, 256)) return LA2_ERR_INVALID_ARG;
+    for (int i = 0; i < nout; ++i)
+      if (overlaps(workspace, p.ws_bytes, outs[i], out_sz[i])) return LA2_ERR_INVALID_ARG;
+    if (overlaps(workspace, p.ws_bytes, lam, nl)) return LA2_ERR_INVALID_ARG;
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t BH = B * H;
+  const Heads hd{BH, BH, static_cast<int32_t>(H), 1};
+  const int nel = (int)(d * dv);
+  const bool bf = dt == LA2_BF16;
+  float* s_kv = p.need_states ? static_cast<float*>(workspace) : nullptr;
+  float* s_u = p.need_states && is_bwd ? s_kv + (size_t)BH * p.C * nel : nullptr;
+  if (p.need_states) {
+    // K^T V of each chunk decayed to its last row, then their decayed prefix
+    s = bf ? run_chunk_states<__nv_bfloat16>(k, v, s_kv, BH, N, (int)d, (int)dv, p, st, (int)H, 1, 1, lam, 1)
+           : run_chunk_states<float>(k, v, s_kv, BH, N, (int)d, (int)dv, p, st, (int)H, 1, 1, lam, 1);
+    if (s != LA2_OK) return s;
+    s = run_scan(s_kv, BH, nel, p, 3, st, nullptr, 0, (int)d, (int)dv, 0, lam, (int)H);
+    if (s != LA2_OK) return s;
+    if (is_bwd) {  // Q^T dO of each chunk decayed to its first row, then their decayed suffix
+      s = bf ? run_chunk_states<__nv_bfloat16>(q, dout, s_u, BH, N, (int)d, (int)dv, p, st, (int)H, 1, 1, lam, 2)
+             : run_chunk_states<float>(q, dout, s_u, BH, N, (int)d, (int)dv, p, st, (int)H, 1, 1, lam, 2);
+      if (s != LA2_OK) return s;
+      s = run_scan(s_u, BH, nel, p, 4, st, nullptr, 0, (int)d, (int)dv, 0, lam, (int)H);
+      if (s != LA2_OK) return s;
+    }
+  }
+  if (!is_bwd)
+    return bf ? forward_simt<__nv_bfloat16>(q, k, v, o, hd, N, (int)d, (int)dv, 1, block, s_kv, p, st, lam)
+              : forward_simt<float>(q, k, v, o, hd, N, (int)d, (int)dv, 1, block, s_kv, p, st, lam);
+  return bf ? backward_simt<__nv_bfloat16>(q, k, v, dout, dq, dk, dvv, hd, N, (int)d, (int)dv, 1,
+                                           block, s_kv, s_u, p, st, lam)
+            : backward_simt<float>(q, k, v, dout, dq, dk, dvv, hd, N, (int)d, (int)dv, 1, block,
+                                   s_kv, s_u, p, st, lam);
+}
+
 }  // namespace la2
 
 extern "C" {
+
+size_t la2_workspace_size_decay(int64_t B, int64_t H, int64_t N, int64_t d, int64_t dv, int block,
+                                la2_dtype dt, int is_backward) {
+  if (check_decay_shape(B, H, N, d, dv, block, dt, is_backward != 0) != LA2_OK) return (size_t)-1;
+  if (B == 0 || H == 0 || N == 0) return 0;
+  const int sms = device_sm_count();
+  if (sms <= 0) return (size_t)-1;
+  return plan_decay(B, H, N, d, dv, block, is_backward != 0, sms).ws_bytes;
+}
+
+la2_status la2_forward_decay(const void* q, const void* k, const void* v, void* o, const float* lambda,
+                             int64_t B, int64_t H, int64_t N, int64_t d, int64_t dv, int block,
+                             la2_dtype dt, void* workspace, size_t workspace_bytes,
+                             la2_stream_t stream) {
+  return decay_impl(q, k, v, nullptr, o, nullptr, nullptr, nullptr, lambda, B, H, N, d, dv, block, dt,
+                    workspace, workspace_bytes, stream, false);
+}
+
+la2_status la2_backward_decay(const void* q, const void* k, const void* v, const void* dout, void* dq,
+                              void* dk, void* dvv, const float* lambda, int64_t B, int64_t H,
+                              int64_t N, int64_t d, int64_t dv, int block, la2_dtype dt,
+                              void* workspace, size_t workspace_bytes, la2_stream_t stream) {
+  return decay_impl(q, k, v, dout, nullptr, dq, dk, dvv, lambda, B, H, N, d, dv, block, dt, workspace,
+                    workspace_bytes, stream, true);
+}
 
 la2_status la2_backward_gqa(const void* q, const void* k, const void* v, const void* dout, void* dq,
                             void* dk, void* dvv, int64_t B, int64_t H, int64_t Hkv, int64_t N,

@@ -12,6 +12,19 @@
 // states of its sequence (la2_chunk_state + la2_chunk_scan), so chunks of one
 // sequence run in parallel. Everything accumulates in fp32; inputs of type T
 // (float or bf16) are widened on load and outputs rounded to T on store.
+//
+// Decayed form (`lam` non-null, causal, one K/V head per query head): head h
+// has a rate lam[h] in [0, 1] and the state is multiplied by it before each
+// token, KV_t = lam KV_{t-1} + k_t^T v_t, so the mask of the left product is
+// D[t][s] = lam^(t-s) for s <= t. (A reading: the article has no decay; with
+// lam = 1 it is the article's op.) Per block of `rows` rows starting at row i0,
+// with KV the state decayed to row i0 - 1:
+//   O_t  = sum_{j<=t} lam^(t-j) (q_t . k_j) v_j + lam^(t+1) q_t KV
+//   KV  <- lam^rows KV + sum_j lam^(rows-1-j) k_j^T v_j
+// and in the reverse walk of dK/dV, with U the suffix decayed to row i0 + rows:
+//   dK_j += lam^(rows-j) v_j U^T + sum_{t>=j} lam^(t-j) (do_t . v_j) q_t   (dV alike)
+//   U   <- lam^rows U + sum_t lam^t q_t^T do_t
+// Powers come from powf in a table of lam^0 .. lam^Bk per CTA.
 #pragma once
 
 #include <algorithm>
@@ -32,10 +45,14 @@ constexpr int kSimtThreads = 256;
 // ----------------------------------------------------------------------------
 constexpr int kStateRowsPerTile = 32;
 
+// Decayed form: `decay` 1 weights row s of the chunk by lam^(t1-1-s) (the
+// state decayed to the chunk's last row, for the prefix of later chunks), 2 by
+// lam^(s-t0) (decayed to its first row, for the suffix of earlier chunks).
 template <typename T>
 __global__ void __launch_bounds__(kSimtThreads)
 chunk_state_kernel(const T* __restrict__ a, const T* __restrict__ b, float* __restrict__ out,
-                   int64_t N, int da, int db, int64_t L, int64_t C, int H, int G, int group) {
+                   int64_t N, int da, int db, int64_t L, int64_t C, int H, int G, int group,
+                   const float* __restrict__ lam, int decay) {
   extern __shared__ float smem[];
   float* As = smem;                              // [32][da]
   float* Bs = smem + kStateRowsPerTile * da;     // [32][db]
@@ -55,7 +72,12 @@ chunk_state_kernel(const T* __restrict__ a, const T* __restrict__ b, float* __re
     const int rows = (int)imin64(kStateRowsPerTile, t1 - s0);
     for (int i = threadIdx.x; i < kStateRowsPerTile * da; i += blockDim.x) {
       const int r = i / da, col = i % da;
-      As[i] = r < rows ? to_f32(ab[(s0 + r) * da + col]) : 0.f;
+      float w = 1.f;
+      if (decay && r < rows) {
+        const float l = lam[bh % H];
+        w = powf(l, static_cast<float>(decay == 1 ? t1 - 1 - (s0 + r) : (s0 + r) - t0));
+      }
+      As[i] = r < rows ? w * to_f32(ab[(s0 + r) * da + col]) : 0.f;
     }
     for (int i = threadIdx.x; i < kStateRowsPerTile * db; i += blockDim.x) {
       const int r = i / db, col = i % db;
@@ -88,6 +110,10 @@ chunk_state_kernel(const T* __restrict__ a, const T* __restrict__ b, float* __re
 //   mode 0: exclusive prefix  P_c = sum_{c' < c} S_c'   (causal, forward order)
 //   mode 1: exclusive suffix  R_c = sum_{c' > c} S_c'   (causal, reverse order)
 //   mode 2: total into slot 0  T = sum_c S_c             (non-causal)
+//   mode 3: decayed exclusive prefix P_c = f P_{c-1} + S_{c-1}, f = lam^L
+//   mode 4: decayed exclusive suffix R_c = S_{c+1} + f R_{c+1}
+// (modes 3, 4: chunk states decayed to their last / first row, lam[seq % H];
+// every chunk but the last has L rows, and the last one's length never enters)
 // `ext` (optional) adds a base to every prefix / suffix: the sum of n_ext
 // states [n_ext][nseq][d][dv] (row-major fp32) of the parts of the sequence
 // before (mode 0) or after (mode 1) this one. `f4_layout` says the chunk
@@ -101,12 +127,24 @@ __device__ __forceinline__ int64_t state_row_major_index(int e, int d, int dv, i
 
 __global__ void __launch_bounds__(kSimtThreads)
 chunk_scan_kernel(float* __restrict__ s, int64_t C, int nel, int mode, const float* __restrict__ ext,
-                  int64_t n_ext, int64_t nseq, int d, int dv, int f4_layout) {
+                  int64_t n_ext, int64_t nseq, int d, int dv, int f4_layout,
+                  const float* __restrict__ lam, int H, int64_t L) {
   pdl_launch_dependents();
   pdl_wait();
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
   if (e >= nel) return;
   float* p = s + (int64_t)blockIdx.y * C * nel + e;
+  if (mode == 3 || mode == 4) {
+    const float f = powf(lam[blockIdx.y % H], static_cast<float>(L));
+    float run = 0.f;
+    for (int64_t i = 0; i < C; ++i) {
+      const int64_t c = mode == 3 ? i : C - 1 - i;
+      const float x = p[c * nel];
+      p[c * nel] = run;
+      run = fmaf(f, run, x);
+    }
+    return;
+  }
   constexpr int U = 8;  // independent loads in flight per thread
   float run = 0.f;
   if (ext) {
@@ -167,13 +205,15 @@ template <typename T>
 __global__ void __launch_bounds__(kSimtThreads)
 fwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                 T* __restrict__ o, const float* __restrict__ states, int64_t N, int d, int dv,
-                int Bk, int64_t L, int64_t C, int causal, int H, int G) {
+                int Bk, int64_t L, int64_t C, int causal, int H, int G, const float* __restrict__ lam) {
   extern __shared__ float smem[];
   float* KV = smem;
   T* Qs = reinterpret_cast<T*>(KV + d * dv);
   T* Ks = Qs + Bk * d;
   T* Vs = Ks + Bk * d;
   T* S = Vs + Bk * dv;  // masked (Q K^T) block, rounded to T
+  float* pw = reinterpret_cast<float*>(S + Bk * Bk);  // decayed form: lam^0 .. lam^Bk
+  const bool dec = lam != nullptr;
   const int64_t unit = blockIdx.x;
   const int64_t bh = unit / C, c = unit % C;
   const int64_t bkv = kv_seq(bh, H, G);  // K/V sequence (and its states)
@@ -187,6 +227,8 @@ fwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
   if (!causal) init = states + bkv * C * nel;           // total in slot 0
   else if (states) init = states + (bkv * C + c) * nel;  // exclusive prefix
   load_state(KV, init, (int)nel);
+  if (dec)
+    for (int i = threadIdx.x; i <= Bk; i += blockDim.x) pw[i] = powf(lam[bh % H], static_cast<float>(i));
 
   for (int64_t i0 = t0; i0 < t1; i0 += Bk) {
     const int rows = (int)imin64(Bk, t1 - i0);
@@ -202,7 +244,8 @@ fwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
         float s = 0.f;
         if (j <= t)
           for (int cc = 0; cc < d; ++cc) s = fmaf(to_f32(Qs[t * d + cc]), to_f32(Ks[j * d + cc]), s);
-        S[i] = from_f32<T>(s);  // M_B: lower-triangular ones, diagonal kept
+        if (dec && j <= t) s *= pw[t - j];
+        S[i] = from_f32<T>(s);  // M_B: lower-triangular ones, diagonal kept (D_B when decayed)
       }
       __syncthreads();
     }
@@ -211,15 +254,25 @@ fwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
       float acc = 0.f;
       if (causal)
         for (int j = 0; j <= t; ++j) acc = fmaf(to_f32(S[t * Bk + j]), to_f32(Vs[j * dv + e]), acc);
-      for (int cc = 0; cc < d; ++cc) acc = fmaf(to_f32(Qs[t * d + cc]), KV[cc * dv + e], acc);
+      if (dec) {
+        float x = 0.f;
+        for (int cc = 0; cc < d; ++cc) x = fmaf(to_f32(Qs[t * d + cc]), KV[cc * dv + e], x);
+        acc = fmaf(pw[t + 1], x, acc);
+      } else {
+        for (int cc = 0; cc < d; ++cc) acc = fmaf(to_f32(Qs[t * d + cc]), KV[cc * dv + e], acc);
+      }
       ob[(i0 + t) * dv + e] = from_f32<T>(acc);
     }
     __syncthreads();
     if (causal) {
       for (int i = threadIdx.x; i < d * dv; i += blockDim.x) {
         const int cc = i / dv, e = i % dv;
-        float acc = KV[i];
-        for (int t = 0; t < rows; ++t) acc = fmaf(to_f32(Ks[t * d + cc]), to_f32(Vs[t * dv + e]), acc);
+        float acc = dec ? pw[rows] * KV[i] : KV[i];
+        if (dec)
+          for (int t = 0; t < rows; ++t)
+            acc = fmaf(pw[rows - 1 - t] * to_f32(Ks[t * d + cc]), to_f32(Vs[t * dv + e]), acc);
+        else
+          for (int t = 0; t < rows; ++t) acc = fmaf(to_f32(Ks[t * d + cc]), to_f32(Vs[t * dv + e]), acc);
         KV[i] = acc;
       }
       __syncthreads();
@@ -237,13 +290,16 @@ template <typename T>
 __global__ void __launch_bounds__(kSimtThreads)
 bwd_dq_simt_kernel(const T* __restrict__ k, const T* __restrict__ v, const T* __restrict__ dout,
                    T* __restrict__ dq, const float* __restrict__ states, int64_t N, int d, int dv,
-                   int Bk, int64_t L, int64_t C, int causal, int H, int G) {
+                   int Bk, int64_t L, int64_t C, int causal, int H, int G,
+                   const float* __restrict__ lam) {
   extern __shared__ float smem[];
   float* KV = smem;
   T* dOs = reinterpret_cast<T*>(KV + d * dv);
   T* Vs = dOs + Bk * dv;
   T* Ks = Vs + Bk * dv;
   T* A = Ks + Bk * d;  // masked (dO V^T) block, rounded to T
+  float* pw = reinterpret_cast<float*>(A + Bk * Bk);  // decayed form: lam^0 .. lam^Bk
+  const bool dec = lam != nullptr;
   const int64_t unit = blockIdx.x;
   const int64_t bh = unit / C, c = unit % C;
   const int64_t bkv = kv_seq(bh, H, G);
@@ -257,6 +313,8 @@ bwd_dq_simt_kernel(const T* __restrict__ k, const T* __restrict__ v, const T* __
   if (!causal) init = states + bkv * C * nel;
   else if (states) init = states + (bkv * C + c) * nel;
   load_state(KV, init, (int)nel);
+  if (dec)
+    for (int i = threadIdx.x; i <= Bk; i += blockDim.x) pw[i] = powf(lam[bh % H], static_cast<float>(i));
 
   for (int64_t i0 = t0; i0 < t1; i0 += Bk) {
     const int rows = (int)imin64(Bk, t1 - i0);
@@ -272,6 +330,7 @@ bwd_dq_simt_kernel(const T* __restrict__ k, const T* __restrict__ v, const T* __
         float s = 0.f;
         if (j <= t)
           for (int e = 0; e < dv; ++e) s = fmaf(to_f32(dOs[t * dv + e]), to_f32(Vs[j * dv + e]), s);
+        if (dec && j <= t) s *= pw[t - j];
         A[i] = from_f32<T>(s);
       }
       __syncthreads();
@@ -281,15 +340,25 @@ bwd_dq_simt_kernel(const T* __restrict__ k, const T* __restrict__ v, const T* __
       float acc = 0.f;
       if (causal)
         for (int j = 0; j <= t; ++j) acc = fmaf(to_f32(A[t * Bk + j]), to_f32(Ks[j * d + cc]), acc);
-      for (int e = 0; e < dv; ++e) acc = fmaf(to_f32(dOs[t * dv + e]), KV[cc * dv + e], acc);
+      if (dec) {
+        float x = 0.f;
+        for (int e = 0; e < dv; ++e) x = fmaf(to_f32(dOs[t * dv + e]), KV[cc * dv + e], x);
+        acc = fmaf(pw[t + 1], x, acc);
+      } else {
+        for (int e = 0; e < dv; ++e) acc = fmaf(to_f32(dOs[t * dv + e]), KV[cc * dv + e], acc);
+      }
       dqb[(i0 + t) * d + cc] = from_f32<T>(acc);
     }
     __syncthreads();
     if (causal) {
       for (int i = threadIdx.x; i < d * dv; i += blockDim.x) {
         const int cc = i / dv, e = i % dv;
-        float acc = KV[i];
-        for (int t = 0; t < rows; ++t) acc = fmaf(to_f32(Ks[t * d + cc]), to_f32(Vs[t * dv + e]), acc);
+        float acc = dec ? pw[rows] * KV[i] : KV[i];
+        if (dec)
+          for (int t = 0; t < rows; ++t)
+            acc = fmaf(pw[rows - 1 - t] * to_f32(Ks[t * d + cc]), to_f32(Vs[t * dv + e]), acc);
+        else
+          for (int t = 0; t < rows; ++t) acc = fmaf(to_f32(Ks[t * d + cc]), to_f32(Vs[t * dv + e]), acc);
         KV[i] = acc;
       }
       __syncthreads();
@@ -330,7 +399,7 @@ __global__ void __launch_bounds__(kSimtThreads)
 bwd_dkdv_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                      const T* __restrict__ dout, T* __restrict__ dk, T* __restrict__ dvv,
                      const float* __restrict__ states, int64_t N, int d, int dv, int Bk,
-                     int64_t L, int64_t C, int causal, int H, int G) {
+                     int64_t L, int64_t C, int causal, int H, int G, const float* __restrict__ lam) {
   extern __shared__ float smem[];
   float* U = smem;
   T* Qs = reinterpret_cast<T*>(U + d * dv);
@@ -339,6 +408,8 @@ bwd_dkdv_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* 
   T* dOs = Vs + Bk * dv;
   T* A = dOs + Bk * dv;  // masked (dO V^T) block, rounded to T
   T* P = A + Bk * Bk;    // masked (Q K^T) block, rounded to T
+  float* pw = reinterpret_cast<float*>(P + Bk * Bk);  // decayed form (one head a sequence): lam^0..lam^Bk
+  const bool dec = lam != nullptr;
   const int64_t unit = blockIdx.x;
   const int64_t bh = unit / C, c = unit % C;  // the K/V sequence
   const int64_t t0 = c * L, t1 = imin64(N, t0 + L);
@@ -353,6 +424,8 @@ bwd_dkdv_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* 
   if (!causal) init = states + bh * C * nel;
   else if (states) init = states + (bh * C + c) * nel;  // exclusive suffix
   load_state(U, init, (int)nel);
+  if (dec)
+    for (int i = threadIdx.x; i <= Bk; i += blockDim.x) pw[i] = powf(lam[bh % H], static_cast<float>(i));
   // strips: dK strip s = (row s / sk, columns 32 * (s % sk)), likewise dV
   const int sk = (d + kStrip - 1) / kStrip, sv = (dv + kStrip - 1) / kStrip;
 
@@ -379,6 +452,9 @@ bwd_dkdv_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* 
           for (int cc = 0; cc < kStrip; ++cc)
             if (c0 + cc < d) ak[r][cc] = fmaf(x, U[(c0 + cc) * dv + e], ak[r][cc]);
         }
+        if (dec)
+#pragma unroll
+          for (int cc = 0; cc < kStrip; ++cc) ak[r][cc] *= pw[rows - j];
       }
     }
 #pragma unroll
@@ -394,6 +470,9 @@ bwd_dkdv_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* 
           for (int e = 0; e < kStrip; ++e)
             if (e0 + e < dv) av[r][e] = fmaf(x, U[cc * dv + e0 + e], av[r][e]);
         }
+        if (dec)
+#pragma unroll
+          for (int e = 0; e < kStrip; ++e) av[r][e] *= pw[rows - j];
       }
     }
     for (int g = 0; causal && g < heads; ++g) {
@@ -408,6 +487,10 @@ bwd_dkdv_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* 
         if (j <= t) {
           for (int e = 0; e < dv; ++e) a = fmaf(to_f32(dOs[t * dv + e]), to_f32(Vs[j * dv + e]), a);
           for (int cc = 0; cc < d; ++cc) p = fmaf(to_f32(Qs[t * d + cc]), to_f32(Ks[j * d + cc]), p);
+        }
+        if (dec && j <= t) {
+          a *= pw[t - j];
+          p *= pw[t - j];
         }
         A[i] = from_f32<T>(a);
         P[i] = from_f32<T>(p);
@@ -428,8 +511,12 @@ bwd_dkdv_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* 
       }
       for (int i = threadIdx.x; i < d * dv; i += blockDim.x) {
         const int cc = i / dv, e = i % dv;
-        float acc = U[i];
-        for (int t = 0; t < rows; ++t) acc = fmaf(to_f32(Qs[t * d + cc]), to_f32(dOs[t * dv + e]), acc);
+        float acc = dec ? pw[rows] * U[i] : U[i];
+        if (dec)
+          for (int t = 0; t < rows; ++t)
+            acc = fmaf(pw[t] * to_f32(Qs[t * d + cc]), to_f32(dOs[t * dv + e]), acc);
+        else
+          for (int t = 0; t < rows; ++t) acc = fmaf(to_f32(Qs[t * d + cc]), to_f32(dOs[t * dv + e]), acc);
         U[i] = acc;
       }
     }
@@ -462,14 +549,18 @@ inline bool bwd_dkdv_simt_fits(int d, int dv, int Bk) {
   return strips <= kStripsPerThread * kSimtThreads;
 }
 
-inline size_t fwd_simt_smem(int d, int dv, int Bk, size_t es) {
-  return sizeof(float) * (size_t)d * dv + es * ((size_t)Bk * (2 * d + dv) + (size_t)Bk * Bk);
+// (`decay`: plus the table lam^0 .. lam^Bk)
+inline size_t fwd_simt_smem(int d, int dv, int Bk, size_t es, bool decay = false) {
+  return sizeof(float) * (size_t)d * dv + es * ((size_t)Bk * (2 * d + dv) + (size_t)Bk * Bk) +
+         (decay ? sizeof(float) * (Bk + 1) : 0);
 }
-inline size_t bwd_dq_simt_smem(int d, int dv, int Bk, size_t es) {
-  return sizeof(float) * (size_t)d * dv + es * ((size_t)Bk * (2 * dv + d) + (size_t)Bk * Bk);
+inline size_t bwd_dq_simt_smem(int d, int dv, int Bk, size_t es, bool decay = false) {
+  return sizeof(float) * (size_t)d * dv + es * ((size_t)Bk * (2 * dv + d) + (size_t)Bk * Bk) +
+         (decay ? sizeof(float) * (Bk + 1) : 0);
 }
-inline size_t bwd_dkdv_simt_smem(int d, int dv, int Bk, size_t es) {
-  return sizeof(float) * (size_t)d * dv + es * ((size_t)Bk * (2 * d + 2 * dv) + 2 * (size_t)Bk * Bk);
+inline size_t bwd_dkdv_simt_smem(int d, int dv, int Bk, size_t es, bool decay = false) {
+  return sizeof(float) * (size_t)d * dv + es * ((size_t)Bk * (2 * d + 2 * dv) + 2 * (size_t)Bk * Bk) +
+         (decay ? sizeof(float) * (Bk + 1) : 0);
 }
 inline size_t chunk_state_smem(int da, int db) {
   return sizeof(float) * (size_t)kStateRowsPerTile * (da + db);

@@ -53,6 +53,11 @@ _SIGS = {
                               _int, _vp, _sz, _vp]),
     "la2_backward_sp": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _i64, _i64, _i64,
                                _i64, _i64, _i64, _int, _int, _vp, _sz, _vp]),
+    "la2_workspace_size_decay": (_sz, [_i64, _i64, _i64, _i64, _i64, _int, _int, _int]),
+    "la2_forward_decay": (_int, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _int, _int,
+                                 _vp, _sz, _vp]),
+    "la2_backward_decay": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64,
+                                  _i64, _int, _int, _vp, _sz, _vp]),
     "la2_check": (_int, [_vp]),
     "la2_status_string": (ctypes.c_char_p, [_int]),
     "la2_set_chunk_len": (_int, [_i64]),
@@ -89,6 +94,9 @@ la2_backward_gqa = _lib.la2_backward_gqa
 la2_workspace_size_sp = _lib.la2_workspace_size_sp
 la2_forward_sp = _lib.la2_forward_sp
 la2_backward_sp = _lib.la2_backward_sp
+la2_workspace_size_decay = _lib.la2_workspace_size_decay
+la2_forward_decay = _lib.la2_forward_decay
+la2_backward_decay = _lib.la2_backward_decay
 la2_set_chunk_len = _lib.la2_set_chunk_len
 la2_plan_ranges = _lib.la2_plan_ranges
 la2_set_spin_limit = _lib.la2_set_spin_limit
@@ -284,6 +292,82 @@ def backward(q, k, v, do, causal: bool = True, block: int = 64, outs=None, works
     _raise(la2_backward_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dvv), B,
                             H, Hkv, N, d, dv, int(causal), block, dt, _ptr(ws),
                             ws.numel() if ws is not None else 0, _stream_handle(stream)))
+    return dq, dk, dvv
+
+
+def workspace_bytes_decay(B, H, N, d, dv, block, dtype_code, is_backward) -> int:
+    n = la2_workspace_size_decay(B, H, N, d, dv, block, dtype_code, int(is_backward))
+    if n == ctypes.c_size_t(-1).value:
+        raise La2Error(LA2_ERR_INVALID_ARG)
+    return int(n)
+
+
+def _decay_rates(lam, q, stream):
+    """Per-head rates as a float32 CUDA tensor of H values on q's device (a
+    copy, when one is needed, is made on the stream the kernels run on)."""
+    import torch
+
+    lam = torch.as_tensor(lam, dtype=torch.float32).reshape(-1)
+    if lam.numel() != q.shape[1]:
+        raise La2Error(LA2_ERR_INVALID_ARG)
+    if stream is None:
+        return lam.to(q.device).contiguous()
+    with torch.cuda.stream(stream):
+        return lam.to(q.device).contiguous()
+
+
+def forward_decay(q, k, v, lam, block: int = 64, out=None, workspace=None, stream=None):
+    """Decayed causal form: o_t = sum_{s<=t} lam_h^(t-s) (q_t . k_s) v_s for
+    [B,H,N,d] CUDA tensors and H per-head rates ``lam``; returns O."""
+    import torch
+
+    _check_inputs(q, k, v)
+    if q.dim() != 4:
+        raise La2Error(LA2_ERR_INVALID_ARG)
+    B, H, N, d = q.shape
+    dv = v.shape[-1]
+    dt = _dtype_code(q)
+    _check_like(q, q.shape, q.dtype, k)
+    _check_like(q, (B, H, N, dv), q.dtype, v)
+    rates = _decay_rates(lam, q, stream)
+    if out is None:
+        out = torch.empty((B, H, N, dv), dtype=q.dtype, device=q.device)
+    _check_inputs(out)
+    _check_like(q, (B, H, N, dv), q.dtype, out)
+    need = workspace_bytes_decay(B, H, N, d, dv, block, dt, False)
+    ws = workspace if workspace is not None else _workspace(need, q.device, stream)
+    _check_workspace(ws, need, q.device)
+    _raise(la2_forward_decay(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(rates), B, H, N, d, dv,
+                             block, dt, _ptr(ws), ws.numel() if ws is not None else 0,
+                             _stream_handle(stream)))
+    return out
+
+
+def backward_decay(q, k, v, do, lam, block: int = 64, outs=None, workspace=None, stream=None):
+    """Gradients (dQ, dK, dV) of <dO, O> for the decayed causal form."""
+    import torch
+
+    _check_inputs(q, k, v, do)
+    if q.dim() != 4:
+        raise La2Error(LA2_ERR_INVALID_ARG)
+    B, H, N, d = q.shape
+    dv = v.shape[-1]
+    dt = _dtype_code(q)
+    _check_like(q, q.shape, q.dtype, k)
+    _check_like(q, (B, H, N, dv), q.dtype, v, do)
+    rates = _decay_rates(lam, q, stream)
+    if outs is None:
+        outs = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
+    dq, dk, dvv = outs
+    _check_inputs(dq, dk, dvv)
+    _check_like(q, q.shape, q.dtype, dq, dk)
+    _check_like(q, (B, H, N, dv), q.dtype, dvv)
+    need = workspace_bytes_decay(B, H, N, d, dv, block, dt, True)
+    ws = workspace if workspace is not None else _workspace(need, q.device, stream)
+    _check_workspace(ws, need, q.device)
+    _raise(la2_backward_decay(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dvv),
+                              _ptr(rates), B, H, N, d, dv, block, dt, _ptr(ws),
+                              ws.numel() if ws is not None else 0, _stream_handle(stream)))
     return dq, dk, dvv
 
 

@@ -223,3 +223,41 @@ def test_binding_checks_grouped_shapes():
     for kv in (torch.zeros(1, 3, 16, 64), torch.zeros(1, 0, 16, 64)):
         with pytest.raises(la2.La2Error):
             la2._kv_heads(q, kv, kv)
+
+
+def _fwd_decay(**kw):
+    args = dict(q=NULL, k=NULL, v=NULL, o=NULL, lam=NULL, B=1, H=1, N=16, d=64, dv=64, block=64,
+                dt=la2.LA2_F32, ws=NULL, wsb=0, stream=NULL)
+    args.update(kw)
+    return la2.la2_forward_decay(args["q"], args["k"], args["v"], args["o"], args["lam"], args["B"],
+                                 args["H"], args["N"], args["d"], args["dv"], args["block"],
+                                 args["dt"], args["ws"], args["wsb"], args["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(B=-1), la2.LA2_ERR_INVALID_ARG),
+    (dict(d=0), la2.LA2_ERR_INVALID_ARG),
+    (dict(dt=7), la2.LA2_ERR_INVALID_ARG),
+    (dict(d=200), la2.LA2_ERR_UNSUPPORTED),
+    (dict(block=48), la2.LA2_ERR_UNSUPPORTED),
+    (dict(B=0), la2.LA2_OK),
+    # valid shape, missing tensors or rates
+    (dict(), la2.LA2_ERR_INVALID_ARG),
+    (dict(q=4096, k=8192, v=12288, o=16384), la2.LA2_ERR_INVALID_ARG),  # no rates
+    (dict(q=4096, k=8192, v=12288, o=16384, lam=16386), la2.LA2_ERR_INVALID_ARG),  # misaligned rates
+    (dict(q=4096, k=8192, v=12288, o=16384, lam=16384), la2.LA2_ERR_INVALID_ARG),  # rates inside o
+])
+def test_forward_decay_rejects_bad_arguments(kw, code):
+    assert _fwd_decay(**kw) == code
+
+
+def test_backward_decay_limits():
+    """The decayed form runs on CUDA cores: bf16 d = dv = 128 fits the forward at
+    block 128 but not the backward's dK/dV tiles (documented in la2.h)."""
+    bf = la2.LA2_BF16
+    assert la2.la2_backward_decay(NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, 1, 1, 16, 128, 128,
+                                  128, bf, NULL, 0, NULL) == la2.LA2_ERR_UNSUPPORTED
+    assert la2.la2_workspace_size_decay(1, 1, 16, 128, 128, 128, bf, 1) == ctypes.c_size_t(-1).value
+    assert la2.la2_backward_decay(NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, 0, 1, 16, 128, 128,
+                                  64, bf, NULL, 0, NULL) == la2.LA2_OK
+    assert "la2_forward_decay" in la2.EXPORTED and "la2_backward_decay" in la2.EXPORTED
