@@ -173,6 +173,8 @@ def workload_from_args(args):
 
     if args.workload in I.WORKLOADS:
         w = I.WORKLOADS[args.workload]
+    elif args.workload in I.EXTRA_WORKLOADS:
+        w = I.EXTRA_WORKLOADS[args.workload]
     elif args.workload.startswith("bf16_sweep_n"):
         n, b = args.workload[len("bf16_sweep_n"):].split("_b")
         w = I.sweep_workload(int(n), int(b))
@@ -203,11 +205,14 @@ def flops_per_token(w, causal=True):
 
 def bytes_per_token(w):
     """HBM bytes per token·head each step must move at least: the forward reads
-    Q, K, V and writes O; the backward reads Q, K, V, dO and writes dQ, dK, dV."""
+    Q, K, V and writes O; the backward reads Q, K, V, dO and writes dQ, dK, dV.
+    With grouped K/V heads (G query heads a K/V head) the K/V side counts once
+    per K/V head: 1/G per query token·head."""
     es = 2 if w.dtype == "bf16" else 4
-    b = (2 * w.d + 2 * w.dv) * es
+    g = w.H // w.extra.get("Hkv", w.H)
+    b = (w.d + w.dv) * es + (w.d + w.dv) * es / g
     if w.backward:
-        b += (4 * w.d + 3 * w.dv) * es
+        b += (w.d + w.dv + w.d) * es + 2 * (w.d + w.dv) * es / g
     return b
 
 
@@ -337,9 +342,14 @@ def run_reference(args):
 
 def config_of(w, causal=True):
     kind = "causal" if causal else "non-causal"
-    return {"workload": f"{w.name}: {kind} forward B={w.B} H={w.H} N={w.N} d={w.d} dv={w.dv} "
-                        f"block={w.block} {w.dtype}", "B": w.B, "H": w.H, "N": w.N, "d": w.d,
-            "dv": w.dv, "block": w.block, "causal": causal}
+    if "decay" in w.extra:
+        kind = f"decayed causal (lambda={w.extra['decay']} every head, CUDA cores)"
+    heads = f"H={w.H} Hkv={w.extra['Hkv']}" if "Hkv" in w.extra else f"H={w.H}"
+    c = {"workload": f"{w.name}: {kind} forward B={w.B} {heads} "
+                     f"N={w.N} d={w.d} dv={w.dv} block={w.block} {w.dtype}", "B": w.B, "H": w.H,
+         "N": w.N, "d": w.d, "dv": w.dv, "block": w.block, "causal": causal}
+    c.update(w.extra)
+    return c
 
 
 # ------------------------------------------------------------------- GPU
@@ -374,6 +384,7 @@ def run_gpu(args):
         others = [I.WORKLOADS["bf16_b4h16_n2k"]]
         others += [I.sweep_workload(N, b) for N in I.SWEEP_N for b in I.SWEEP_BLOCKS]
         others += [I.WORKLOADS["bf16_long_512k"], I.WORKLOADS["bf16_fwdbwd_b2h32_n8k"]]
+        others += list(I.EXTRA_WORKLOADS.values())
         for sw in others:
             if sw.name == w.name:
                 continue
@@ -425,6 +436,9 @@ def bench_workload(args, w, dev, la2, world, rank, local, hbm, peak_kind, main, 
 
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
+    Hkv = w.extra.get("Hkv", w.H)
+    decay = w.extra.get("decay")
+    rates = torch.full((w.H,), float(decay), dtype=torch.float32, device=dev) if decay is not None else None
     set_bytes = w.tokens * bytes_per_token(w)
     nsets = max(1, math.ceil(3 * L2_BYTES / set_bytes)) if set_bytes < 3 * L2_BYTES else 1
     nsets = min(nsets, 8)
@@ -437,28 +451,48 @@ def bench_workload(args, w, dev, la2, world, rank, local, hbm, peak_kind, main, 
         if s > 0:  # distinct buffers, same values
             pass
         o = torch.empty((w.B, w.H, w.N, w.dv), dtype=w.torch_dtype, device=dev)
+        if Hkv < w.H:  # grouped K/V heads: the first Hkv heads of the draw
+            k, v = k[:, :Hkv].contiguous(), v[:, :Hkv].contiguous()
         sets.append((q, k, v, o))
     dt = la2.LA2_BF16 if w.dtype == "bf16" else la2.LA2_F32
-    ws_bytes = la2.workspace_bytes(w.B, w.H, w.N, w.d, w.dv, causal, w.block, dt, False)
+
+    def ws_size(bwd):
+        if decay is not None:
+            return la2.workspace_bytes_decay(w.B, w.H, w.N, w.d, w.dv, w.block, dt, bwd)
+        return la2.workspace_bytes_gqa(w.B, w.H, Hkv, w.N, w.d, w.dv, causal, w.block, dt, bwd)
+
+    ws_bytes = ws_size(False)
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
     st = la2._stream_handle(stream)
 
     if w.backward:  # one step = forward + backward of the same batch
         dO = I.make_inputs(w, with_grad_out=True)["do"].to(dev)
-        grads = tuple(torch.empty_like(sets[0][0]) for _ in range(3))
-        wsb_bytes = la2.workspace_bytes(w.B, w.H, w.N, w.d, w.dv, True, w.block, dt, True)
+        grads = (torch.empty_like(sets[0][0]), torch.empty_like(sets[0][1]), torch.empty_like(sets[0][2]))
+        wsb_bytes = ws_size(True)
         wsb = torch.empty(max(wsb_bytes, 1), dtype=torch.uint8, device=dev)
 
     def step(i):
         q, k, v, o = sets[i % nsets]
-        rc = la2.la2_forward(la2._ptr(q), la2._ptr(k), la2._ptr(v), la2._ptr(o), w.B, w.H, w.N, w.d,
-                             w.dv, int(causal), w.block, dt, la2._ptr(ws), ws_bytes, st)
+        if decay is not None:
+            rc = la2.la2_forward_decay(la2._ptr(q), la2._ptr(k), la2._ptr(v), la2._ptr(o),
+                                       la2._ptr(rates), w.B, w.H, w.N, w.d, w.dv, w.block, dt,
+                                       la2._ptr(ws), ws_bytes, st)
+        else:
+            rc = la2.la2_forward_gqa(la2._ptr(q), la2._ptr(k), la2._ptr(v), la2._ptr(o), w.B, w.H,
+                                     Hkv, w.N, w.d, w.dv, int(causal), w.block, dt, la2._ptr(ws),
+                                     ws_bytes, st)
         if rc != 0:
             raise la2.La2Error(rc)
         if w.backward:
-            rc = la2.la2_backward(la2._ptr(q), la2._ptr(k), la2._ptr(v), la2._ptr(dO),
-                                  la2._ptr(grads[0]), la2._ptr(grads[1]), la2._ptr(grads[2]), w.B,
-                                  w.H, w.N, w.d, w.dv, 1, w.block, dt, la2._ptr(wsb), wsb_bytes, st)
+            g = (la2._ptr(grads[0]), la2._ptr(grads[1]), la2._ptr(grads[2]))
+            if decay is not None:
+                rc = la2.la2_backward_decay(la2._ptr(q), la2._ptr(k), la2._ptr(v), la2._ptr(dO), *g,
+                                            la2._ptr(rates), w.B, w.H, w.N, w.d, w.dv, w.block, dt,
+                                            la2._ptr(wsb), wsb_bytes, st)
+            else:
+                rc = la2.la2_backward_gqa(la2._ptr(q), la2._ptr(k), la2._ptr(v), la2._ptr(dO), *g,
+                                          w.B, w.H, Hkv, w.N, w.d, w.dv, 1, w.block, dt,
+                                          la2._ptr(wsb), wsb_bytes, st)
             if rc != 0:
                 raise la2.La2Error(rc)
 
@@ -562,9 +596,10 @@ def bench_workload(args, w, dev, la2, world, rank, local, hbm, peak_kind, main, 
     if w.backward:
         line["metric"] = FWDBWD_METRIC
         line["config"]["workload"] += " (+ backward)"
-    if main and not args.no_e2e and not w.backward:
+    # (the e2e leg and the CPU oracle time the plain op: not for the follow-on workloads)
+    if main and not args.no_e2e and not w.backward and not w.extra:
         line["e2e"] = e2e_measure(args, w, dev, la2, world, base, ws, ws_bytes, dt, causal)
-    if main and rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if main and rank == 0 and world == 1 and not args.no_cpu_baseline and not w.extra:
         line["cpu_baseline"] = cpu_oracle_rate(w, budget_s=10.0, causal=causal)
     return line
 

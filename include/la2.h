@@ -183,9 +183,11 @@ LA2_API la2_status la2_backward_sp(const void *q, const void *k, const void *v, 
  * device memory, 4-byte aligned, read only (powers are taken with powf; rates
  * outside [0, 1] are not rejected and follow the same formula). One K/V head per
  * query head; q, k, v, o, dout, dq, dk, dvv as for la2_forward / la2_backward
- * (causal only). Runs on CUDA cores for every shape and dtype la2_forward takes,
- * with the shared-memory limits of that path: bf16 d = dv = 128 at block 128
- * fits the forward but not the backward (LA2_ERR_UNSUPPORTED). Workspace:
+ * (causal only). The forward runs on tensor cores at bf16 d = dv = 128 (the
+ * chunk kernels with decayed chunk states), on CUDA cores for every other shape
+ * and dtype la2_forward takes; the backward runs on CUDA cores, with the
+ * shared-memory limits of that path: bf16 d = dv = 128 at block 128 does not fit
+ * the backward (LA2_ERR_UNSUPPORTED). Workspace:
  * la2_workspace_size_decay. Other conventions and errors as for la2_forward /
  * la2_backward; `lambda` must not overlap the outputs.
  */

@@ -1007,9 +1007,12 @@ static la2_status backward_impl(const void* q, const void* k, const void* v, con
 
 // ------------------------------------------------------------------ decayed form
 
-// CUDA-core plan of the decayed form: chunks of L rows (about two units per
-// SM, at least four blocks a chunk), chunk states decayed to a chunk edge and
-// their decayed scan when a sequence has more than one chunk.
+// Plan of the decayed form: chunks of L rows, chunk states decayed to a chunk
+// edge and their decayed scan when a sequence has more than one chunk. The
+// chunk count is chosen by waves of SMs (one CTA per (b, h, chunk)): the
+// fewest waves times (chunk blocks + a fixed cost of 3 blocks), chunks of at
+// least four blocks (B4 H16 N2K: 2 chunks, 128 CTAs in one wave, where 5 ran
+// three waves).
 static Plan plan_decay(int64_t B, int64_t H, int64_t N, int64_t d, int64_t dv, int block,
                        bool is_bwd, int sms) {
   Plan p;
@@ -1018,8 +1021,17 @@ static Plan plan_decay(int64_t B, int64_t H, int64_t N, int64_t d, int64_t dv, i
   if (g_chunk_len > 0) {
     L = ((g_chunk_len + block - 1) / block) * block;
   } else {
-    int64_t C = std::max<int64_t>(1, (2 * (int64_t)std::max(sms, 1) + BH - 1) / std::max<int64_t>(BH, 1));
-    C = std::min<int64_t>(C, std::max<int64_t>(1, T / 4));
+    const int64_t G = std::max(sms, 1), cmax = std::max<int64_t>(1, T / 4);
+    int64_t C = 1;
+    double best = 0.0;
+    for (int64_t c = 1; c <= cmax; ++c) {
+      const double cost = static_cast<double>((BH * c + G - 1) / G) *
+                          (static_cast<double>((T + c - 1) / c) + 3.0);
+      if (c == 1 || cost < best) {
+        best = cost;
+        C = c;
+      }
+    }
     L = ((T + C - 1) / C) * block;
   }
   p.L = std::max<int64_t>(L, block);
@@ -1027,6 +1039,51 @@ static Plan plan_decay(int64_t B, int64_t H, int64_t N, int64_t d, int64_t dv, i
   p.need_states = p.C > 1;
   p.ws_bytes = p.need_states ? (size_t)BH * p.C * d * dv * sizeof(float) * (is_bwd ? 2 : 1) : 0;
   return p;
+}
+
+template <int BK>
+static la2_status decay_forward_tc(const void* q, const void* k, const void* v, void* o,
+                                  const float* lam, int64_t BH, int64_t H, int64_t N,
+                                  float* states, const Plan& p, cudaStream_t st) {
+  constexpr int D = 128, DV = 128;
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap_3d(&tq, q, BH, N, D, BK) || !make_tmap_3d(&tk, k, BH, N, D, BK) ||
+      !make_tmap_3d(&tv, v, BH, N, DV, BK))
+    return LA2_ERR_CUDA;
+  sm100::Params prm{};
+  prm.N = N;
+  prm.L = p.L;
+  prm.C = p.C;
+  prm.units_per_seq = p.C;
+  prm.spin_limit = spin_limit();
+  prm.H = static_cast<int32_t>(H);
+  prm.G = 1;
+  prm.state_group = 1;
+  prm.lam = lam;
+  la2_status s = LA2_OK;
+  if (p.need_states) {
+    sm100::Params ps = prm;
+    ps.out_states = states;
+    {
+      LaunchTimer t(K_STATE_TC, st);
+      s = launch_fwd_sm100<BK, D, DV, sm100::MODE_STATE, false, true>(tk, tk, tv, tk, ps, BH * p.C, st);
+    }
+    if (s != LA2_OK) return s;
+    // A few chunks a sequence: each chunk adds up the earlier chunks' states
+    // itself (decay-weighted, no scan launch); many: their decayed prefix first.
+    if (p.C > kSumInKernel) {
+      s = run_scan(states, BH, D * DV, p, 3, st, nullptr, 0, D, DV, 0, lam, static_cast<int>(H));
+      if (s != LA2_OK) return s;
+    } else {
+      prm.decay_sum = 1;
+    }
+  }
+  prm.o = static_cast<__nv_bfloat16*>(o);
+  prm.init_states = p.need_states ? states : nullptr;
+  CUtensorMap to = tq;
+  if (sm100::Cfg<BK, D, DV>::TMA_STORE && !make_tmap_3d(&to, o, BH, N, DV, 16)) return LA2_ERR_CUDA;
+  LaunchTimer t(K_FWD_TC, st);
+  return launch_fwd_sm100<BK, D, DV, sm100::MODE_CAUSAL, false, true>(tq, tk, tv, to, prm, BH * p.C, st);
 }
 
 static la2_status check_decay_shape(int64_t B, int64_t H, int64_t N, int64_t d, int64_t dv,
@@ -1086,6 +1143,12 @@ static la2_status decay_impl(const void* q, const void* k, const void* v, const 
   const bool bf = dt == LA2_BF16;
   float* s_kv = p.need_states ? static_cast<float*>(workspace) : nullptr;
   float* s_u = p.need_states && is_bwd ? s_kv + (size_t)BH * p.C * nel : nullptr;
+  // The forward at the tensor-core shapes: the chunk kernels with the decayed
+  // form (chunk states decayed to their last row, their decayed prefix, then
+  // every chunk's block loop from it).
+  if (!is_bwd && bf && sm100_supports(d, dv, block, false))
+    return block == 64 ? decay_forward_tc<64>(q, k, v, o, lam, BH, H, N, s_kv, p, st)
+                       : decay_forward_tc<128>(q, k, v, o, lam, BH, H, N, s_kv, p, st);
   if (p.need_states) {
     // K^T V of each chunk decayed to its last row, then their decayed prefix
     s = bf ? run_chunk_states<__nv_bfloat16>(k, v, s_kv, BH, N, (int)d, (int)dv, p, st, (int)H, 1, 1, lam, 1)

@@ -248,6 +248,32 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                : "memory");
 }
 
+__device__ __forceinline__ void ld_shared_v4(uint32_t addr, uint32_t& a, uint32_t& b, uint32_t& c,
+                                             uint32_t& d) {
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(a), "=r"(b), "=r"(c), "=r"(d)
+               : "r"(addr)
+               : "memory");
+}
+
+// Multiplies row r of a [ROWS x 128] bf16 operand tile (two 64-column panels
+// of ROWS 128-byte rows, 128B-swizzled as TMA writes them) by f, in place.
+template <int ROWS>
+__device__ __forceinline__ void scale_tile_row(uint32_t base, int r, float f) {
+#pragma unroll
+  for (int ch = 0; ch < 16; ++ch) {
+    const int panel = ch >> 3, cj = ch & 7;
+    const uint32_t addr = base + panel * ROWS * 128 + r * 128 + ((cj ^ (r & 7)) << 4);
+    uint32_t x[4];
+    ld_shared_v4(addr, x[0], x[1], x[2], x[3]);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162*>(&x[e]);
+      x[e] = pack_bf16x2(__low2float(h) * f, __high2float(h) * f);
+    }
+    st_shared_v4(addr, x[0], x[1], x[2], x[3]);
+  }
+}
+
 // ------------------------------------------------------ operand descriptors
 //
 // Shared-memory matrix descriptor (tcgen05): start address, leading and stride
@@ -356,6 +382,12 @@ struct Params {
   // MODE_CAUSAL: every chunk, the first included, starts from its slot of
   // init_states (a sequence part whose earlier parts are summarised there).
   int32_t init_all;
+  // Decayed form (kernels built with DEC): one rate per query head, lam[bh % H].
+  const float* lam;
+  // DEC, MODE_CAUSAL: init_states hold the sequence's raw chunk states (each
+  // decayed to its chunk's last row, no scan ran); chunk c adds the first c of
+  // them, state c' weighted by lam^(L (c-1-c')).
+  int32_t decay_sum;
 };
 
 // Shared state of one CTA.
@@ -443,13 +475,23 @@ __device__ __forceinline__ int acc_row(int w4, int t) {
 // product P K gives the intra-block part of dQ, the state update is
 // KV += K^T V from the swapped slots, and the inter-block part is dO KV^T
 // (the bf16 snapshot read K-major).
-template <int BK, int D, int DV, int MODE, bool DQ = false>
+// DEC = true (MODE_STATE, MODE_CAUSAL forward) is the decayed form with rate
+// lam = prm.lam[bh % H]: KV_t = lam KV_{t-1} + k_t^T v_t. MODE_STATE scales the
+// K rows of its chunk by lam^(t1-1-s) (the chunk's state decayed to its last
+// row). MODE_CAUSAL keeps KV decayed to the row before the block and, per block:
+// the mask warpgroup weights S by lam^(t-j) and then, in shared memory, scales
+// Q's rows by lam^(t+1) and K's by lam^(Bk-1-j) (S has read them unscaled);
+// the MMA warp issues Q KV and the update only after that; the state warpgroup
+// writes lam^Bk KV back to TMEM beside each snapshot, so the update adds onto
+// the decayed state.
+template <int BK, int D, int DV, int MODE, bool DQ = false, bool DEC = false>
 __global__ void __launch_bounds__(kThreads, 1)
 la2_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v,
                      const __grid_constant__ CUtensorMap tm_o, const Params prm) {
   using CF = Cfg<BK, D, DV>;
+  static_assert(!DEC || (!DQ && MODE != MODE_NONCAUSAL), "decayed form: forward, causal");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -492,6 +534,7 @@ la2_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                         (MODE == MODE_CAUSAL && prm.init_states && (c > 0 || prm.init_all));
   const float* init = nullptr;
   if (MODE == MODE_NONCAUSAL) init = prm.init_states + bkv * prm.C * (int64_t)(D * DV);
+  else if (DEC && prm.decay_sum && has_init) init = prm.init_states + bkv * prm.C * (int64_t)(D * DV);
   else if (has_init) init = prm.init_states + (bkv * prm.C + c) * (int64_t)(D * DV);
 
   // ---- setup
@@ -593,10 +636,12 @@ la2_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         const uint32_t va = smem_u32(sV + ks * CF::VTILE);
         if constexpr (MODE == MODE_STATE) {
           if (!wait_w(&b.kv_full[ks], (i / CF::KS) & 1, 10)) { ok = false; break; }
+          if (DEC && !wait_w(b.p_full, i & 1, 17)) { ok = false; break; }  // K rows scaled
           tc_fence_after();
           for (int kk = 0; kk < BK / 16; ++kk)
             mma_bf16_ss_warp(tKV, make_desc(ka + kk * 2048, BK * 128, 1024),
                         make_desc(va + kk * 2048, BK * 128, 1024), CF::ID_UPD, (i > 0 || kk > 0));
+          if (DEC) mma_commit_warp(b.p_empty);
           mma_commit_warp(&b.kv_empty[ks]);
           continue;
         }
@@ -618,6 +663,8 @@ la2_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           }
           mma_commit_warp(&b.s_full[sb]);
         }
+        // Decayed form: P, and the scaled Q and K rows, before Q KV and the update
+        if (DEC && !wait_w(b.p_full, i & 1, 18)) { ok = false; break; }
         // O_i = Q_i * bf16(KV)
         const int ob = i & 1;
         const uint32_t tO = tmem + (ob ? CF::COL_O1 : CF::COL_O0);
@@ -653,7 +700,7 @@ la2_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                       (have_snap || kk > 0) ? 1u : 0u);
         mma_commit_warp(b.kv_updated);
         // O_i += P_i V_i
-        if (!wait_w(b.p_full, i & 1, 16)) { ok = false; break; }
+        if (!DEC && !wait_w(b.p_full, i & 1, 16)) { ok = false; break; }
         tc_fence_after();
         const uint32_t pa = smem_u32(sP);
         for (int kk = 0; kk < BK / 16; ++kk) {
@@ -672,6 +719,23 @@ la2_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
   } else if (wg == kWgMask) {
     // ================================================ mask + convert S -> P
+    const float lam = DEC ? prm.lam[bh % prm.H] : 1.f;
+    if (DEC && MODE == MODE_STATE) {
+      // Scale row r of each K tile by lam^(t1-1-s), s its row in the sequence.
+      const int r = threadIdx.x % 128;
+      for (int i = 0; i < nblk; ++i) {
+        const int ks = i % CF::KS;
+        if (!__all_sync(0xffffffffu, wait_bar(&b.kv_full[ks], (i / CF::KS) & 1, lim, b.abort_flag, 22))) break;
+        if (!__all_sync(0xffffffffu, wait_bar(b.p_empty, (i & 1) ^ 1, lim, b.abort_flag, 23))) break;
+        if (r < BK) {
+          const int64_t srow = t0 + static_cast<int64_t>(i) * BK + r;
+          const int64_t e = t1 - 1 - srow;  // rows past the chunk end are zero (past N)
+          scale_tile_row<BK>(smem_u32(sK + ks * CF::KTILE), r, e >= 0 ? powf(lam, static_cast<float>(e)) : 0.f);
+        }
+        fence_proxy_async();
+        mbar_arrive(b.p_full);
+      }
+    }
     if (MODE == MODE_CAUSAL) {
       const int t = lane;
       const int r = acc_row<BK>(w4, t);
@@ -690,6 +754,19 @@ la2_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           tmem_ld32(tS + c32 * 32, v);
           tmem_ld_wait();
           if (r >= 0) {
+            if constexpr (DEC) {
+              // D_B: column col gets lam^(r - col); walk down from the last
+              // kept column of this chunk, multiplying by lam (no division)
+              const int c0 = c32 * 32, hi = min(r, c0 + 31);
+              float wgt = hi >= c0 ? powf(lam, static_cast<float>(r - hi)) : 0.f;
+#pragma unroll
+              for (int jj = 31; jj >= 0; --jj) {
+                if (c0 + jj <= hi) {
+                  v[jj] = __float_as_uint(__uint_as_float(v[jj]) * wgt);
+                  wgt *= lam;
+                }
+              }
+            }
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {  // 16-byte chunks (8 columns) of row r
               uint32_t w[4];
@@ -705,6 +782,14 @@ la2_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
               const uint32_t addr = pbase + panel * BK * 128 + r * 128 + ((cj ^ (r & 7)) << 4);
               st_shared_v4(addr, w[0], w[1], w[2], w[3]);
             }
+          }
+        }
+        if constexpr (DEC) {
+          // S(i) has completed (s_full): its Q and K tiles can take their scales
+          if (r >= 0) {
+            scale_tile_row<BK>(smem_u32(sQ + (i % CF::QS) * CF::QTILE), r, powf(lam, static_cast<float>(r + 1)));
+            scale_tile_row<BK>(smem_u32(sK + (i % CF::KS) * CF::KTILE), r,
+                               powf(lam, static_cast<float>(BK - 1 - r)));
           }
         }
         tc_fence_before();
@@ -733,6 +818,9 @@ la2_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                      pack_bf16x2(vals[q4 * 8 + 6], vals[q4 * 8 + 7]));
       }
     };
+    // Decayed form: the state the next update adds onto is lam^Bk times the one
+    // the snapshot shows (every block of a chunk but its last has Bk rows).
+    const float decay_bk = DEC ? powf(prm.lam[bh % prm.H], static_cast<float>(BK)) : 1.f;
     if (MODE == MODE_STATE) {
       // Chunk state out: TMEM (fp32) -> HBM, column-chunk-major (state_f4).
       if (__all_sync(0xffffffffu, wait_bar(b.kv_updated, 0, lim, b.abort_flag, 30))) {
@@ -763,15 +851,20 @@ la2_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
             // Non-causal: the total is the sum of the sequence's first
             // init_count chunk states, added here in chunk order (a few chunk
             // states: no separate scan launch; many: scanned into slot 0).
-            const int64_t nsum = MODE == MODE_NONCAUSAL ? prm.init_count : 1;
+            const bool dsum = DEC && prm.decay_sum;
+            const int64_t nsum = MODE == MODE_NONCAUSAL ? prm.init_count : (dsum ? c : 1);
 #pragma unroll
             for (int j = 0; j < 32; ++j) vals[j] = 0.f;
             for (int64_t cc = 0; cc < nsum; ++cc) {
               const float4* src = reinterpret_cast<const float4*>(init + cc * (int64_t)(D * DV));
+              const float wc = dsum ? powf(prm.lam[bh % prm.H], static_cast<float>(prm.L * (c - 1 - cc))) : 1.f;
 #pragma unroll
               for (int q4 = 0; q4 < 8; ++q4) {
                 const float4 x = src[state_f4<D>(r, c32 * 8 + q4)];
-                vals[4 * q4] += x.x; vals[4 * q4 + 1] += x.y; vals[4 * q4 + 2] += x.z; vals[4 * q4 + 3] += x.w;
+                vals[4 * q4] = fmaf(wc, x.x, vals[4 * q4]);
+                vals[4 * q4 + 1] = fmaf(wc, x.y, vals[4 * q4 + 1]);
+                vals[4 * q4 + 2] = fmaf(wc, x.z, vals[4 * q4 + 2]);
+                vals[4 * q4 + 3] = fmaf(wc, x.w, vals[4 * q4 + 3]);
               }
             }
           } else {
@@ -779,7 +872,7 @@ la2_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
             for (int j = 0; j < 32; ++j) vals[j] = 0.f;
           }
 #pragma unroll
-          for (int j = 0; j < 32; ++j) u[j] = __float_as_uint(vals[j]);
+          for (int j = 0; j < 32; ++j) u[j] = __float_as_uint(DEC ? decay_bk * vals[j] : vals[j]);
           if (MODE == MODE_CAUSAL) tmem_st32(tKV + c32 * 32, u);
           if (r >= 0) write_snap_row(vals, c32 * 32);
         }
@@ -803,7 +896,13 @@ la2_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
               for (int j = 0; j < 32; ++j) vals[j] = __uint_as_float(v[j]);
               write_snap_row(vals, c32 * 32);
             }
+            if constexpr (DEC) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(decay_bk * __uint_as_float(v[j]));
+              tmem_st32(tKV + c32 * 32, v);
+            }
           }
+          if (DEC) tmem_st_wait();
           fence_proxy_async();
           tc_fence_before();
           mbar_arrive(b.snap_full);
@@ -955,12 +1054,12 @@ inline bool make_tmap_3d(CUtensorMap* m, const void* base, int64_t BH, int64_t N
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BK, int D, int DV, int MODE, bool DQ = false>
+template <int BK, int D, int DV, int MODE, bool DQ = false, bool DEC = false>
 inline la2_status launch_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk,
                                    const CUtensorMap& tv, const CUtensorMap& to,
                                    const sm100::Params& p, int64_t units, cudaStream_t st) {
   using CF = sm100::Cfg<BK, D, DV>;
-  auto kern = sm100::la2_fwd_sm100_kernel<BK, D, DV, MODE, DQ>;
+  auto kern = sm100::la2_fwd_sm100_kernel<BK, D, DV, MODE, DQ, DEC>;
   static bool attr_done[128];  // one per template instantiation
   if (!smem_attribute_set(kern, CF::SMEM, attr_done)) return LA2_ERR_CUDA;
   if (launch_pdl(kern, dim3(static_cast<unsigned>(units)), dim3(sm100::kThreads), CF::SMEM, st, tq,

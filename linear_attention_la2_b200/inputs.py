@@ -55,6 +55,21 @@ WORKLOADS = {
                                       backward=True),
 }
 
+# Follow-on rows measured beside the five: grouped K/V heads (NEXT-3; ``Hkv`` K/V
+# heads, query head h reads K/V head h // (H // Hkv)) and the decayed form (NEXT-4;
+# one rate for every head), at the shapes of the B4 H16 N2K and B2 H32 N8K
+# workloads (same seeds; K and V keep their first Hkv heads).
+EXTRA_WORKLOADS = {
+    "bf16_gqa_b4h16kv4_n2k": Workload("bf16_gqa_b4h16kv4_n2k", 4, 16, 2048, 128, 128, 64, "bf16", 1,
+                                      extra={"Hkv": 4}),
+    "bf16_gqa_fwdbwd_b2h32kv8_n8k": Workload("bf16_gqa_fwdbwd_b2h32kv8_n8k", 2, 32, 8192, 128, 128,
+                                             64, "bf16", 4, backward=True, extra={"Hkv": 8}),
+    "bf16_decay_b4h16_n2k": Workload("bf16_decay_b4h16_n2k", 4, 16, 2048, 128, 128, 64, "bf16", 1,
+                                     extra={"decay": 0.99}),
+    "bf16_decay_fwdbwd_b4h16_n2k": Workload("bf16_decay_fwdbwd_b4h16_n2k", 4, 16, 2048, 128, 128, 64,
+                                            "bf16", 1, backward=True, extra={"decay": 0.99}),
+}
+
 SWEEP_N = (1024, 4096, 16384, 65536)
 SWEEP_BLOCKS = (64, 128)
 

@@ -63,7 +63,7 @@ CASES = [
     ("f32", 2, 3, 777, 64, 64, 64, 128, [0.99, 0.7, 1.0]),     # several chunks, ragged tail
     ("f32", 1, 1, 300, 16, 24, 16, 64, [0.0]),                 # lam = 0: the diagonal only
     ("f32", 1, 2, 513, 64, 32, 64, 0, [1.0, 1.0]),             # lam = 1: the plain op
-    ("bf16", 1, 2, 1000, 128, 128, 64, 0, [0.995, 0.9]),       # tensor-core shape, CUDA cores
+    ("bf16", 1, 2, 1000, 128, 128, 64, 0, [0.995, 0.9]),       # tensor-core forward, CUDA-core backward
     ("bf16", 2, 2, 4096, 64, 64, 64, 512, [0.999, 0.98]),      # eight chunks a sequence
     ("bf16", 1, 3, 650, 128, 64, 64, 256, [0.5, 0.97, 1.0]),
 ]
@@ -87,12 +87,20 @@ def test_decay_forward_backward(la2, case):
         assert rel(o[:, :, r], ref[:, :, r]) <= 4 * TOL[dt]
 
 
-def test_decay_forward_bf16_block128(la2):
-    """Block 128 at d = dv = 128: the forward fits the CUDA-core path."""
-    lam = [0.99, 0.8]
-    ins = la2_inputs.make_custom(1, 2, 700, 128, 128, "bf16", seed=7)
-    o = run(la2, ins, lam, 128)
-    assert rel(o, oracle.forward_decay(ins["q"], ins["k"], ins["v"], lam)) <= TOL["bf16"]
+@pytest.mark.parametrize("block,chunk,lam", [(128, 0, [0.99, 0.8]), (128, 512, [0.0, 0.999]),
+                                             (64, 256, [0.5, 1.0]), (64, 0, [0.97, 0.9])])
+def test_decay_forward_tensor_cores(la2, block, chunk, lam):
+    """bf16 d = dv = 128: the decayed forward on the tensor-core chunk kernels
+    (decayed chunk states, their decayed prefix, scaled Q and K rows, the
+    state decayed in TMEM), one and several chunks, lam = 0 and 1."""
+    B, H, N = 2, 2, 3000
+    ins = la2_inputs.make_custom(B, H, N, 128, 128, "bf16", seed=block + chunk)
+    o = run(la2, ins, lam, block, chunk)
+    ref = oracle.forward_decay(ins["q"], ins["k"], ins["v"], lam)
+    assert rel(o, ref) <= TOL["bf16"]
+    step = chunk if chunk else block
+    for r in sorted({r for s in range(0, N, step) for r in (max(0, s - 1), s)} | {N - 1}):
+        assert rel(o[:, :, r], ref[:, :, r]) <= 4 * TOL["bf16"]
 
 
 def test_decay_rates_are_per_head(la2):
