@@ -53,8 +53,9 @@ def parse():
                     help="0: the non-causal form O = Q (K^T V) of the same workload")
     ap.add_argument("--impl", default="la2", choices=["la2", "reference"])
     ap.add_argument("--sweep", action="store_true",
-                    help="also print one line per sequence-length sweep point, the 512K case and "
-                         "the decode step")
+                    help="also print one line per sequence-length sweep point, B4 H16 N2K, the 512K "
+                         "case, fwd+bwd, the grouped-head and decayed workloads, the non-causal form "
+                         "and the decode step")
     ap.add_argument("--decode", action="store_true",
                     help="also print the decode-step line (one RNN-mode token per sequence)")
     ap.add_argument("--no-e2e", action="store_true")
