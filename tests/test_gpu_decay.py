@@ -112,3 +112,14 @@ def test_decay_rates_are_per_head(la2):
     assert rel(o[:, 0], oracle.forward_decay(same["q"], same["k"], same["v"], [0.3, 0.95])[:, 0]) <= 1e-5
     assert rel(o[:, 1], oracle.forward_decay(same["q"], same["k"], same["v"], [0.3, 0.95])[:, 1]) <= 1e-5
     assert rel(o[:, 0], o[:, 1]) > 1e-2
+
+
+@pytest.mark.parametrize("N,block", [(1, 64), (63, 64), (65, 64), (130, 128), (1, 128), (257, 128)])
+def test_decay_forward_tensor_cores_edges(la2, N, block):
+    """The tensor-core decayed forward on one token, fewer rows than a block, a
+    block plus a row and ragged tails (rows past N are zero in the tiles; the
+    scaled Q and K rows there stay zero)."""
+    lam = [0.9, 0.6]
+    ins = la2_inputs.make_custom(1, 2, N, 128, 128, "bf16", seed=N + block)
+    o = run(la2, ins, lam, block)
+    assert rel(o, oracle.forward_decay(ins["q"], ins["k"], ins["v"], lam)) <= TOL["bf16"]
