@@ -344,7 +344,7 @@ def run_reference(args):
 def config_of(w, causal=True):
     kind = "causal" if causal else "non-causal"
     if "decay" in w.extra:
-        kind = f"decayed causal (lambda={w.extra['decay']} every head, CUDA cores)"
+        kind = f"decayed causal (lambda={w.extra['decay']} every head)"
     heads = f"H={w.H} Hkv={w.extra['Hkv']}" if "Hkv" in w.extra else f"H={w.H}"
     c = {"workload": f"{w.name}: {kind} forward B={w.B} {heads} "
                      f"N={w.N} d={w.d} dv={w.dv} block={w.block} {w.dtype}", "B": w.B, "H": w.H,

@@ -183,12 +183,15 @@ LA2_API la2_status la2_backward_sp(const void *q, const void *k, const void *v, 
  * device memory, 4-byte aligned, read only (powers are taken with powf; rates
  * outside [0, 1] are not rejected and follow the same formula). One K/V head per
  * query head; q, k, v, o, dout, dq, dk, dvv as for la2_forward / la2_backward
- * (causal only). The forward runs on tensor cores at bf16 d = dv = 128 (the
- * chunk kernels with decayed chunk states), on CUDA cores for every other shape
- * and dtype la2_forward takes; the backward runs on CUDA cores, with the
- * shared-memory limits of that path: bf16 d = dv = 128 at block 128 does not fit
- * the backward (LA2_ERR_UNSUPPORTED). Workspace:
- * la2_workspace_size_decay. Other conventions and errors as for la2_forward /
+ * (causal only). At bf16 d = dv = 128 (block 64 or 128) both directions run
+ * on tensor cores: the forward as the chunk kernels with decayed chunk states;
+ * the backward as three such forwards, dQ from (dO, V, K) and dK, dV from
+ * time-reversed copies of q, k, v, dout kept in the workspace (B*H*N at most
+ * 2^31 - 1, else LA2_ERR_UNSUPPORTED). Every other shape and dtype la2_forward
+ * takes runs on CUDA cores, with the shared-memory limits of that path (f32
+ * d = dv = 128 at block 128 does not fit the backward: LA2_ERR_UNSUPPORTED).
+ * Workspace: la2_workspace_size_decay; it must not overlap the inputs, the
+ * outputs or `lambda`. Other conventions and errors as for la2_forward /
  * la2_backward; `lambda` must not overlap the outputs.
  */
 LA2_API size_t la2_workspace_size_decay(int64_t B, int64_t H, int64_t N, int64_t d, int64_t dv,

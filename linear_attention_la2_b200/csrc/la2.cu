@@ -37,6 +37,7 @@ enum KernelId : int {
   K_BWD_DKDV_TC,
   K_DECODE,
   K_STATE_ACC,
+  K_REVERSE,
   K_COUNT
 };
 
@@ -44,7 +45,7 @@ static const char* kKernelNames[K_COUNT] = {
     "la2_chunk_state_simt", "la2_chunk_scan",      "la2_fwd_simt",
     "la2_bwd_dq_simt",      "la2_bwd_dkdv_simt",   "la2_fwd_sm100",
     "la2_chunk_state_sm100", "la2_bwd_dq_sm100",   "la2_bwd_dkdv_sm100",
-    "la2_decode_step",      "la2_state_accumulate"};
+    "la2_decode_step",      "la2_state_accumulate", "la2_reverse_rows"};
 
 struct EventRecord {
   int kernel;
@@ -1007,14 +1008,85 @@ static la2_status backward_impl(const void* q, const void* k, const void* v, con
 
 // ------------------------------------------------------------------ decayed form
 
+// Time reversal of up to four [S, N, 16 * kRevVecs bytes] row-major tensors
+// (blockIdx.y picks the tensor): dst[s][N-1-t] = src[s][t]. With src == dst the
+// reversal is in place: a thread swaps rows t and N-1-t of one 16-byte column
+// for t < N/2 (the middle row of an odd N stays). Row index 32-bit: S * N
+// <= INT32_MAX (checked by the caller). Each thread moves kRevUnroll columns a
+// grid-stride step, all loads before the stores.
+constexpr int kRevVecs = 16;  // 256-byte rows: 128 bf16
+constexpr int kRevUnroll = 4;
+struct RevArgs {
+  const uint4* src[4];
+  uint4* dst[4];
+};
+
+__global__ void __launch_bounds__(256) reverse_rows_kernel(RevArgs a, uint32_t N, uint32_t S) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const uint4* src = a.src[blockIdx.y];  // may be dst itself: no __restrict__
+  uint4* dst = a.dst[blockIdx.y];
+  const bool in_place = static_cast<const void*>(src) == static_cast<const void*>(dst);
+  const uint32_t rows = in_place ? N / 2 : N;
+  const uint64_t total = static_cast<uint64_t>(S) * rows * kRevVecs;
+  const uint64_t step = static_cast<uint64_t>(gridDim.x) * blockDim.x;
+  for (uint64_t e0 = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e0 < total;
+       e0 += step * kRevUnroll) {
+    uint64_t i[kRevUnroll], j[kRevUnroll];
+    uint4 x[kRevUnroll], z[kRevUnroll];
+#pragma unroll
+    for (int u = 0; u < kRevUnroll; ++u) {
+      const uint64_t e = e0 + u * step;
+      if (e >= total) break;
+      const uint32_t r = static_cast<uint32_t>(e / kRevVecs), c = static_cast<uint32_t>(e % kRevVecs);
+      const uint32_t sq = r / rows, t = r - sq * rows;
+      const uint64_t base = static_cast<uint64_t>(sq) * N;
+      i[u] = (base + t) * kRevVecs + c;
+      j[u] = (base + (N - 1 - t)) * kRevVecs + c;
+      x[u] = src[i[u]];
+      if (in_place) z[u] = dst[j[u]];
+    }
+#pragma unroll
+    for (int u = 0; u < kRevUnroll; ++u) {
+      if (e0 + u * step >= total) break;
+      dst[j[u]] = x[u];
+      if (in_place) dst[i[u]] = z[u];
+    }
+  }
+}
+
+// Reverses n (<= 4) bf16 [S, N, 128] tensors (src[i] == dst[i]: in place).
+static la2_status reverse_rows(const void* const* src, void* const* dst, int n, int64_t S, int64_t N,
+                               int sms, cudaStream_t st) {
+  RevArgs a{};
+  for (int i = 0; i < n; ++i) {
+    a.src[i] = static_cast<const uint4*>(src[i]);
+    a.dst[i] = static_cast<uint4*>(dst[i]);
+  }
+  const int64_t per = S * N * kRevVecs, threads = 256;
+  const int64_t want = (per + threads * kRevUnroll - 1) / (threads * kRevUnroll);
+  const unsigned blocks = static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(want, 8LL * sms / n)));
+  LaunchTimer t(K_REVERSE, st);
+  if (launch_pdl(reverse_rows_kernel, dim3(blocks, static_cast<unsigned>(n)), dim3(threads), 0, st, a,
+                 static_cast<uint32_t>(N), static_cast<uint32_t>(S)) != cudaSuccess)
+    return LA2_ERR_CUDA;
+  return LA2_OK;
+}
+
+// The decayed form on tensor cores: bf16, d = dv = 128, block 64 or 128.
+static bool decay_tc(int64_t d, int64_t dv, int block, la2_dtype dt) {
+  return dt == LA2_BF16 && sm100_supports(d, dv, block, false);
+}
+
 // Plan of the decayed form: chunks of L rows, chunk states decayed to a chunk
 // edge and their decayed scan when a sequence has more than one chunk. The
 // chunk count is chosen by waves of SMs (one CTA per (b, h, chunk)): the
 // fewest waves times (chunk blocks + a fixed cost of 3 blocks), chunks of at
 // least four blocks (B4 H16 N2K: 2 chunks, 128 CTAs in one wave, where 5 ran
-// three waves).
+// three waves). The tensor-core backward keeps one set of chunk states (its
+// three passes run one after another) and the four time-reversed inputs.
 static Plan plan_decay(int64_t B, int64_t H, int64_t N, int64_t d, int64_t dv, int block,
-                       bool is_bwd, int sms) {
+                       bool is_bwd, bool tc, int sms) {
   Plan p;
   const int64_t BH = B * H, T = (N + block - 1) / block;
   int64_t L;
@@ -1037,7 +1109,11 @@ static Plan plan_decay(int64_t B, int64_t H, int64_t N, int64_t d, int64_t dv, i
   p.L = std::max<int64_t>(L, block);
   p.C = std::max<int64_t>(1, (N + p.L - 1) / p.L);
   p.need_states = p.C > 1;
-  p.ws_bytes = p.need_states ? (size_t)BH * p.C * d * dv * sizeof(float) * (is_bwd ? 2 : 1) : 0;
+  const size_t states = p.need_states ? (size_t)BH * p.C * d * dv * sizeof(float) : 0;
+  if (is_bwd && tc)
+    p.ws_bytes = states + 4 * (size_t)BH * N * d * sizeof(__nv_bfloat16);
+  else
+    p.ws_bytes = states * (is_bwd ? 2 : 1);
   return p;
 }
 
@@ -1086,10 +1162,44 @@ static la2_status decay_forward_tc(const void* q, const void* k, const void* v, 
   return launch_fwd_sm100<BK, D, DV, sm100::MODE_CAUSAL, false, true>(tq, tk, tv, to, prm, BH * p.C, st);
 }
 
+// Gradients of the decayed form from three decayed forwards (bf16, d = dv =
+// 128). dQ_t = sum_{s<=t} lam^(t-s) (dO_t . v_s) k_s is the forward with dO,
+// V, K in the places of Q, K, V. dK_s = sum_{t>=s} lam^(t-s) (dO_t . v_s) q_t
+// and dV_s = sum_{t>=s} lam^(t-s) (q_t . k_s) dO_t run over later rows: on
+// the time-reversed sequences (row t at N-1-t) they are the causal forwards
+// dK~ = F(V~, dO~, Q~) and dV~ = F(K~, Q~, dO~), written into dk / dvv and
+// reversed there in place. `rev`: room for the four reversed inputs.
+template <int BK>
+static la2_status decay_backward_tc(const void* q, const void* k, const void* v, const void* dout,
+                                    void* dq, void* dk, void* dvv, const float* lam, int64_t BH,
+                                    int64_t H, int64_t N, float* states, void* rev, const Plan& p,
+                                    int sms, cudaStream_t st) {
+  la2_status s = decay_forward_tc<BK>(dout, v, k, dq, lam, BH, H, N, states, p, st);
+  if (s != LA2_OK) return s;
+  const size_t n = (size_t)BH * N * 128;
+  __nv_bfloat16* qr = static_cast<__nv_bfloat16*>(rev);
+  __nv_bfloat16 *kr = qr + n, *vr = kr + n, *dor = vr + n;
+  const void* src[4] = {q, k, v, dout};
+  void* dst[4] = {qr, kr, vr, dor};
+  s = reverse_rows(src, dst, 4, BH, N, sms, st);
+  if (s != LA2_OK) return s;
+  s = decay_forward_tc<BK>(kr, qr, dor, dvv, lam, BH, H, N, states, p, st);
+  if (s != LA2_OK) return s;
+  s = decay_forward_tc<BK>(vr, dor, qr, dk, lam, BH, H, N, states, p, st);
+  if (s != LA2_OK) return s;
+  void* outs[2] = {dk, dvv};
+  s = reverse_rows(outs, outs, 2, BH, N, sms, st);
+  if (s != LA2_OK) return s;
+  return launch_status();
+}
+
 static la2_status check_decay_shape(int64_t B, int64_t H, int64_t N, int64_t d, int64_t dv,
                                     int block, la2_dtype dt, bool is_bwd) {
   const la2_status s = check_shape(B, H, N, d, dv, 1, block, dt, is_bwd);
   if (s != LA2_OK) return s;
+  // tensor cores both ways; the backward's time reversal indexes rows in 32 bits
+  if (decay_tc(d, dv, block, dt))
+    return is_bwd && double(B) * double(H) * double(N) > 2147483647.0 ? LA2_ERR_UNSUPPORTED : LA2_OK;
   const size_t es = dt == LA2_BF16 ? 2 : 4, lim = 227 * 1024;
   if (fwd_simt_smem((int)d, (int)dv, block, es, true) > lim) return LA2_ERR_UNSUPPORTED;
   if (is_bwd && (bwd_dq_simt_smem((int)d, (int)dv, block, es, true) > lim ||
@@ -1128,12 +1238,15 @@ static la2_status decay_impl(const void* q, const void* k, const void* v, const 
   }
   const int sms = device_sm_count();
   if (sms <= 0) return LA2_ERR_CUDA;
-  const Plan p = plan_decay(B, H, N, d, dv, block, is_bwd, sms);
+  const bool tc = decay_tc(d, dv, block, dt);
+  const Plan p = plan_decay(B, H, N, d, dv, block, is_bwd, tc, sms);
   if (p.ws_bytes > 0) {
     if (!workspace || workspace_bytes < p.ws_bytes) return LA2_ERR_WORKSPACE;
     if (!is_aligned(workspace, 256)) return LA2_ERR_INVALID_ARG;
     for (int i = 0; i < nout; ++i)
       if (overlaps(workspace, p.ws_bytes, outs[i], out_sz[i])) return LA2_ERR_INVALID_ARG;
+    for (int j = 0; j < 4; ++j)
+      if (overlaps(workspace, p.ws_bytes, ins[j], in_sz[j])) return LA2_ERR_INVALID_ARG;
     if (overlaps(workspace, p.ws_bytes, lam, nl)) return LA2_ERR_INVALID_ARG;
   }
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -1143,12 +1256,19 @@ static la2_status decay_impl(const void* q, const void* k, const void* v, const 
   const bool bf = dt == LA2_BF16;
   float* s_kv = p.need_states ? static_cast<float*>(workspace) : nullptr;
   float* s_u = p.need_states && is_bwd ? s_kv + (size_t)BH * p.C * nel : nullptr;
-  // The forward at the tensor-core shapes: the chunk kernels with the decayed
-  // form (chunk states decayed to their last row, their decayed prefix, then
-  // every chunk's block loop from it).
-  if (!is_bwd && bf && sm100_supports(d, dv, block, false))
+  // The tensor-core shapes: the chunk kernels with the decayed form (chunk
+  // states decayed to their last row, their decayed prefix, then every chunk's
+  // block loop from it); the backward as three such forwards.
+  if (tc && !is_bwd)
     return block == 64 ? decay_forward_tc<64>(q, k, v, o, lam, BH, H, N, s_kv, p, st)
                        : decay_forward_tc<128>(q, k, v, o, lam, BH, H, N, s_kv, p, st);
+  if (tc) {
+    const size_t states = p.need_states ? (size_t)BH * p.C * nel * sizeof(float) : 0;
+    void* rev = static_cast<char*>(workspace) + states;
+    return block == 64
+               ? decay_backward_tc<64>(q, k, v, dout, dq, dk, dvv, lam, BH, H, N, s_kv, rev, p, sms, st)
+               : decay_backward_tc<128>(q, k, v, dout, dq, dk, dvv, lam, BH, H, N, s_kv, rev, p, sms, st);
+  }
   if (p.need_states) {
     // K^T V of each chunk decayed to its last row, then their decayed prefix
     s = bf ? run_chunk_states<__nv_bfloat16>(k, v, s_kv, BH, N, (int)d, (int)dv, p, st, (int)H, 1, 1, lam, 1)
@@ -1183,7 +1303,7 @@ size_t la2_workspace_size_decay(int64_t B, int64_t H, int64_t N, int64_t d, int6
   if (B == 0 || H == 0 || N == 0) return 0;
   const int sms = device_sm_count();
   if (sms <= 0) return (size_t)-1;
-  return plan_decay(B, H, N, d, dv, block, is_backward != 0, sms).ws_bytes;
+  return plan_decay(B, H, N, d, dv, block, is_backward != 0, decay_tc(d, dv, block, dt), sms).ws_bytes;
 }
 
 la2_status la2_forward_decay(const void* q, const void* k, const void* v, void* o, const float* lambda,

@@ -63,9 +63,12 @@ CASES = [
     ("f32", 2, 3, 777, 64, 64, 64, 128, [0.99, 0.7, 1.0]),     # several chunks, ragged tail
     ("f32", 1, 1, 300, 16, 24, 16, 64, [0.0]),                 # lam = 0: the diagonal only
     ("f32", 1, 2, 513, 64, 32, 64, 0, [1.0, 1.0]),             # lam = 1: the plain op
-    ("bf16", 1, 2, 1000, 128, 128, 64, 0, [0.995, 0.9]),       # tensor-core forward, CUDA-core backward
+    ("bf16", 1, 2, 1000, 128, 128, 64, 0, [0.995, 0.9]),       # tensor cores both ways
     ("bf16", 2, 2, 4096, 64, 64, 64, 512, [0.999, 0.98]),      # eight chunks a sequence
     ("bf16", 1, 3, 650, 128, 64, 64, 256, [0.5, 0.97, 1.0]),
+    ("bf16", 2, 2, 1537, 128, 128, 128, 0, [0.99, 0.7]),       # tensor cores, block 128, odd N
+    ("bf16", 1, 2, 3001, 128, 128, 128, 256, [0.999, 0.95]),   # twelve chunks: the decayed scan
+    ("bf16", 1, 2, 2100, 128, 128, 64, 512, [0.0, 1.0]),       # five chunks summed in the kernel
 ]
 
 
@@ -123,3 +126,39 @@ def test_decay_forward_tensor_cores_edges(la2, N, block):
     ins = la2_inputs.make_custom(1, 2, N, 128, 128, "bf16", seed=N + block)
     o = run(la2, ins, lam, block)
     assert rel(o, oracle.forward_decay(ins["q"], ins["k"], ins["v"], lam)) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("N,block", [(1, 64), (2, 128), (63, 64), (129, 128), (200, 64)])
+def test_decay_backward_tensor_cores_edges(la2, N, block):
+    """The tensor-core decayed backward (three decayed forwards, two of them on
+    the time-reversed rows) on one and two tokens, under a block, a block plus a
+    row and a ragged tail: the in-place reversal of dK and dV leaves an odd N's
+    middle row where it is."""
+    lam = [0.8, 0.97]
+    ins = la2_inputs.make_custom(1, 2, N, 128, 128, "bf16", seed=3 * N + block, with_grad_out=True)
+    _, (dq, dk, dv_) = run(la2, ins, lam, block, grad=True)
+    rq, rk, rv = oracle.backward_decay(ins["q"], ins["k"], ins["v"], ins["do"], lam)
+    assert rel(dq, rq) <= TOL["bf16"]
+    assert rel(dk, rk) <= TOL["bf16"]
+    assert rel(dv_, rv) <= TOL["bf16"]
+
+
+def test_decay_backward_runs_on_tensor_cores(la2):
+    """bf16 d = dv = 128: the backward launches the tensor-core chunk kernels and
+    the row reversal, and no CUDA-core attention kernel."""
+    ins = la2_inputs.make_custom(1, 2, 700, 128, 128, "bf16", seed=5, with_grad_out=True)
+    torch.cuda.synchronize()
+    assert la2.la2_profile_enable(1) == la2.LA2_OK
+    try:
+        run(la2, ins, [0.9, 0.99], 64, 256, grad=True)
+        torch.cuda.synchronize()
+        ran = {}
+        for kid in range(la2.la2_profile_num_kernels()):
+            n, _ = la2.la2_profile_collect(kid)
+            if n:
+                ran[la2.la2_profile_kernel_name(kid)] = n
+    finally:
+        la2.la2_profile_enable(0)
+    assert ran.get("la2_reverse_rows") == 2
+    assert ran.get("la2_fwd_sm100", 0) >= 4  # the forward, then dQ, dV, dK
+    assert not any(name.endswith("_simt") for name in ran), ran

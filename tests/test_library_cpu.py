@@ -252,12 +252,17 @@ def test_forward_decay_rejects_bad_arguments(kw, code):
 
 
 def test_backward_decay_limits():
-    """The decayed form runs on CUDA cores: bf16 d = dv = 128 fits the forward at
-    block 128 but not the backward's dK/dV tiles (documented in la2.h)."""
-    bf = la2.LA2_BF16
+    """bf16 d = dv = 128 runs both ways on tensor cores, at block 64 and 128 (the
+    shape passes; here only the missing tensors are refused). Off those shapes
+    the backward runs on CUDA cores with their shared-memory limits: f32 d = dv =
+    128 at block 128 does not fit the dK/dV tiles (documented in la2.h)."""
+    bf, f32 = la2.LA2_BF16, la2.LA2_F32
+    for block in (64, 128):
+        assert la2.la2_backward_decay(NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, 1, 1, 16, 128,
+                                      128, block, bf, NULL, 0, NULL) == la2.LA2_ERR_INVALID_ARG
     assert la2.la2_backward_decay(NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, 1, 1, 16, 128, 128,
-                                  128, bf, NULL, 0, NULL) == la2.LA2_ERR_UNSUPPORTED
-    assert la2.la2_workspace_size_decay(1, 1, 16, 128, 128, 128, bf, 1) == ctypes.c_size_t(-1).value
+                                  128, f32, NULL, 0, NULL) == la2.LA2_ERR_UNSUPPORTED
+    assert la2.la2_workspace_size_decay(1, 1, 16, 128, 128, 128, f32, 1) == ctypes.c_size_t(-1).value
     assert la2.la2_backward_decay(NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, 0, 1, 16, 128, 128,
                                   64, bf, NULL, 0, NULL) == la2.LA2_OK
     assert "la2_forward_decay" in la2.EXPORTED and "la2_backward_decay" in la2.EXPORTED
