@@ -342,7 +342,7 @@ struct Cfg {
   static constexpr int OTILE = BK * DV * 2;
   static constexpr int OFF_OST = OFF_SNAP + SNAP;
   static constexpr int OFF_BAR = OFF_OST + (TMA_STORE ? 2 * OTILE : 0);
-  static constexpr int NBAR = 2 * QS + 2 * KS + 16;
+  static constexpr int NBAR = 2 * QS + 2 * KS + 20;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;  // + alignment slack
   // TMEM columns
   static constexpr uint32_t COL_KV = 0;
@@ -405,6 +405,9 @@ struct Bars {
   uint64_t* o_full;      // [2]
   uint64_t* o_empty;     // [2]
   uint64_t* drain;
+  uint64_t* qk_ready;    // decayed form: Q and K rows of the block scaled
+  uint64_t* k_scaled;    // [2] decayed chunk state: K rows of block i scaled (slot i % 2)
+  uint64_t* k_free;      // [2] ... and the update that read them done
   uint32_t* tmem_base;
   volatile int* abort_flag;
 };
@@ -478,12 +481,12 @@ __device__ __forceinline__ int acc_row(int w4, int t) {
 // DEC = true (MODE_STATE, MODE_CAUSAL forward) is the decayed form with rate
 // lam = prm.lam[bh % H]: KV_t = lam KV_{t-1} + k_t^T v_t. MODE_STATE scales the
 // K rows of its chunk by lam^(t1-1-s) (the chunk's state decayed to its last
-// row). MODE_CAUSAL keeps KV decayed to the row before the block and, per block:
-// the mask warpgroup weights S by lam^(t-j) and then, in shared memory, scales
-// Q's rows by lam^(t+1) and K's by lam^(Bk-1-j) (S has read them unscaled);
-// the MMA warp issues Q KV and the update only after that; the state warpgroup
-// writes lam^Bk KV back to TMEM beside each snapshot, so the update adds onto
-// the decayed state.
+// row), one block ahead of the update MMA (k_scaled / k_free, two slots). MODE_CAUSAL keeps KV decayed to the row before the block and, per block:
+// once S has read Q and K unscaled, the mask warpgroup scales, in shared
+// memory, Q's rows by lam^(t+1) and K's by lam^(Bk-1-j) (qk_ready), then weights
+// S by lam^(t-j) into P; the MMA warp issues Q KV and the update on qk_ready,
+// while P is made, and P V on p_full; the state warpgroup writes lam^Bk KV back
+// to TMEM beside each snapshot, so the update adds onto the decayed state.
 template <int BK, int D, int DV, int MODE, bool DQ = false, bool DEC = false>
 __global__ void __launch_bounds__(kThreads, 1)
 la2_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -516,7 +519,10 @@ la2_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   b.o_full = b.kv_updated + 1;
   b.o_empty = b.o_full + 2;
   b.drain = b.o_empty + 2;
-  b.tmem_base = reinterpret_cast<uint32_t*>(b.drain + 1);
+  b.qk_ready = b.drain + 1;
+  b.k_scaled = b.qk_ready + 1;
+  b.k_free = b.k_scaled + 2;
+  b.tmem_base = reinterpret_cast<uint32_t*>(b.k_free + 2);
   b.abort_flag = reinterpret_cast<volatile int*>(b.tmem_base + 1);
 
   // ---- unit of work
@@ -552,6 +558,8 @@ la2_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     mbar_init(b.snap_full, 128);
     mbar_init(b.kv_updated, 1);
     mbar_init(b.drain, 1);
+    mbar_init(b.qk_ready, 128);
+    for (int s = 0; s < 2; ++s) { mbar_init(&b.k_scaled[s], 128); mbar_init(&b.k_free[s], 1); }
     *b.abort_flag = 0;
     fence_barrier_init();
   }
@@ -636,12 +644,12 @@ la2_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         const uint32_t va = smem_u32(sV + ks * CF::VTILE);
         if constexpr (MODE == MODE_STATE) {
           if (!wait_w(&b.kv_full[ks], (i / CF::KS) & 1, 10)) { ok = false; break; }
-          if (DEC && !wait_w(b.p_full, i & 1, 17)) { ok = false; break; }  // K rows scaled
+          if (DEC && !wait_w(&b.k_scaled[i & 1], (i >> 1) & 1, 17)) { ok = false; break; }  // K rows scaled
           tc_fence_after();
           for (int kk = 0; kk < BK / 16; ++kk)
             mma_bf16_ss_warp(tKV, make_desc(ka + kk * 2048, BK * 128, 1024),
                         make_desc(va + kk * 2048, BK * 128, 1024), CF::ID_UPD, (i > 0 || kk > 0));
-          if (DEC) mma_commit_warp(b.p_empty);
+          if (DEC) mma_commit_warp(&b.k_free[i & 1]);
           mma_commit_warp(&b.kv_empty[ks]);
           continue;
         }
@@ -663,8 +671,8 @@ la2_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           }
           mma_commit_warp(&b.s_full[sb]);
         }
-        // Decayed form: P, and the scaled Q and K rows, before Q KV and the update
-        if (DEC && !wait_w(b.p_full, i & 1, 18)) { ok = false; break; }
+        // Decayed form: the scaled Q and K rows before Q KV and the update
+        if (DEC && !wait_w(b.qk_ready, i & 1, 18)) { ok = false; break; }
         // O_i = Q_i * bf16(KV)
         const int ob = i & 1;
         const uint32_t tO = tmem + (ob ? CF::COL_O1 : CF::COL_O0);
@@ -700,7 +708,7 @@ la2_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                       (have_snap || kk > 0) ? 1u : 0u);
         mma_commit_warp(b.kv_updated);
         // O_i += P_i V_i
-        if (!DEC && !wait_w(b.p_full, i & 1, 16)) { ok = false; break; }
+        if (!wait_w(b.p_full, i & 1, 16)) { ok = false; break; }
         tc_fence_after();
         const uint32_t pa = smem_u32(sP);
         for (int kk = 0; kk < BK / 16; ++kk) {
@@ -722,18 +730,20 @@ la2_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     const float lam = DEC ? prm.lam[bh % prm.H] : 1.f;
     if (DEC && MODE == MODE_STATE) {
       // Scale row r of each K tile by lam^(t1-1-s), s its row in the sequence.
+      // Two hand-off slots: block i+1's rows are scaled while the update of
+      // block i runs (a slot is reused once the update two blocks back is done).
       const int r = threadIdx.x % 128;
       for (int i = 0; i < nblk; ++i) {
         const int ks = i % CF::KS;
         if (!__all_sync(0xffffffffu, wait_bar(&b.kv_full[ks], (i / CF::KS) & 1, lim, b.abort_flag, 22))) break;
-        if (!__all_sync(0xffffffffu, wait_bar(b.p_empty, (i & 1) ^ 1, lim, b.abort_flag, 23))) break;
+        if (!__all_sync(0xffffffffu, wait_bar(&b.k_free[i & 1], ((i >> 1) & 1) ^ 1, lim, b.abort_flag, 23))) break;
         if (r < BK) {
           const int64_t srow = t0 + static_cast<int64_t>(i) * BK + r;
           const int64_t e = t1 - 1 - srow;  // rows past the chunk end are zero (past N)
           scale_tile_row<BK>(smem_u32(sK + ks * CF::KTILE), r, e >= 0 ? powf(lam, static_cast<float>(e)) : 0.f);
         }
         fence_proxy_async();
-        mbar_arrive(b.p_full);
+        mbar_arrive(&b.k_scaled[i & 1]);
       }
     }
     if (MODE == MODE_CAUSAL) {
@@ -746,6 +756,17 @@ la2_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         const int s_use = CF::NSB == 2 ? (i >> 1) : i;
         const uint32_t tS = tmem + (sb ? CF::COL_S1 : CF::COL_S0) + lane_off;
         if (!__all_sync(0xffffffffu, wait_bar(&b.s_full[sb], s_use & 1, lim, b.abort_flag, 20))) break;
+        if constexpr (DEC) {
+          // S(i) has completed (s_full): its Q and K tiles can take their
+          // scales now, ahead of P (which waits for P V of the block before)
+          if (r >= 0) {
+            scale_tile_row<BK>(smem_u32(sQ + (i % CF::QS) * CF::QTILE), r, powf(lam, static_cast<float>(r + 1)));
+            scale_tile_row<BK>(smem_u32(sK + (i % CF::KS) * CF::KTILE), r,
+                               powf(lam, static_cast<float>(BK - 1 - r)));
+          }
+          fence_proxy_async();
+          mbar_arrive(b.qk_ready);
+        }
         if (!__all_sync(0xffffffffu, wait_bar(b.p_empty, (i & 1) ^ 1, lim, b.abort_flag, 21))) break;
         tc_fence_after();
 #pragma unroll
@@ -782,14 +803,6 @@ la2_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
               const uint32_t addr = pbase + panel * BK * 128 + r * 128 + ((cj ^ (r & 7)) << 4);
               st_shared_v4(addr, w[0], w[1], w[2], w[3]);
             }
-          }
-        }
-        if constexpr (DEC) {
-          // S(i) has completed (s_full): its Q and K tiles can take their scales
-          if (r >= 0) {
-            scale_tile_row<BK>(smem_u32(sQ + (i % CF::QS) * CF::QTILE), r, powf(lam, static_cast<float>(r + 1)));
-            scale_tile_row<BK>(smem_u32(sK + (i % CF::KS) * CF::KTILE), r,
-                               powf(lam, static_cast<float>(BK - 1 - r)));
           }
         }
         tc_fence_before();
