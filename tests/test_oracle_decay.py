@@ -138,3 +138,20 @@ def test_rejects_wrong_rate_count():
     q, k, v = _inputs(1, 2, 5, 2, 2, 81)
     with pytest.raises(ValueError):
         oracle.forward_decay(q, k, v, [0.5])
+
+
+@pytest.mark.parametrize("N,lams", [(1, [0.5]), (9, [0.0, 1.0]), (40, [0.7, 0.95])])
+def test_backward_as_forwards_on_reversed_rows(N, lams):
+    """The gradients are decayed forwards: dQ = F(dO, V, K), and with row t moved
+    to N-1-t (R), dV = R F(R K, R Q, R dO) and dK = R F(R V, R dO, R Q) (the
+    sums over later rows become sums over earlier ones with the same gaps). The
+    tensor-core backward is built on this identity; here both sides are the
+    oracle's own, independently written forward and backward."""
+    H = len(lams)
+    q, k, v = _inputs(1, H, N, 4, 3, 91)
+    do = _rand((1, H, N, 3), 95)
+    gq, gk, gv = oracle.backward_decay(q, k, v, do, lams)
+    rev = lambda x: x[:, :, ::-1]
+    assert oracle.relative_frobenius(oracle.forward_decay(do, v, k, lams), gq) <= 1e-12
+    assert oracle.relative_frobenius(rev(oracle.forward_decay(rev(k), rev(q), rev(do), lams)), gv) <= 1e-12
+    assert oracle.relative_frobenius(rev(oracle.forward_decay(rev(v), rev(do), rev(q), lams)), gk) <= 1e-12
