@@ -265,4 +265,12 @@ def test_backward_decay_limits():
     assert la2.la2_workspace_size_decay(1, 1, 16, 128, 128, 128, f32, 1) == ctypes.c_size_t(-1).value
     assert la2.la2_backward_decay(NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, 0, 1, 16, 128, 128,
                                   64, bf, NULL, 0, NULL) == la2.LA2_OK
+    # the tensor-core backward's row reversal indexes B*H*N rows in 32 bits; the
+    # forward has no such limit (there only the missing tensors are refused)
+    big = 2 ** 31
+    assert la2.la2_backward_decay(NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, 1, 1, big, 128, 128,
+                                  64, bf, NULL, 0, NULL) == la2.LA2_ERR_UNSUPPORTED
+    assert la2.la2_backward_decay(NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, 1, 1, big - 1, 128,
+                                  128, 64, bf, NULL, 0, NULL) == la2.LA2_ERR_INVALID_ARG
+    assert _fwd_decay(N=big, d=128, dv=128, dt=bf) == la2.LA2_ERR_INVALID_ARG
     assert "la2_forward_decay" in la2.EXPORTED and "la2_backward_decay" in la2.EXPORTED
